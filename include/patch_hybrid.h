@@ -1,0 +1,186 @@
+/*
+ * patch_hybrid.h - C ABI of the B200 (sm_100a) hybrid dense / 2:4 linear layer.
+ *
+ * The layer is PATCH's inference hot path: a frozen weight W[N,K] is cut into
+ * tiles, each tile either dense or 2:4 sparse (two kept in every group of four
+ * consecutive k), and the output is Y = X . (W (.) Mask)^T.
+ *   - Tiles dense or 2:4, global sparsity continuous in 0..50%: abstract of
+ *     "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs"; model card
+ *     "llama_3.2_1b-PATCH-45Sparse", method paragraph.
+ *   - The mask is a bit-packed keep/prune mask; applying it zeroes the pruned
+ *     weights: the same card, release paragraph and "How to use"
+ *     (apply_patch_mask).
+ *   - Tile shapes 128x128, 128x64, 64x128, 64x64: the same card,
+ *     "Training hyper-parameters" table, mask tile size row.
+ *   - A hybrid sparse kernel is what turns the mask into speed: the same
+ *     card, last sentence of "How to use".
+ *
+ * Conventions for every call:
+ *   - W, X, Y are bf16, row-major (K contiguous for W and X, N contiguous
+ *     for Y). "dev" pointers are CUDA device pointers on the current device;
+ *     "host" pointers are host memory (pinned is fastest).
+ *   - stream is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream. Calls are stream-ordered and asynchronous unless stated.
+ *   - No call throws, aborts or traps. Each returns a patch_status; the
+ *     message of the last failure on the calling thread is patch_last_error().
+ *   - The caller owns every buffer it passes. A handle owns only the packed
+ *     copy of the weights and its own tables.
+ *   - A handle is immutable after patch_pack: concurrent patch_linear calls on
+ *     one handle from several streams or threads are safe.
+ */
+#ifndef PATCH_HYBRID_H
+#define PATCH_HYBRID_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct patch_handle_s* patch_handle;
+
+typedef enum {
+    PATCH_OK = 0,
+    PATCH_ERR_ARG = 1,         /* null pointer, bad enum value, negative size */
+    PATCH_ERR_SHAPE = 2,       /* a dimension does not fit the tiling rules */
+    PATCH_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+    PATCH_ERR_MASK = 4,        /* a group inside a 2:4 tile does not keep exactly two */
+    PATCH_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    PATCH_ERR_TIMEOUT = 6,     /* a device-side wait ran past its limit */
+    PATCH_ERR_NOMEM = 7,       /* device or host allocation failed */
+    PATCH_ERR_UNSUPPORTED = 8  /* current device is not compute capability 10.x */
+} patch_status;
+
+/* Which kernel patch_linear_path runs. AUTO picks by M. */
+typedef enum {
+    PATCH_PATH_AUTO = 0,
+    PATCH_PATH_GEMM = 1,  /* tcgen05 tensor-core kernel (TMA, TMEM accumulators) */
+    PATCH_PATH_GEMV = 2   /* CUDA-core kernel for decode-sized M (M <= 16) */
+} patch_path;
+
+typedef struct {
+    int64_t N, K;               /* weight shape */
+    int32_t tile_rows, tile_cols;
+    int64_t tiles_total;        /* (N/tile_rows) * (K/tile_cols) */
+    int64_t tiles_sparse;       /* tiles flagged 2:4 */
+    int64_t slabs_total;        /* (N/128) * (K/64) storage slabs */
+    int64_t slabs_sparse;       /* slabs stored compressed */
+    int64_t packed_bytes;       /* device bytes of the packed weights */
+    int64_t pruned;             /* mask zeros over all N*K elements */
+    int64_t stray_zeros;        /* mask zeros inside tiles flagged dense */
+    double sparsity;            /* pruned / (N*K) */
+} patch_info_t;
+
+/*
+ * patch_pack - validate the mask and build the packed weights (one-time).
+ *
+ * Realises apply_patch_mask ("How to use" on the PATCH model cards) for one
+ * weight matrix, storing each dense tile as a bf16 block of W (.) Mask and
+ * each 2:4 tile as its kept values plus 2-bit position codes.
+ *
+ *   W_bf16      dev, N*K bf16, row-major, 16-byte aligned. Not retained.
+ *   N, K        weight rows (outputs) and columns (inputs). N % 128 == 0,
+ *               K % 64 == 0, N % tile_rows == 0, K % tile_cols == 0.
+ *   mask_bits   dev, ceil(N*K/8) bytes: bit (n*K + k) is the keep bit of
+ *               W[n][k]; it lives in byte (n*K+k)/8 at bit 7-((n*K+k)%8)
+ *               when bitorder == 0 (MSB first, numpy packbits default) or at
+ *               bit (n*K+k)%8 when bitorder == 1. Not retained.
+ *   tile_flags  host, (N/tile_rows)*(K/tile_cols) bytes, row-major over the
+ *               tile grid: 0 = dense tile, 1 = 2:4 tile. Not retained.
+ *   tile_rows, tile_cols  one of 128x128, 128x64, 64x128, 64x64.
+ *   stream      stream for the pack kernel.
+ *   out         receives the new handle (NULL on failure).
+ *
+ * Every group of four consecutive k inside a tile flagged 2:4 must keep
+ * exactly two weights, else PATCH_ERR_MASK (nothing is allocated on return).
+ * Pruned weights inside dense tiles are allowed and counted (stray_zeros).
+ * Synchronises the stream once to read the validation counters.
+ */
+patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t* mask_bits,
+                        int bitorder, const uint8_t* tile_flags, int tile_rows,
+                        int tile_cols, void* stream, patch_handle* out);
+
+/*
+ * patch_plan - the slab table and packed size patch_pack would produce for
+ * these tile flags, computed on the host without touching any device.
+ *
+ *   N, K, tile_flags, tile_rows, tile_cols  as for patch_pack.
+ *   table_host    host, (N/128)*(K/64) uint32 (layout as for
+ *                 patch_copy_packed), or NULL.
+ *   packed_bytes  receives the device bytes of the packed weights, or NULL.
+ * Same shape rules and errors as patch_pack; no mask is read.
+ */
+patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
+                        uint32_t* table_host, int64_t* packed_bytes);
+
+/*
+ * patch_linear - Y = X . (W (.) Mask)^T for the packed weights of h.
+ *
+ *   X_bf16  dev, M*K bf16 row-major, 16-byte aligned.
+ *   M       number of tokens (rows of X), M >= 0. M == 0 is a no-op.
+ *   Y_bf16  dev, M*N bf16 row-major, 16-byte aligned. Every element is
+ *           written: fp32 accumulation, one round-to-nearest-even to bf16.
+ * Picks the tensor-core kernel or the decode kernel by M. The first call for
+ * a new value of M builds and uploads that M's work schedule (allocates); do
+ * one such call before capturing later ones in a CUDA graph.
+ */
+patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
+                          void* stream);
+
+/* patch_linear with an explicit kernel choice (patch_path). GEMV requires
+ * M <= 16. */
+patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
+                               int path, void* stream);
+
+/*
+ * patch_linear_host - the same product from and to HOST memory.
+ *
+ *   X_host  host, M*K bf16 row-major.  Y_host  host, M*N bf16 row-major.
+ * Copies X to a device staging buffer owned by h (grown on demand), runs
+ * patch_linear on it, copies Y back, and synchronises the stream before it
+ * returns. Calls on one handle must not overlap (shared staging buffer).
+ */
+patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, void* Y_host,
+                               void* stream);
+
+/* patch_unpack - write W (.) Mask (N*K bf16, dev, row-major, 16-byte aligned)
+ * decoded from the packed weights. */
+patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream);
+
+/* patch_info - shape, tile and sparsity figures of a handle (host struct). */
+patch_status patch_info(patch_handle h, patch_info_t* info);
+
+/*
+ * patch_copy_packed - copy the packed bytes and the slab table to the host.
+ *   packed_host  host, packed_cap bytes (>= info.packed_bytes) or NULL.
+ *   table_host   host, table_cap uint32 (>= info.slabs_total) or NULL.
+ * Table entry per (strip s, slab b), index s*(K/64)+b:
+ *   (byte_offset/16) << 2 | has_metadata << 1 | sparse.
+ * Synchronous.
+ */
+patch_status patch_copy_packed(patch_handle h, void* packed_host, int64_t packed_cap,
+                               uint32_t* table_host, int64_t table_cap);
+
+/*
+ * patch_check - synchronise the stream and report device-side failures of
+ * earlier calls on h (a wait that ran past its limit gives PATCH_ERR_TIMEOUT).
+ * Clears the handle's device status word.
+ */
+patch_status patch_check(patch_handle h, void* stream);
+
+/* patch_free - release a handle and its device memory (synchronises the
+ * device first). NULL is ignored. */
+void patch_free(patch_handle h);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* patch_last_error(void);
+
+/* ABI version, bumped on any incompatible change. */
+int patch_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PATCH_HYBRID_H */

@@ -1,0 +1,291 @@
+"""Parity of the CUDA path with the CPU oracle, through the C ABI (needs a B200).
+
+Bar: the packed bytes and slab table are bit-exact; the product is within
+|err| <= 1e-2 * sum_k |x_k w_k| per element and relative Frobenius error
+<= 5e-3 of the oracle's fp32 result. Full-size workloads are checked on a
+seeded sample of token rows (rows of the product are independent, so the
+oracle computes exactly those rows), always including the first and last row.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_ELEM = 1e-2
+TOL_FRO = 5e-3
+
+
+@pytest.fixture(scope="module")
+def hsg():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import hybrid_sparse_gemm_b200 as m
+    return m
+
+
+def sample_rows(M, n=128, seed=0):
+    if M <= n:
+        return np.arange(M)
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(M, size=n - 2, replace=False).tolist()) | {0, M - 1}
+    return np.array(sorted(rows))
+
+
+def assert_close(Y, oracle_lib, X, W, bits, keep, rows=None, what=""):
+    Xc, Wc = X.cpu(), W.cpu()
+    Yo, _ = oracle_lib.linear(Xc, Wc, bits.cpu().numpy(), rows=rows)
+    Wm = oracle_lib.apply_mask(Wc, keep.cpu().numpy().astype(np.uint8))
+    S = oracle_lib.abs_scale(Xc, Wm, rows=rows)
+    Yg = Y.float().cpu().numpy()
+    if rows is not None:
+        Yg = Yg[rows]
+    assert np.isfinite(Yg).all(), f"{what}: non-finite output"
+    err = np.abs(Yg - Yo)
+    bad = err > TOL_ELEM * S
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside tolerance, "
+                           f"worst err {err[bad].max()} at scale {S[bad][np.argmax(err[bad])]}")
+    denom = np.linalg.norm(Yo)
+    if denom > 0:
+        fro = np.linalg.norm(Yg - Yo) / denom
+        assert fro <= TOL_FRO, f"{what}: relative Frobenius error {fro}"
+    else:
+        assert np.all(Yg == 0)
+
+
+def pack(hsg, p):
+    return hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu(), p.R, p.C, bitorder=p.bitorder)
+
+
+def check_pack(hsg, oracle_lib, p, lin):
+    packed, table = lin.packed()
+    keep = p.keep.cpu().numpy().astype(np.uint8)
+    op, ot = oracle_lib.pack(p.W.cpu(), keep, p.flags.cpu().numpy().reshape(-1), p.R, p.C)
+    assert np.array_equal(table.numpy().astype(np.uint32), ot)
+    assert packed.numel() == op.size
+    diff = np.flatnonzero(packed.numpy() != op)
+    assert diff.size == 0, f"{diff.size} packed bytes differ, first at {diff[:8]}"
+
+
+# ------------------------------------------------------------------ pack ---
+
+@pytest.mark.parametrize("R,C", [(128, 128), (128, 64), (64, 128), (64, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+@pytest.mark.parametrize("bitorder", [0, 1])
+def test_pack_bit_exact(hsg, oracle_lib, R, C, frac, bitorder):
+    N, K = 256, (448 if C == 64 else 384)
+    p = synth.make_problem(N, K, 0, R=R, C=C, frac=frac, seed=7, device="cuda", bitorder=bitorder)
+    lin = pack(hsg, p)
+    check_pack(hsg, oracle_lib, p, lin)
+    info = lin.info()
+    assert info.tiles_sparse == int(p.flags.sum())
+    assert info.pruned == int((~p.keep).sum())
+    assert info.stray_zeros == 0
+    Wm = lin.unpack()
+    torch.cuda.synchronize()
+    ref = oracle_lib.apply_mask(p.W.cpu(), p.keep.cpu().numpy().astype(np.uint8))
+    assert np.array_equal(Wm.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+    lin.free()
+
+
+def test_pack_rejects_bad_mask(hsg):
+    p = synth.make_problem(256, 256, 0, frac=1.0, seed=1, device="cuda")
+    keep = p.keep.clone()
+    keep[5, 8:12] = True  # four kept in one group of a 2:4 tile
+    bits = synth.pack_bits(keep)
+    with pytest.raises(hsg.PatchError) as e:
+        hsg.PackedLinear.pack(p.W, bits, p.flags.cpu())
+    assert e.value.status == 4
+
+
+def test_stray_zeros_in_dense_tiles(hsg, oracle_lib):
+    p = synth.make_problem(256, 256, 32, frac=0.5, seed=2, device="cuda")
+    keep = p.keep.clone()
+    fl = p.flags.cpu().numpy()
+    ti, tj = np.argwhere(fl == 0)[0]
+    keep[ti * 128 + 3, tj * 128 + 10] = False
+    keep[ti * 128 + 77, tj * 128 + 100] = False
+    bits = synth.pack_bits(keep)
+    lin = hsg.PackedLinear.pack(p.W, bits, p.flags.cpu())
+    assert lin.info().stray_zeros == 2
+    Y = lin(p.X, path=hsg.PATH_GEMM)
+    torch.cuda.synchronize()
+    assert_close(Y, oracle_lib, p.X, p.W, bits, keep, what="stray zeros")
+    lin.free()
+
+
+# --------------------------------------------------------------- product ---
+
+SMALL = [(256, 384, 128, 128), (384, 448, 128, 64), (256, 512, 64, 128), (384, 320, 64, 64)]
+
+
+@pytest.mark.parametrize("N,K,R,C", SMALL)
+@pytest.mark.parametrize("frac", [0.0, 0.6, 1.0])
+@pytest.mark.parametrize("M", [1, 5, 16, 17, 128, 129, 300])
+def test_gemm_small(hsg, oracle_lib, N, K, R, C, frac, M):
+    p = synth.make_problem(N, K, M, R=R, C=C, frac=frac, seed=M, device="cuda")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMM)
+    torch.cuda.synchronize()
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"gemm M={M}")
+    lin.free()
+
+
+@pytest.mark.parametrize("N,K,R,C", SMALL)
+@pytest.mark.parametrize("frac", [0.0, 0.6, 1.0])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 8, 12, 16])
+def test_gemv_small(hsg, oracle_lib, N, K, R, C, frac, M):
+    p = synth.make_problem(N, K, M, R=R, C=C, frac=frac, seed=M + 100, device="cuda")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMV)
+    torch.cuda.synchronize()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"gemv M={M}")
+    lin.free()
+
+
+def test_single_strip_single_slab(hsg, oracle_lib):
+    for frac in (0.0, 1.0):
+        p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")
+        lin = pack(hsg, p)
+        for path in (hsg.PATH_GEMM, hsg.PATH_GEMV):
+            Y = lin(p.X, path=path)
+            torch.cuda.synchronize()
+            assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"single slab {path}")
+        lin.free()
+
+
+def test_zero_weights_and_checkerboard(hsg, oracle_lib):
+    N, K = 256, 256
+    W = torch.zeros(N, K, dtype=torch.bfloat16, device="cuda")
+    fl = torch.from_numpy((np.indices((N // 64, K // 64)).sum(0) % 2).astype(np.uint8))
+    keep = synth.top2_keep(W, fl, 64, 64)  # ties -> lowest two positions kept
+    bits = synth.pack_bits(keep)
+    X = synth.normal_bf16((40, K), 1.0, "cuda", "zero", "X")
+    lin = hsg.PackedLinear.pack(W, bits, fl, 64, 64)
+    for path, M in ((hsg.PATH_GEMM, 40), (hsg.PATH_GEMV, 16)):
+        Y = lin(X[:M].contiguous(), path=path)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(Y.float()) == 0
+    lin.free()
+    # checkerboard with real weights
+    p = synth.make_problem(N, K, 33, R=64, C=64, seed=4, device="cuda")
+    keep = synth.top2_keep(p.W, fl, 64, 64)
+    bits = synth.pack_bits(keep)
+    lin = hsg.PackedLinear.pack(p.W, bits, fl, 64, 64)
+    assert lin.info().slabs_sparse == 0
+    Y = lin(p.X, path=hsg.PATH_GEMM)
+    torch.cuda.synchronize()
+    assert_close(Y, oracle_lib, p.X, p.W, bits, keep, what="checkerboard")
+    lin.free()
+
+
+def test_one_sparse_tile(hsg, oracle_lib):
+    p = synth.make_problem(512, 512, 50, R=128, C=128, n_sparse=1, seed=5, device="cuda")
+    lin = pack(hsg, p)
+    for path, M in ((hsg.PATH_GEMM, 50), (hsg.PATH_GEMV, 16)):
+        X = p.X[:M].contiguous()
+        Y = lin(X, path=path)
+        torch.cuda.synchronize()
+        assert_close(Y, oracle_lib, X, p.W, p.bits, p.keep, what=f"one sparse tile {path}")
+    lin.free()
+
+
+def test_empty_and_misaligned(hsg):
+    p = synth.make_problem(256, 256, 8, seed=6, device="cuda")
+    lin = pack(hsg, p)
+    Y = torch.full((0, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    lin(p.X[:0], out=Y)  # M = 0: nothing to do
+    buf = torch.zeros(8 * 256 + 8, dtype=torch.bfloat16, device="cuda")
+    Xmis = buf[1:1 + 8 * 256].view(8, 256)
+    with pytest.raises(hsg.PatchError) as e:
+        lin(Xmis)
+    assert e.value.status == 3
+    with pytest.raises(hsg.PatchError) as e:  # the decode kernel takes M <= 16
+        lin(torch.zeros(17, 256, dtype=torch.bfloat16, device="cuda"), path=hsg.PATH_GEMV)
+    assert e.value.status == 2
+    lin.free()
+
+
+def test_deterministic_and_host_path(hsg):
+    p = synth.make_problem(512, 1024, 300, R=128, C=64, frac=0.7, seed=8, device="cuda")
+    lin = pack(hsg, p)
+    Y1 = lin(p.X, path=hsg.PATH_GEMM)
+    Y2 = lin(p.X, path=hsg.PATH_GEMM)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    Yh = lin.host(p.X.cpu().pin_memory())
+    assert torch.equal(Yh, Y1.cpu())
+    Xs = p.X[:5].contiguous()
+    Yh5 = lin.host(Xs.cpu())
+    assert torch.equal(Yh5, lin(Xs).cpu())
+    lin.free()
+
+
+def test_gemm_and_gemv_agree_with_oracle_on_config_1(hsg, oracle_lib):
+    """512x512 layer, M = 16, a 4x4 grid of 128x128 tiles with 8 seeded 2:4 tiles."""
+    p = synth.make_problem(512, 512, 16, R=128, C=128, n_sparse=8, seed=0, device="cuda")
+    lin = pack(hsg, p)
+    check_pack(hsg, oracle_lib, p, lin)
+    assert abs(lin.info().sparsity - 0.25) < 1e-12
+    for path in (hsg.PATH_GEMM, hsg.PATH_GEMV, hsg.PATH_AUTO):
+        Y = lin(p.X, path=path)
+        torch.cuda.synchronize()
+        assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"config1 {path}")
+    lin.free()
+
+
+# ------------------------------------------------------ full-size workloads ---
+
+def _layer(hsg, oracle_lib, shapes, M, fracs, R=128, C=128, seed=0, tag="cfg", paths=None,
+           check_bytes=False, rows_n=128):
+    X_by_k = {}
+    for lin_shape, f in zip(shapes, fracs):
+        N, K = lin_shape.N, lin_shape.K
+        if K not in X_by_k:
+            X_by_k[K] = synth.normal_bf16((M, K), 1.0, "cuda", tag, "X", seed, M, K)
+        X = X_by_k[K]
+        T = (N // R) * (K // C)
+        p = synth.make_problem(N, K, 0, R=R, C=C, n_sparse=int(round(f * T)), seed=seed,
+                               device="cuda", tag=f"{tag}-{lin_shape.name}")
+        lin = pack(hsg, p)
+        if check_bytes:
+            check_pack(hsg, oracle_lib, p, lin)
+        rows = sample_rows(M, rows_n, seed)
+        for path in (paths or [hsg.PATH_AUTO]):
+            Y = lin(X, path=path)
+            torch.cuda.synchronize()
+            lin.check()
+            assert_close(Y, oracle_lib, X, p.W, p.bits, p.keep, rows=None if M <= rows_n else rows,
+                         what=f"{tag} {lin_shape.name} path {path}")
+        lin.free()
+        del p
+
+
+def test_config2_llama32_1b_m4096(hsg, oracle_lib):
+    shapes = synth.llama32_1b()
+    T = [(l.N // 128) * (l.K // 128) for l in shapes]
+    cnt = synth.split_fraction(T, 0.9, 0.8, 1.0, "cfg2")
+    _layer(hsg, oracle_lib, shapes, 4096, [c / t for c, t in zip(cnt, T)], tag="cfg2", check_bytes=True)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_config3_llama2_7b_decode(hsg, oracle_lib, M):
+    shapes = synth.llama2_7b()
+    _layer(hsg, oracle_lib, shapes, M, [0.7] * 7, tag="cfg3",
+           paths=[hsg.PATH_GEMV, hsg.PATH_GEMM], check_bytes=(M == 1))
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.5, 0.7, 0.9, 1.0])
+def test_config4_llama2_7b_prefill_sweep(hsg, oracle_lib, frac):
+    shapes = synth.llama2_7b()
+    _layer(hsg, oracle_lib, shapes, 2048, [frac] * 7, tag=f"cfg4-{frac}", rows_n=64)
+
+
+@pytest.mark.parametrize("R,C", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_config5_llama2_13b_tiles(hsg, oracle_lib, R, C):
+    shapes = [l for l in synth.llama2_13b() if l.name in ("q", "gate", "down")]
+    _layer(hsg, oracle_lib, shapes, 8192, [0.9] * 3, R=R, C=C, tag=f"cfg5-{R}x{C}", rows_n=64,
+           check_bytes=(R == 64 and C == 64))
