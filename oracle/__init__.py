@@ -56,12 +56,14 @@ def _load():
         lib.oracle_apply_mask.argtypes = [P, P, I64, I64, P]
         lib.oracle_linear_f32.argtypes = [P, I64, I64, P, I64, P, I64, P]
         lib.oracle_abs_scale.argtypes = [P, I64, P, I64, P, I64, P]
-        lib.oracle_pack_table.argtypes = [I64, I64, P, I, I, P]
+        lib.oracle_pack_table.argtypes = [I64, I64, P, I, I, P, P, P]
         lib.oracle_pack_table.restype = I64
-        lib.oracle_pack.argtypes = [P, P, I64, I64, P, I, I, P, P]
+        lib.oracle_pack.argtypes = [P, P, I64, I64, P, P, P, P]
         lib.oracle_pack.restype = I
-        lib.oracle_unpack.argtypes = [P, P, I64, I64, P]
+        lib.oracle_unpack.argtypes = [P, P, P, I64, I64, P]
         lib.oracle_unpack.restype = I
+        lib.oracle_unpack_gemm.argtypes = [P, P, P, I64, I64, P]
+        lib.oracle_unpack_gemm.restype = I
         _lib = lib
     return _lib
 
@@ -174,33 +176,46 @@ def linear(X, W, bits: np.ndarray, bitorder: int = 0, rows=None):
     return Y, round_bf16(Y)
 
 
+class Tables:
+    """The three uint32 tables of a packed weight (see oracle.c)."""
+
+    def __init__(self, slab, meta, gemm, nbytes):
+        self.slab, self.meta, self.gemm, self.nbytes = slab, meta, gemm, nbytes
+
+
+def pack_table(N: int, K: int, flags, R: int, C: int) -> Tables:
+    flags = np.ascontiguousarray(flags, dtype=np.uint8).reshape(-1)
+    KB = K // 64
+    KC = (KB + 1) // 2
+    slab = np.empty((N // 128) * KB, np.uint32)
+    meta = np.empty((N // 128) * KC, np.uint32)
+    gemm = np.empty((N // 128) * KB, np.uint32)
+    total = _load().oracle_pack_table(N, K, _p(flags), R, C, _p(slab), _p(meta), _p(gemm))
+    return Tables(slab, meta, gemm, int(total))
+
+
 def pack(W, keep: np.ndarray, flags: np.ndarray, R: int, C: int):
-    """Independent CPU pack: returns (packed bytes, slab table)."""
+    """Independent CPU pack: returns (packed bytes, Tables)."""
     Wu = _u16(W)
     N, K = Wu.shape
-    flags = np.ascontiguousarray(flags, dtype=np.uint8)
     keep = np.ascontiguousarray(keep, dtype=np.uint8)
-    table = np.empty((N // 128) * (K // 64), np.uint32)
-    total = _load().oracle_pack_table(N, K, _p(flags), R, C, _p(table))
-    out = np.zeros(total, np.uint8)
-    rc = _load().oracle_pack(_p(Wu), _p(keep), N, K, _p(flags), R, C, _p(table), _p(out))
+    t = pack_table(N, K, flags, R, C)
+    out = np.zeros(t.nbytes, np.uint8)
+    rc = _load().oracle_pack(_p(Wu), _p(keep), N, K, _p(t.slab), _p(t.meta), _p(t.gemm), _p(out))
     if rc != 0:
         raise ValueError("mask is not 2:4 inside a tile flagged 2:4")
-    return out, table
+    return out, t
 
 
-def pack_table(N: int, K: int, flags: np.ndarray, R: int, C: int):
-    flags = np.ascontiguousarray(flags, dtype=np.uint8)
-    table = np.empty((N // 128) * (K // 64), np.uint32)
-    total = _load().oracle_pack_table(N, K, _p(flags), R, C, _p(table))
-    return table, int(total)
-
-
-def unpack(packed: np.ndarray, table: np.ndarray, N: int, K: int) -> np.ndarray:
+def unpack(packed: np.ndarray, t: Tables, N: int, K: int, view: str = "slab") -> np.ndarray:
+    """Decode to W' from the per-strip records (view='slab') or from the
+    records the tensor-core table points at (view='gemm')."""
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
-    table = np.ascontiguousarray(table, dtype=np.uint32)
     Wm = np.empty((N, K), np.uint16)
-    rc = _load().oracle_unpack(_p(packed), _p(table), N, K, _p(Wm))
+    if view == "slab":
+        rc = _load().oracle_unpack(_p(packed), _p(t.slab), _p(t.meta), N, K, _p(Wm))
+    else:
+        rc = _load().oracle_unpack_gemm(_p(packed), _p(t.gemm), _p(t.meta), N, K, _p(Wm))
     if rc != 0:
         raise ValueError("invalid packed data")
     return Wm

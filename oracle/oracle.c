@@ -31,24 +31,32 @@
  *
  * The packed format is this library's own (the pages give none). Its
  * independent restatement here lets tests check the GPU pack byte by byte:
- *   - A "strip" is 128 consecutive rows of W; a "slab" is a strip times 64
- *     consecutive columns. Slabs are stored strip-major, K ascending.
+ *   - A "strip" is 128 consecutive rows of W, a "slab" a strip times 64
+ *     consecutive columns, a "chunk" two slabs (128 columns). Strips s and
+ *     s^1 are partners (the last strip of an odd count is its own partner).
  *   - A slab is sparse when every mask tile it overlaps is flagged 2:4,
- *     otherwise dense.
- *   - Dense slab: 16384 bytes, element (r, c) of W' (r < 128, c < 64) at
- *     byte r*128 + ((c/8) ^ (r%8))*16 + (c%8)*2.
- *   - Sparse slab values: 8192 bytes, the two kept bf16 of each group in
- *     ascending k; compressed element (r, j) (j < 32) at byte
+ *     otherwise dense; a slab is pair-sparse when it and its partner's slab
+ *     are both sparse.
+ *   - Region V, strip-major then slab: a dense slab is 16384 bytes, element
+ *     (r, c) of W' (r < 128, c < 64) at byte r*128 + ((c/8) ^ (r%8))*16 +
+ *     (c%8)*2; a sparse slab is 8192 bytes of the two kept bf16 of each
+ *     group in ascending k, compressed element (r, j) (j < 32) at byte
  *     r*64 + ((j/8) ^ ((r/2)%4))*16 + (j%8)*2.
- *   - Metadata: one 2048-byte block per (strip, 128-column chunk) that holds
- *     at least one sparse slab, stored right after the values of the first
- *     sparse slab in the chunk. The group that starts at chunk column k of
- *     row r has the 4-bit code i0 | i1<<2 (i0 < i1 the kept positions) in
- *     32-bit little-endian word (lane, k/32) at byte lane*16 + (k/32)*4, with
- *     lane = r%8 + 8*((k%32)/16) + 16*(r/16), at bit k%16 + 16*((r/8)%2).
- *     Codes of dense slabs in the chunk are zero.
- *   - Slab table: one uint32 per slab, (byte_offset/16)<<2 | has_meta<<1 |
- *     sparse.
+ *   - Region E, strip-major then chunk: one 2048-byte block per chunk that
+ *     holds a sparse slab. The group starting at chunk column k of row r has
+ *     the 4-bit code i0 | i1<<2 (i0 < i1 the kept positions) in the 32-bit
+ *     little-endian word at byte lane*16 + (k/32)*4, lane = r%8 +
+ *     8*((k%32)/16) + 16*(r/16), at bit k%16 + 16*((r/8)%2). Codes of dense
+ *     or absent slabs are zero.
+ *   - Region D, strip-major then slab: a 16384-byte dense image (layout of a
+ *     dense slab) of every sparse slab that is not pair-sparse.
+ *   - Tables (uint32): slab[s*KB+b] = (V offset/16)<<2 | first<<1 | sparse,
+ *     first marking the first sparse slab of its chunk;
+ *     meta[s*KC+c] = E offset/16 or 0xFFFFFFFF (KC = ceil(KB/2));
+ *     gemm[s*KB+b] = (offset/16)<<2 | load_meta<<1 | pair_sparse, where the
+ *     offset is the V record when the slab is pair-sparse or dense and the
+ *     D image otherwise, and load_meta marks the first pair-sparse slab of
+ *     its chunk.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -181,59 +189,95 @@ static int or_slab_sparse(const uint8_t* flags, int64_t K, int R, int C, int64_t
     return 1;
 }
 
-/* Fills table[S*KB] and returns the total packed byte count. */
+static int or_pair_sparse(const uint8_t* flags, int64_t N, int64_t K, int R, int C, int64_t s,
+                          int64_t b) {
+    int64_t S = N / OR_STRIP;
+    int64_t partner = ((s ^ 1) < S) ? (s ^ 1) : s;
+    return or_slab_sparse(flags, K, R, C, s, b) && or_slab_sparse(flags, K, R, C, partner, b);
+}
+
+/* Fills the three tables and returns the total packed byte count. */
 int64_t oracle_pack_table(int64_t N, int64_t K, const uint8_t* flags, int R, int C,
-                          uint32_t* table) {
-    int64_t S = N / OR_STRIP, KB = K / OR_SLAB, off = 0;
-    for (int64_t s = 0; s < S; ++s) {
-        int meta_done_chunk = -1;
+                          uint32_t* slab, uint32_t* meta, uint32_t* gemm) {
+    int64_t S = N / OR_STRIP, KB = K / OR_SLAB, KC = (KB + 1) / 2, off = 0;
+    /* region V */
+    for (int64_t s = 0; s < S; ++s)
         for (int64_t b = 0; b < KB; ++b) {
             int sp = or_slab_sparse(flags, K, R, C, s, b);
-            int has_meta = 0;
-            int64_t chunk = b / 2;
-            if (sp && meta_done_chunk != (int)chunk) {
-                has_meta = 1;
-                meta_done_chunk = (int)chunk;
+            int first = sp && (b % 2 == 0 || !or_slab_sparse(flags, K, R, C, s, b - 1));
+            slab[s * KB + b] = (uint32_t)((off / 16) << 2) | (uint32_t)(first << 1) | (uint32_t)sp;
+            off += sp ? 8192 : 16384;
+        }
+    /* region E */
+    for (int64_t s = 0; s < S; ++s)
+        for (int64_t c = 0; c < KC; ++c) {
+            int any = 0;
+            for (int64_t b = 2 * c; b < 2 * c + 2 && b < KB; ++b)
+                any |= or_slab_sparse(flags, K, R, C, s, b);
+            if (any) {
+                meta[s * KC + c] = (uint32_t)(off / 16);
+                off += 2048;
+            } else {
+                meta[s * KC + c] = 0xFFFFFFFFu;
             }
-            table[s * KB + b] = (uint32_t)((off / 16) << 2) | (uint32_t)(has_meta << 1) |
-                                (uint32_t)sp;
-            off += sp ? 8192 + (has_meta ? 2048 : 0) : 16384;
+        }
+    /* region D and the tensor-core table */
+    for (int64_t s = 0; s < S; ++s)
+        for (int64_t b = 0; b < KB; ++b) {
+            int sp = or_slab_sparse(flags, K, R, C, s, b);
+            int psp = or_pair_sparse(flags, N, K, R, C, s, b);
+            int64_t a_off;
+            if (sp && !psp) {
+                a_off = off;
+                off += 16384;
+            } else {
+                a_off = (int64_t)(slab[s * KB + b] >> 2) * 16;
+            }
+            int load_meta = psp && (b % 2 == 0 || !or_pair_sparse(flags, N, K, R, C, s, b - 1));
+            gemm[s * KB + b] = (uint32_t)((a_off / 16) << 2) | (uint32_t)(load_meta << 1) |
+                               (uint32_t)psp;
+        }
+    return off;
+}
+
+static void or_put16(uint8_t* p, uint16_t v) {
+    p[0] = (uint8_t)(v & 0xff);
+    p[1] = (uint8_t)(v >> 8);
+}
+
+static void or_dense_image(const uint16_t* W, const uint8_t* keep, int64_t K, int64_t s, int64_t b,
+                           uint8_t* base) {
+    int64_t k0 = b * OR_SLAB;
+    for (int r = 0; r < OR_STRIP; ++r) {
+        int64_t n = s * OR_STRIP + r;
+        for (int c = 0; c < OR_SLAB; ++c) {
+            uint16_t v = keep[n * K + k0 + c] ? W[n * K + k0 + c] : 0;
+            or_put16(base + (int64_t)r * 128 + (((c / 8) ^ (r % 8)) * 16) + (c % 8) * 2, v);
         }
     }
-    return off;
 }
 
 /* Writes the packed bytes. The mask must already be valid (every group of a
  * 2:4-flagged tile keeps exactly two); returns -1 otherwise. */
 int oracle_pack(const uint16_t* W, const uint8_t* keep, int64_t N, int64_t K,
-                const uint8_t* flags, int R, int C, const uint32_t* table, uint8_t* out) {
-    int64_t S = N / OR_STRIP, KB = K / OR_SLAB;
+                const uint32_t* slab, const uint32_t* meta, const uint32_t* gemm, uint8_t* out) {
+    int64_t S = N / OR_STRIP, KB = K / OR_SLAB, KC = (KB + 1) / 2;
+    for (int64_t s = 0; s < S; ++s)
+        for (int64_t c = 0; c < KC; ++c)
+            if (meta[s * KC + c] != 0xFFFFFFFFu) memset(out + (int64_t)meta[s * KC + c] * 16, 0, 2048);
     for (int64_t s = 0; s < S; ++s) {
-        uint8_t* meta = NULL;
-        int64_t meta_chunk = -1;
         for (int64_t b = 0; b < KB; ++b) {
-            uint32_t d = table[s * KB + b];
-            uint8_t* base = out + (int64_t)(d >> 2) * 16;
-            int sp = d & 1;
+            uint8_t* base = out + (int64_t)(slab[s * KB + b] >> 2) * 16;
             int64_t k0 = b * OR_SLAB;
-            if (!sp) {
-                for (int r = 0; r < OR_STRIP; ++r) {
-                    int64_t n = s * OR_STRIP + r;
-                    for (int c = 0; c < OR_SLAB; ++c) {
-                        uint16_t v = keep[n * K + k0 + c] ? W[n * K + k0 + c] : 0;
-                        int64_t at = (int64_t)r * 128 + (((c / 8) ^ (r % 8)) * 16) + (c % 8) * 2;
-                        base[at] = (uint8_t)(v & 0xff);
-                        base[at + 1] = (uint8_t)(v >> 8);
-                    }
-                }
+            if (!(slab[s * KB + b] & 1)) {
+                or_dense_image(W, keep, K, s, b, base);
                 continue;
             }
-            if (d & 2) {
-                meta = base + 8192;
-                meta_chunk = b / 2;
-                memset(meta, 0, 2048);
-            }
-            if (meta == NULL || meta_chunk != b / 2) return -1;
+            if (!(gemm[s * KB + b] & 1))
+                or_dense_image(W, keep, K, s, b, out + (int64_t)(gemm[s * KB + b] >> 2) * 16);
+            uint32_t mo = meta[s * KC + b / 2];
+            if (mo == 0xFFFFFFFFu) return -1;
+            uint8_t* mb = out + (int64_t)mo * 16;
             for (int r = 0; r < OR_STRIP; ++r) {
                 int64_t n = s * OR_STRIP + r;
                 for (int g = 0; g < OR_SLAB / 4; ++g) {
@@ -246,17 +290,14 @@ int oracle_pack(const uint16_t* W, const uint8_t* keep, int64_t N, int64_t K,
                     if (cnt != 2) return -1;
                     for (int t = 0; t < 2; ++t) {
                         int j = 2 * g + t;
-                        uint16_t v = W[n * K + k0 + 4 * g + idx[t]];
-                        int64_t at = (int64_t)r * 64 + (((j / 8) ^ ((r / 2) % 4)) * 16) + (j % 8) * 2;
-                        base[at] = (uint8_t)(v & 0xff);
-                        base[at + 1] = (uint8_t)(v >> 8);
+                        or_put16(base + (int64_t)r * 64 + (((j / 8) ^ ((r / 2) % 4)) * 16) + (j % 8) * 2,
+                                 W[n * K + k0 + 4 * g + idx[t]]);
                     }
                     int code = idx[0] | (idx[1] << 2);
                     int kc = (int)((b % 2) * OR_SLAB + 4 * g); /* column inside the chunk */
                     int lane = (r % 8) + 8 * ((kc % 32) / 16) + 16 * (r / 16);
-                    int word = kc / 32;
                     int bit = (kc % 16) + 16 * ((r / 8) % 2);
-                    uint8_t* wp = meta + lane * 16 + word * 4;
+                    uint8_t* wp = mb + lane * 16 + (kc / 32) * 4;
                     uint32_t wv = (uint32_t)wp[0] | ((uint32_t)wp[1] << 8) |
                                   ((uint32_t)wp[2] << 16) | ((uint32_t)wp[3] << 24);
                     wv |= (uint32_t)code << bit;
@@ -271,18 +312,16 @@ int oracle_pack(const uint16_t* W, const uint8_t* keep, int64_t N, int64_t K,
     return 0;
 }
 
-/* Decodes packed bytes back to W' (N x K bf16 bits). */
-int oracle_unpack(const uint8_t* packed, const uint32_t* table, int64_t N, int64_t K,
-                  uint16_t* Wm) {
-    int64_t S = N / OR_STRIP, KB = K / OR_SLAB;
+/* Decodes region V (with the metadata of region E) back to W' (N x K bf16
+ * bits). */
+int oracle_unpack(const uint8_t* packed, const uint32_t* slab, const uint32_t* meta, int64_t N,
+                  int64_t K, uint16_t* Wm) {
+    int64_t S = N / OR_STRIP, KB = K / OR_SLAB, KC = (KB + 1) / 2;
     for (int64_t s = 0; s < S; ++s) {
-        const uint8_t* meta = NULL;
-        int64_t meta_chunk = -1;
         for (int64_t b = 0; b < KB; ++b) {
-            uint32_t d = table[s * KB + b];
-            const uint8_t* base = packed + (int64_t)(d >> 2) * 16;
+            const uint8_t* base = packed + (int64_t)(slab[s * KB + b] >> 2) * 16;
             int64_t k0 = b * OR_SLAB;
-            if (!(d & 1)) {
+            if (!(slab[s * KB + b] & 1)) {
                 for (int r = 0; r < OR_STRIP; ++r)
                     for (int c = 0; c < OR_SLAB; ++c) {
                         int64_t at = (int64_t)r * 128 + (((c / 8) ^ (r % 8)) * 16) + (c % 8) * 2;
@@ -291,17 +330,15 @@ int oracle_unpack(const uint8_t* packed, const uint32_t* table, int64_t N, int64
                     }
                 continue;
             }
-            if (d & 2) {
-                meta = base + 8192;
-                meta_chunk = b / 2;
-            }
-            if (meta == NULL || meta_chunk != b / 2) return -1;
+            uint32_t mo = meta[s * KC + b / 2];
+            if (mo == 0xFFFFFFFFu) return -1;
+            const uint8_t* mb = packed + (int64_t)mo * 16;
             for (int r = 0; r < OR_STRIP; ++r) {
                 int64_t n = s * OR_STRIP + r;
                 for (int g = 0; g < OR_SLAB / 4; ++g) {
                     int kc = (int)((b % 2) * OR_SLAB + 4 * g);
                     int lane = (r % 8) + 8 * ((kc % 32) / 16) + 16 * (r / 16);
-                    const uint8_t* wp = meta + lane * 16 + (kc / 32) * 4;
+                    const uint8_t* wp = mb + lane * 16 + (kc / 32) * 4;
                     uint32_t wv = (uint32_t)wp[0] | ((uint32_t)wp[1] << 8) |
                                   ((uint32_t)wp[2] << 16) | ((uint32_t)wp[3] << 24);
                     int code = (int)((wv >> ((kc % 16) + 16 * ((r / 8) % 2))) & 0xf);
@@ -318,5 +355,26 @@ int oracle_unpack(const uint8_t* packed, const uint32_t* table, int64_t N, int64
             }
         }
     }
+    return 0;
+}
+
+/* Decodes the tensor-core view: for every slab, the record the gemm table
+ * points at, back to W' (checks that dense images equal W' too). */
+int oracle_unpack_gemm(const uint8_t* packed, const uint32_t* gemm, const uint32_t* meta,
+                       int64_t N, int64_t K, uint16_t* Wm) {
+    int64_t S = N / OR_STRIP, KB = K / OR_SLAB, KC = (KB + 1) / 2;
+    uint32_t* one = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)KB);
+    if (!one) return -1;
+    for (int64_t s = 0; s < S; ++s) {
+        for (int64_t b = 0; b < KB; ++b) one[b] = gemm[s * KB + b];
+        /* decode strip s as a one-strip matrix through oracle_unpack */
+        uint16_t* dst = Wm + s * OR_STRIP * K;
+        int rc = oracle_unpack(packed, one, meta + s * KC, OR_STRIP, K, dst);
+        if (rc != 0) {
+            free(one);
+            return rc;
+        }
+    }
+    free(one);
     return 0;
 }

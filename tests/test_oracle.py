@@ -230,50 +230,92 @@ VALID_CODES = {(0, 1): 0x4, (0, 2): 0x8, (0, 3): 0xC, (1, 2): 0x9, (1, 3): 0xD, 
 
 
 @pytest.mark.parametrize("R,C", [(128, 128), (128, 64), (64, 128), (64, 64)])
-def test_pack_roundtrip(oracle_lib, R, C):
-    N, K = 256, (448 if C == 64 else 384)  # K % 128 == 64 leaves a half chunk
-    p = synth.make_problem(N, K, 0, R=R, C=C, frac=0.6, seed=R + C)
+@pytest.mark.parametrize("N", [256, 384])
+def test_pack_roundtrip(oracle_lib, R, C, N):
+    K = 448 if C == 64 else 384  # K % 128 == 64 leaves a half chunk
+    p = synth.make_problem(N, K, 0, R=R, C=C, frac=0.6, seed=R + C + N)
     keep = p.keep.numpy().astype(np.uint8)
     flags = p.flags.numpy().reshape(-1)
-    packed, table = oracle_lib.pack(p.W, keep, flags, R, C)
+    packed, t = oracle_lib.pack(p.W, keep, flags, R, C)
     Wm = oracle_lib.apply_mask(p.W, keep)
-    assert np.array_equal(oracle_lib.unpack(packed, table, N, K), Wm)
-    # slab kinds: sparse iff all overlapped tiles are 2:4
+    # both views decode to W (.) Mask: the per-strip records and the records
+    # the tensor-core table points at (dense images of unpaired 2:4 slabs)
+    assert np.array_equal(oracle_lib.unpack(packed, t, N, K), Wm)
+    assert np.array_equal(oracle_lib.unpack(packed, t, N, K, view="gemm"), Wm)
     fl = p.flags.numpy()
-    KB = K // 64
-    for s in range(N // 128):
+    KB, S = K // 64, N // 128
+
+    def sparse(s, b):
+        rows = range(s * 128 // R, (s + 1) * 128 // R)
+        return all(fl[r, (b * 64) // C] for r in rows)
+
+    n_shadow = 0
+    for s in range(S):
+        partner = s ^ 1 if (s ^ 1) < S else s
         for b in range(KB):
-            rows = range(s * 128 // R, (s + 1) * 128 // R)
-            want = all(fl[r, (b * 64) // C] for r in rows)
-            assert int(table[s * KB + b] & 1) == int(want)
+            sp = sparse(s, b)
+            psp = sp and sparse(partner, b)
+            assert int(t.slab[s * KB + b] & 1) == int(sp)
+            first_sp = sp and (b % 2 == 0 or not sparse(s, b - 1))
+            assert int((t.slab[s * KB + b] >> 1) & 1) == int(first_sp)
+            assert int(t.gemm[s * KB + b] & 1) == int(psp)
+            assert int(t.gemm[partner * KB + b] & 1) == int(psp)  # symmetric in a pair
+            n_shadow += sp and not psp
+            if psp:
+                first = b % 2 == 0 or not (sparse(s, b - 1) and sparse(partner, b - 1))
+                assert int((t.gemm[s * KB + b] >> 1) & 1) == int(first)
+        for c in range((KB + 1) // 2):
+            has = any(sparse(s, b) for b in (2 * c, 2 * c + 1) if b < KB)
+            assert (t.meta[s * ((KB + 1) // 2) + c] != 0xFFFFFFFF) == has
+    n_sparse = int(sum((t.slab & 1)))
+    n_meta = int((t.meta != 0xFFFFFFFF).sum())
+    assert t.nbytes == (S * KB - n_sparse) * 16384 + n_sparse * 8192 + n_meta * 2048 + n_shadow * 16384
 
 
 def test_pack_metadata_codes_and_sizes(oracle_lib):
-    N, K = 128, 256
+    N, K = 256, 256
     W = synth.normal_bf16((N, K), 0.02, "cpu", "meta", "W")
     keep = np.zeros((N, K), np.uint8)
     for n in range(N):
         for g in range(K // 4):
             i0, i1 = PAIRS[(n + 5 * g) % 6]
             keep[n, 4 * g + i0] = keep[n, 4 * g + i1] = 1
-    flags = np.ones(2, np.uint8)
-    packed, table = oracle_lib.pack(W, keep, flags, 128, 128)
-    # 4 sparse slabs, two metadata blocks: 4*8192 + 2*2048 bytes
-    assert packed.size == 4 * 8192 + 2 * 2048
-    assert [int(t & 3) for t in table] == [3, 1, 3, 1]
+    flags = np.ones(4, np.uint8)
+    packed, t = oracle_lib.pack(W, keep, flags, 128, 128)
+    # 8 sparse slabs, 4 metadata blocks, no dense images
+    assert packed.size == 8 * 8192 + 4 * 2048
+    assert [int(x & 1) for x in t.slab] == [1] * 8
+    assert [int(x & 3) for x in t.gemm] == [3, 1, 3, 1, 3, 1, 3, 1]
     codes = []
-    for chunk in range(2):
-        meta = packed[int(table[2 * chunk] >> 2) * 16 + 8192:][:2048].view(np.uint32)
-        for w in meta:
+    for m in t.meta:
+        block = packed[int(m) * 16:][:2048].view(np.uint32)
+        for w in block:
             for sh in range(0, 32, 4):
                 codes.append((int(w) >> sh) & 0xF)
     assert sorted(set(codes)) == sorted(VALID_CODES.values())
     assert len(codes) == N * K // 4
-    counts = {c: codes.count(c) for c in VALID_CODES.values()}
-    assert sum(counts.values()) == N * K // 4
-    # every kept value appears in the compressed values, in ascending k per group
-    vals = np.concatenate([packed[int(table[b] >> 2) * 16:][:8192].view(np.uint16) for b in range(4)])
+    # every kept value appears in the compressed values
+    vals = np.concatenate([packed[int(x >> 2) * 16:][:8192].view(np.uint16) for x in t.slab])
     assert sorted(vals.tolist()) == sorted(bits_of(W)[keep.astype(bool)].tolist())
+
+
+def test_pair_rule_dense_images(oracle_lib):
+    """A 2:4 slab whose partner strip is dense gets a dense image for the
+    tensor-core view; the per-strip view stays compressed."""
+    N, K = 256, 128
+    p = synth.make_problem(N, K, 0, R=128, C=128, n_sparse=0, seed=0)
+    flags = np.array([1, 0], np.uint8)  # strip 0 2:4, strip 1 dense
+    keep = synth.top2_keep(p.W, torch.from_numpy(flags).view(2, 1), 128, 128).numpy().astype(np.uint8)
+    packed, t = oracle_lib.pack(p.W, keep, flags, 128, 128)
+    assert [int(x & 1) for x in t.slab] == [1, 1, 0, 0]
+    assert [int(x & 1) for x in t.gemm] == [0, 0, 0, 0]
+    assert packed.size == 2 * 8192 + 2048 + 2 * 16384 + 2 * 16384
+    Wm = oracle_lib.apply_mask(p.W, keep)
+    assert np.array_equal(oracle_lib.unpack(packed, t, N, K, view="gemm"), Wm)
+    # odd strip count: the last strip pairs with itself
+    p3 = synth.make_problem(384, 128, 0, R=128, C=128, frac=1.0, seed=1)
+    _, t3 = oracle_lib.pack(p3.W, p3.keep.numpy().astype(np.uint8), p3.flags.numpy().reshape(-1), 128, 128)
+    assert all(int(x & 1) for x in t3.gemm)
 
 
 def test_pack_rejects_bad_mask(oracle_lib):
