@@ -28,7 +28,7 @@ PATCH_OK = 0
 STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_ARG", 2: "PATCH_ERR_SHAPE", 3: "PATCH_ERR_ALIGN",
                 4: "PATCH_ERR_MASK", 5: "PATCH_ERR_CUDA", 6: "PATCH_ERR_TIMEOUT",
                 7: "PATCH_ERR_NOMEM", 8: "PATCH_ERR_UNSUPPORTED"}
-PATH_AUTO, PATH_GEMM, PATH_GEMV = 0, 1, 2
+PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR = 0, 1, 2, 3, 4
 
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
@@ -40,7 +40,8 @@ class patch_info_t(ctypes.Structure):
                 ("tile_rows", ctypes.c_int32), ("tile_cols", ctypes.c_int32),
                 ("tiles_total", ctypes.c_int64), ("tiles_sparse", ctypes.c_int64),
                 ("slabs_total", ctypes.c_int64), ("slabs_sparse", ctypes.c_int64),
-                ("packed_bytes", ctypes.c_int64), ("pruned", ctypes.c_int64),
+                ("slabs_pair_sparse", ctypes.c_int64), ("meta_blocks", ctypes.c_int64),
+                ("dense_images", ctypes.c_int64), ("packed_bytes", ctypes.c_int64), ("pruned", ctypes.c_int64),
                 ("stray_zeros", ctypes.c_int64), ("sparsity", ctypes.c_double)]
 
 
@@ -53,9 +54,9 @@ _lib.patch_linear_path.argtypes = [_P, _P, _I64, _P, _I, _P]
 _lib.patch_linear_host.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_unpack.argtypes = [_P, _P, _P]
 _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]
-_lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64]
+_lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
 _lib.patch_check.argtypes = [_P, _P]
-_lib.patch_plan.argtypes = [_I64, _I64, _P, _I, _I, _P, ctypes.POINTER(_I64)]
+_lib.patch_plan.argtypes = [_I64, _I64, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I64)]
 _lib.patch_free.argtypes = [_P]
 _lib.patch_free.restype = None
 _lib.patch_last_error.restype = ctypes.c_char_p
@@ -92,14 +93,22 @@ def version() -> int:
 
 # ---- thin functions with the C ABI's names -----------------------------------
 
+def _table_sizes(N: int, K: int):
+    S, KB = N // 128, K // 64
+    return S * KB, S * ((KB + 1) // 2), S * KB
+
+
 def patch_plan(N: int, K: int, tile_flags, tile_rows: int = 128, tile_cols: int = 128):
-    """Host-only: (slab table as int64 CPU tensor, packed byte count)."""
-    flags = torch.as_tensor(tile_flags, dtype=torch.uint8).reshape(-1).contiguous().cpu()
-    table = torch.empty((N // 128) * (K // 64) if N % 128 == 0 and K % 64 == 0 else 0, dtype=torch.int32)
+    """Host-only: ((slab, meta, gemm) tables as uint32 numpy arrays, packed byte count)."""
+    import numpy as np
+    flags = np.ascontiguousarray(np.asarray(tile_flags, dtype=np.uint8).reshape(-1))
+    ok = N > 0 and K > 0 and N % 128 == 0 and K % 64 == 0
+    ns, nm, ng = _table_sizes(N, K) if ok else (0, 0, 0)
+    slab, meta, gemm = (np.zeros(max(n, 1), np.uint32) for n in (ns, nm, ng))
     nbytes = _I64(0)
-    _check(_lib.patch_plan(N, K, flags.data_ptr(), tile_rows, tile_cols,
-                           table.data_ptr() if table.numel() else None, ctypes.byref(nbytes)))
-    return table.to(torch.int64) & 0xFFFFFFFF, int(nbytes.value)
+    _check(_lib.patch_plan(N, K, flags.ctypes.data, tile_rows, tile_cols, slab.ctypes.data,
+                           meta.ctypes.data, gemm.ctypes.data, ctypes.byref(nbytes)))
+    return (slab[:ns], meta[:nm], gemm[:ng]), int(nbytes.value)
 
 
 def patch_pack(W: torch.Tensor, mask_bits: torch.Tensor, tile_flags, tile_rows: int = 128,
@@ -141,12 +150,15 @@ def patch_info(h: int) -> patch_info_t:
 
 
 def patch_copy_packed(h: int):
-    """(packed bytes as uint8 CPU tensor, slab table as int64 CPU tensor)."""
+    """(packed bytes as a uint8 numpy array, (slab, meta, gemm) uint32 tables)."""
+    import numpy as np
     info = patch_info(h)
-    packed = torch.empty(int(info.packed_bytes), dtype=torch.uint8)
-    table = torch.empty(int(info.slabs_total), dtype=torch.int32)
-    _check(_lib.patch_copy_packed(h, packed.data_ptr(), packed.numel(), table.data_ptr(), table.numel()))
-    return packed, table.view(torch.int32).to(torch.int64) & 0xFFFFFFFF
+    ns, nm, ng = _table_sizes(int(info.N), int(info.K))
+    packed = np.empty(int(info.packed_bytes), np.uint8)
+    slab, meta, gemm = np.empty(ns, np.uint32), np.empty(nm, np.uint32), np.empty(ng, np.uint32)
+    _check(_lib.patch_copy_packed(h, packed.ctypes.data, packed.size, slab.ctypes.data, ns,
+                                  meta.ctypes.data, nm, gemm.ctypes.data, ng))
+    return packed, (slab, meta, gemm)
 
 
 def patch_check(h: int, stream=None):

@@ -1,5 +1,5 @@
 // Host runtime behind the C ABI in patch_hybrid.h: argument checks, the slab
-// table, the cost-balanced persistent schedule, tensor maps and launches.
+// tables, the cost-balanced persistent schedules, tensor maps and launches.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -17,6 +17,11 @@
 
 using namespace patch;
 
+namespace patch {
+cudaError_t gemm_prepare_single();
+cudaError_t gemm_prepare_pair(int* max_clusters);
+}  // namespace patch
+
 namespace {
 
 thread_local std::string g_err;
@@ -31,48 +36,71 @@ patch_status fail(patch_status st, const char* fmt, ...) {
     return st;
 }
 
+patch_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(PATCH_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define PATCH_CUDA(call)                                    \
+    do {                                                    \
+        cudaError_t e_ = (call);                            \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+    } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 patch_status check_shape(int64_t N, int64_t K, int tile_rows, int tile_cols) {
     const bool shape_ok = (tile_rows == 128 || tile_rows == 64) && (tile_cols == 128 || tile_cols == 64);
     if (!shape_ok)
         return fail(PATCH_ERR_SHAPE, "tile shape %dx%d is not one of 128x128, 128x64, 64x128, 64x64", tile_rows,
                     tile_cols);
     if (N <= 0 || K <= 0) return fail(PATCH_ERR_SHAPE, "N and K must be positive");
-    if (N % 128 || K % 64 || N % tile_rows || K % tile_cols)
+    if (N % kStrip || K % kSlabK || N % tile_rows || K % tile_cols)
         return fail(PATCH_ERR_SHAPE,
                     "need N %% 128 == 0, K %% 64 == 0 and both divisible by the tile (N=%lld K=%lld)",
                     (long long)N, (long long)K);
-    if (N > (1 << 24) || K > (1 << 24) || N * K > ((int64_t)1 << 36)) return fail(PATCH_ERR_SHAPE, "weight too large");
+    if (N > (1 << 24) || K > (1 << 24) || N * K > ((int64_t)1 << 36))
+        return fail(PATCH_ERR_SHAPE, "weight too large");
     return PATCH_OK;
 }
 
-patch_status cuda_fail(cudaError_t e, const char* what) {
-    return fail(PATCH_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+patch_status check_flags(const uint8_t* flags, int64_t n) {
+    for (int64_t i = 0; i < n; ++i)
+        if (flags[i] > 1) return fail(PATCH_ERR_ARG, "tile flag %lld is %d, must be 0 or 1", (long long)i, (int)flags[i]);
+    return PATCH_OK;
 }
 
-#define PATCH_CUDA(call)                                   \
-    do {                                                   \
-        cudaError_t e_ = (call);                           \
-        if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
-    } while (0)
+struct DeviceInfo {
+    int sms = 0;
+    int pair_clusters = 0;
+};
+std::mutex g_dev_mu;
+std::map<int, DeviceInfo> g_dev;
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-patch_status check_device(int* dev_out, int* sms_out) {
+patch_status prepare_device(int* dev_out, DeviceInfo* info_out) {
     int dev = 0;
     PATCH_CUDA(cudaGetDevice(&dev));
-    int major = 0, sms = 0;
-    PATCH_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
-    PATCH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    if (major != 10) return fail(PATCH_ERR_UNSUPPORTED, "device %d has compute capability %d.x, need 10.x", dev, major);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        int major = 0, sms = 0;
+        PATCH_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+        PATCH_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+        if (major != 10)
+            return fail(PATCH_ERR_UNSUPPORTED, "device %d has compute capability %d.x, need 10.x", dev, major);
+        DeviceInfo di;
+        di.sms = sms;
+        PATCH_CUDA(gemm_prepare_single());
+        PATCH_CUDA(gemm_prepare_pair(&di.pair_clusters));
+        if (di.pair_clusters <= 0) di.pair_clusters = 1;
+        it = g_dev.emplace(dev, di).first;
+    }
     *dev_out = dev;
-    *sms_out = sms;
+    *info_out = it->second;
     return PATCH_OK;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
-std::mutex g_prep_mu;
-std::map<int, bool> g_prepared;  // per device: kernel attributes set
 
 patch_status get_encode() {
     std::call_once(g_encode_once, [] {
@@ -86,36 +114,117 @@ patch_status get_encode() {
     return PATCH_OK;
 }
 
-patch_status prepare_device(int dev) {
-    std::lock_guard<std::mutex> lk(g_prep_mu);
-    if (g_prepared[dev]) return PATCH_OK;
-    PATCH_CUDA(gemm_prepare());
-    g_prepared[dev] = true;
+// 2-D bf16 tensor map: `rows` rows of `cols` elements (row pitch cols*2 bytes),
+// box of box_cols x box_rows.
+patch_status encode_2d(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols,
+                       int box_rows, CUtensorMapSwizzle swizzle) {
+    patch_status st = get_encode();
+    if (st != PATCH_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PATCH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return PATCH_OK;
 }
 
 struct WorkList {
-    int grid = 0;
+    int grid = 0;         // CTAs (single kernel) or clusters (pair kernel)
     int* off = nullptr;   // device, grid + 1
     int* work = nullptr;  // device, units
 };
+
+// Host copy of the three tables and the derived per-strip costs.
+struct Plan {
+    int S = 0, KB = 0, KC = 0;
+    std::vector<uint32_t> slab, meta, gemm;
+    std::vector<double> strip_cost, pair_cost;
+    int64_t bytes = 0, sparse = 0, pair_sparse = 0, meta_blocks = 0, images = 0;
+};
+
+// Region V (every slab), region E (a metadata block per chunk holding a 2:4
+// slab), region D (dense images of 2:4 slabs whose partner strip is dense).
+void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flags) {
+    p.S = (int)(N / kStrip);
+    p.KB = (int)(K / kSlabK);
+    p.KC = (p.KB + 1) / 2;
+    const int64_t tiles_k = K / C;
+    std::vector<uint8_t> sp((size_t)p.S * p.KB);
+    for (int s = 0; s < p.S; ++s)
+        for (int b = 0; b < p.KB; ++b) {
+            bool all = true;
+            for (int r0 = s * kStrip; r0 < (s + 1) * kStrip; r0 += R)
+                all = all && flags[(int64_t)(r0 / R) * tiles_k + ((int64_t)b * kSlabK) / C] != 0;
+            sp[(size_t)s * p.KB + b] = all;
+        }
+    auto is_sp = [&](int s, int b) { return sp[(size_t)s * p.KB + b] != 0; };
+    auto partner = [&](int s) { return ((s ^ 1) < p.S) ? (s ^ 1) : s; };
+    auto pair_sp = [&](int s, int b) { return is_sp(s, b) && is_sp(partner(s), b); };
+    p.slab.assign((size_t)p.S * p.KB, 0u);
+    p.meta.assign((size_t)p.S * p.KC, kNoMeta);
+    p.gemm.assign((size_t)p.S * p.KB, 0u);
+    p.strip_cost.assign(p.S, 0.0);
+    p.pair_cost.assign((p.S + 1) / 2, 0.0);
+    int64_t off = 0;
+    for (int s = 0; s < p.S; ++s)
+        for (int b = 0; b < p.KB; ++b) {
+            const bool x = is_sp(s, b);
+            const bool first = x && (b % 2 == 0 || !is_sp(s, b - 1));
+            p.slab[(size_t)s * p.KB + b] =
+                (uint32_t)((off / 16) << 2) | (first ? kSlabFirst : 0u) | (x ? kSlabSparse : 0u);
+            off += x ? kSparseValBytes : kDenseSlabBytes;
+            p.sparse += x;
+            p.strip_cost[s] += x ? 0.5 : 1.0;
+        }
+    for (int s = 0; s < p.S; ++s)
+        for (int c = 0; c < p.KC; ++c) {
+            bool any = is_sp(s, 2 * c) || (2 * c + 1 < p.KB && is_sp(s, 2 * c + 1));
+            if (any) {
+                p.meta[(size_t)s * p.KC + c] = (uint32_t)(off / 16);
+                off += kMetaBytes;
+                ++p.meta_blocks;
+            }
+        }
+    for (int s = 0; s < p.S; ++s)
+        for (int b = 0; b < p.KB; ++b) {
+            const bool x = is_sp(s, b), px = pair_sp(s, b);
+            int64_t a_off;
+            if (x && !px) {
+                a_off = off;
+                off += kDenseSlabBytes;
+                ++p.images;
+            } else {
+                a_off = (int64_t)slab_offset_bytes(p.slab[(size_t)s * p.KB + b]);
+            }
+            const bool first = px && (b % 2 == 0 || !pair_sp(s, b - 1));
+            p.gemm[(size_t)s * p.KB + b] =
+                (uint32_t)((a_off / 16) << 2) | (first ? kSlabFirst : 0u) | (px ? kSlabSparse : 0u);
+            p.pair_sparse += px;
+            if ((s & 1) == 0) p.pair_cost[s / 2] += px ? 0.5 : 1.0;
+        }
+    p.bytes = off;
+}
 
 }  // namespace
 
 struct patch_handle_s {
     int device = 0;
-    int sms = 0;
+    DeviceInfo dev;
     int64_t N = 0, K = 0;
-    int R = 0, C = 0, S = 0, KB = 0;
+    int R = 0, C = 0;
+    Plan plan;
     uint8_t* packed = nullptr;
-    int64_t packed_bytes = 0;
-    uint32_t* table_dev = nullptr;
-    std::vector<uint32_t> table;
-    std::vector<double> strip_cost;
+    uint32_t* slab_dev = nullptr;
+    uint32_t* meta_dev = nullptr;
+    uint32_t* gemm_dev = nullptr;
     int* status_dev = nullptr;
+    CUtensorMap tm_a16, tm_a8, tm_e;
     patch_info_t info{};
     std::mutex mu;
-    std::map<std::pair<int, int>, WorkList> work;  // (bn, m_blocks) -> schedule
+    std::map<std::pair<int, int>, WorkList> work;  // (kernel, m_blocks) -> schedule
     void* stage_x = nullptr;
     size_t stage_x_bytes = 0;
     void* stage_y = nullptr;
@@ -128,7 +237,9 @@ void free_handle(patch_handle h) {
     if (!h) return;
     cudaDeviceSynchronize();
     cudaFree(h->packed);
-    cudaFree(h->table_dev);
+    cudaFree(h->slab_dev);
+    cudaFree(h->meta_dev);
+    cudaFree(h->gemm_dev);
     cudaFree(h->status_dev);
     for (auto& kv : h->work) {
         cudaFree(kv.second.off);
@@ -139,57 +250,27 @@ void free_handle(patch_handle h) {
     delete h;
 }
 
-// Slab table: a slab (128 rows x 64 columns) is stored compressed only when
-// every mask tile it overlaps is flagged 2:4; the first compressed slab of a
-// 128-column chunk carries that chunk's metadata block.
-int64_t build_table(patch_handle h, const uint8_t* flags) {
-    const int64_t tiles_k = h->K / h->C;
-    h->table.assign((size_t)h->S * h->KB, 0u);
-    h->strip_cost.assign(h->S, 0.0);
-    int64_t off = 0, sparse_slabs = 0;
-    for (int s = 0; s < h->S; ++s) {
-        int meta_chunk = -1;
-        for (int b = 0; b < h->KB; ++b) {
-            bool sp = true;
-            for (int r0 = s * kStrip; r0 < (s + 1) * kStrip; r0 += h->R)
-                sp = sp && flags[(int64_t)(r0 / h->R) * tiles_k + ((int64_t)b * kSlabK) / h->C] != 0;
-            bool meta = false;
-            if (sp && meta_chunk != b / 2) {
-                meta = true;
-                meta_chunk = b / 2;
-            }
-            h->table[(size_t)s * h->KB + b] =
-                (uint32_t)((off / 16) << 2) | (meta ? kSlabHasMeta : 0u) | (sp ? kSlabSparse : 0u);
-            off += sp ? kSparseValBytes + (meta ? kMetaBytes : 0) : kDenseSlabBytes;
-            sparse_slabs += sp;
-            h->strip_cost[s] += sp ? 0.5 : 1.0;
-        }
-    }
-    h->info.slabs_total = (int64_t)h->S * h->KB;
-    h->info.slabs_sparse = sparse_slabs;
-    return off;
-}
-
-// Greedy longest-processing-time assignment of output tiles (strip, token
-// block) to persistent CTAs. A tile's cost is its slab work (dense 1, sparse
-// 1/2, the ratio of tensor-core time) plus a fixed epilogue share.
-patch_status get_worklist(patch_handle h, int bn, int mb, WorkList** out) {
+// Greedy longest-processing-time assignment of output tiles to persistent
+// CTAs (or CTA pairs). A tile's cost is its slab work (dense 1, sparse 1/2,
+// the ratio of tensor-core time) plus a fixed epilogue share.
+patch_status get_worklist(patch_handle h, int kernel, int mb, WorkList** out) {
     std::lock_guard<std::mutex> lk(h->mu);
-    auto key = std::make_pair(bn, mb);
+    auto key = std::make_pair(kernel, mb);
     auto it = h->work.find(key);
     if (it != h->work.end()) {
         *out = &it->second;
         return PATCH_OK;
     }
-    const int units = h->S * mb;
-    const int grid = std::max(1, std::min(h->sms, units));
+    const std::vector<double>& cost = kernel == 0 ? h->plan.strip_cost : h->plan.pair_cost;
+    const int rows = (int)cost.size();
+    const int units = rows * mb;
+    const int slots = kernel == 0 ? h->dev.sms : h->dev.pair_clusters;
+    const int grid = std::max(1, std::min(slots, units));
     std::vector<int> order(units);
     for (int u = 0; u < units; ++u) order[u] = u;
     const double epi = 1.0;
-    std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
-        return h->strip_cost[x / mb] > h->strip_cost[y / mb];
-    });
-    using Item = std::pair<double, int>;  // (load, cta)
+    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x / mb] > cost[y / mb]; });
+    using Item = std::pair<double, int>;  // (load, slot)
     std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
     for (int c = 0; c < grid; ++c) pq.push({0.0, c});
     std::vector<std::vector<int>> lists(grid);
@@ -197,7 +278,7 @@ patch_status get_worklist(patch_handle h, int bn, int mb, WorkList** out) {
         Item top = pq.top();
         pq.pop();
         lists[top.second].push_back(u);
-        top.first += h->strip_cost[u / mb] + epi;
+        top.first += cost[u / mb] + epi;
         pq.push(top);
     }
     std::vector<int> off(grid + 1, 0), work;
@@ -212,6 +293,7 @@ patch_status get_worklist(patch_handle h, int bn, int mb, WorkList** out) {
     if (cudaMalloc(&wl.off, sizeof(int) * (grid + 1)) != cudaSuccess ||
         cudaMalloc(&wl.work, sizeof(int) * std::max(units, 1)) != cudaSuccess) {
         cudaFree(wl.off);
+        cudaGetLastError();
         return fail(PATCH_ERR_NOMEM, "schedule allocation failed");
     }
     PATCH_CUDA(cudaMemcpy(wl.off, off.data(), sizeof(int) * (grid + 1), cudaMemcpyHostToDevice));
@@ -221,67 +303,85 @@ patch_status get_worklist(patch_handle h, int bn, int mb, WorkList** out) {
     return PATCH_OK;
 }
 
-patch_status make_x_map(CUtensorMap* map, const void* X, int64_t M, int64_t K, int bn) {
-    patch_status st = get_encode();
-    if (st != PATCH_OK) return st;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kSlabK, (cuuint32_t)bn};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(PATCH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return PATCH_OK;
-}
-
 patch_status check_handle_device(patch_handle h) {
     int dev = -1;
     PATCH_CUDA(cudaGetDevice(&dev));
-    if (dev != h->device) return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", h->device, dev);
+    if (dev != h->device)
+        return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", h->device, dev);
     return PATCH_OK;
 }
 
+constexpr int64_t kPairMinM = 256;  // below this the single-CTA tiles keep more SMs busy
+
 patch_status run_linear(patch_handle h, const void* X, int64_t M, void* Y, int path, cudaStream_t st) {
     if (path == PATCH_PATH_AUTO) path = (M <= 8) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
+    if (path == PATCH_PATH_GEMM) path = (M >= kPairMinM) ? PATCH_PATH_GEMM_PAIR : PATCH_PATH_GEMM_SINGLE;
     if (path == PATCH_PATH_GEMV) {
         if (M > 16) return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
         GemvArgs a;
         a.packed = h->packed;
-        a.table = h->table_dev;
+        a.slab = h->slab_dev;
+        a.meta = h->meta_dev;
         a.X = static_cast<const __nv_bfloat16*>(X);
         a.Y = static_cast<__nv_bfloat16*>(Y);
         a.M = (int)M;
         a.N = (int)h->N;
         a.K = (int)h->K;
-        a.KB = h->KB;
+        a.KB = h->plan.KB;
+        a.KC = h->plan.KC;
         cudaError_t e = launch_gemv(a, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
         return PATCH_OK;
     }
-    if (path != PATCH_PATH_GEMM) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
-    const int bn = gemm_bn_for((int)M);
-    const int mb = (int)((M + bn - 1) / bn);
+    if (path == PATCH_PATH_GEMM_SINGLE) {
+        const int mb = (int)((M + kGemmBN - 1) / kGemmBN);
+        WorkList* wl = nullptr;
+        patch_status s = get_worklist(h, 0, mb, &wl);
+        if (s != PATCH_OK) return s;
+        CUtensorMap map;
+        s = encode_2d(&map, X, h->K, M, kSlabK, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s != PATCH_OK) return s;
+        GemmArgs a;
+        a.packed = h->packed;
+        a.slab = h->slab_dev;
+        a.meta = h->meta_dev;
+        a.work_off = wl->off;
+        a.work = wl->work;
+        a.M = (int)M;
+        a.N = (int)h->N;
+        a.KB = h->plan.KB;
+        a.KC = h->plan.KC;
+        a.MB = mb;
+        a.Y = static_cast<__nv_bfloat16*>(Y);
+        a.status = h->status_dev;
+        cudaError_t e = launch_gemm(map, a, wl->grid, st);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+        return PATCH_OK;
+    }
+    if (path != PATCH_PATH_GEMM_PAIR) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    const int mb = (int)((M + kGemm2BN - 1) / kGemm2BN);
     WorkList* wl = nullptr;
-    patch_status s = get_worklist(h, bn, mb, &wl);
+    patch_status s = get_worklist(h, 1, mb, &wl);
     if (s != PATCH_OK) return s;
     CUtensorMap map;
-    s = make_x_map(&map, X, M, h->K, bn);
+    s = encode_2d(&map, X, h->K, M, kSlabK, kGemm2BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != PATCH_OK) return s;
-    GemmArgs a;
-    a.packed = h->packed;
-    a.table = h->table_dev;
+    Gemm2Args a;
+    a.gemm = h->gemm_dev;
+    a.meta = h->meta_dev;
     a.work_off = wl->off;
     a.work = wl->work;
     a.M = (int)M;
     a.N = (int)h->N;
-    a.KB = h->KB;
+    a.S = h->plan.S;
+    a.KB = h->plan.KB;
+    a.KC = h->plan.KC;
     a.MB = mb;
     a.Y = static_cast<__nv_bfloat16*>(Y);
     a.status = h->status_dev;
-    cudaError_t e = launch_gemm(map, a, wl->grid, bn, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+    cudaError_t e = launch_gemm2(map, h->tm_a16, h->tm_a8, h->tm_e, a, wl->grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "CTA-pair tensor-core kernel launch");
     return PATCH_OK;
 }
 
@@ -291,7 +391,24 @@ extern "C" {
 
 const char* patch_last_error(void) { return g_err.c_str(); }
 
-int patch_version(void) { return 1; }
+int patch_version(void) { return 2; }
+
+patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
+                        uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table, int64_t* packed_bytes) {
+    g_err.clear();
+    if (!tile_flags) return fail(PATCH_ERR_ARG, "tile_flags is NULL");
+    patch_status st = check_shape(N, K, tile_rows, tile_cols);
+    if (st != PATCH_OK) return st;
+    st = check_flags(tile_flags, (N / tile_rows) * (K / tile_cols));
+    if (st != PATCH_OK) return st;
+    Plan p;
+    build_plan(p, N, K, tile_rows, tile_cols, tile_flags);
+    if (slab_table) memcpy(slab_table, p.slab.data(), sizeof(uint32_t) * p.slab.size());
+    if (meta_table) memcpy(meta_table, p.meta.data(), sizeof(uint32_t) * p.meta.size());
+    if (gemm_table) memcpy(gemm_table, p.gemm.data(), sizeof(uint32_t) * p.gemm.size());
+    if (packed_bytes) *packed_bytes = p.bytes;
+    return PATCH_OK;
+}
 
 patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t* mask_bits, int bitorder,
                         const uint8_t* tile_flags, int tile_rows, int tile_cols, void* stream,
@@ -299,44 +416,37 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     g_err.clear();
     if (!out) return fail(PATCH_ERR_ARG, "out is NULL");
     *out = nullptr;
-    if (!W_bf16 || !mask_bits || !tile_flags) return fail(PATCH_ERR_ARG, "W, mask_bits and tile_flags must be non-NULL");
+    if (!W_bf16 || !mask_bits || !tile_flags)
+        return fail(PATCH_ERR_ARG, "W, mask_bits and tile_flags must be non-NULL");
     if (bitorder != 0 && bitorder != 1) return fail(PATCH_ERR_ARG, "bitorder must be 0 or 1");
-    {
-        patch_status sst = check_shape(N, K, tile_rows, tile_cols);
-        if (sst != PATCH_OK) return sst;
-    }
-    if (!aligned16(W_bf16)) return fail(PATCH_ERR_ALIGN, "W must be 16-byte aligned");
-    int dev = 0, sms = 0;
-    patch_status st = check_device(&dev, &sms);
+    patch_status st = check_shape(N, K, tile_rows, tile_cols);
     if (st != PATCH_OK) return st;
-    st = prepare_device(dev);
+    if (!aligned16(W_bf16)) return fail(PATCH_ERR_ALIGN, "W must be 16-byte aligned");
+    const int64_t ntiles = (N / tile_rows) * (K / tile_cols);
+    st = check_flags(tile_flags, ntiles);
+    if (st != PATCH_OK) return st;
+    int dev = 0;
+    DeviceInfo di;
+    st = prepare_device(&dev, &di);
     if (st != PATCH_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     patch_handle h = new (std::nothrow) patch_handle_s();
     if (!h) return fail(PATCH_ERR_NOMEM, "host allocation failed");
     h->device = dev;
-    h->sms = sms;
+    h->dev = di;
     h->N = N;
     h->K = K;
     h->R = tile_rows;
     h->C = tile_cols;
-    h->S = (int)(N / kStrip);
-    h->KB = (int)(K / kSlabK);
-    const int64_t ntiles = (N / tile_rows) * (K / tile_cols);
-    int64_t tiles_sparse = 0;
-    for (int64_t i = 0; i < ntiles; ++i) {
-        if (tile_flags[i] > 1) {
-            free_handle(h);
-            return fail(PATCH_ERR_ARG, "tile flag %lld is %d, must be 0 or 1", (long long)i, (int)tile_flags[i]);
-        }
-        tiles_sparse += tile_flags[i];
-    }
-    h->packed_bytes = build_table(h, tile_flags);
-    if (h->packed_bytes / 16 >= ((int64_t)1 << 30)) {
+    build_plan(h->plan, N, K, tile_rows, tile_cols, tile_flags);
+    const Plan& p = h->plan;
+    if (p.bytes / 16 >= ((int64_t)1 << 30)) {
         free_handle(h);
-        return fail(PATCH_ERR_SHAPE, "packed weight exceeds the 16 GiB slab-table range");
+        return fail(PATCH_ERR_SHAPE, "packed weight exceeds the 16 GiB table range");
     }
+    int64_t tiles_sparse = 0;
+    for (int64_t i = 0; i < ntiles; ++i) tiles_sparse += tile_flags[i];
 
     uint8_t* flags_dev = nullptr;
     unsigned long long* counters = nullptr;
@@ -346,16 +456,29 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         if (code != PATCH_OK) free_handle(h);
         return code;
     };
-    if (cudaMalloc(&h->packed, std::max<int64_t>(h->packed_bytes, 16)) != cudaSuccess ||
-        cudaMalloc(&h->table_dev, sizeof(uint32_t) * h->table.size()) != cudaSuccess ||
+    if (cudaMalloc(&h->packed, std::max<int64_t>(p.bytes, 2048)) != cudaSuccess ||
+        cudaMalloc(&h->slab_dev, sizeof(uint32_t) * p.slab.size()) != cudaSuccess ||
+        cudaMalloc(&h->meta_dev, sizeof(uint32_t) * p.meta.size()) != cudaSuccess ||
+        cudaMalloc(&h->gemm_dev, sizeof(uint32_t) * p.gemm.size()) != cudaSuccess ||
         cudaMalloc(&h->status_dev, sizeof(int)) != cudaSuccess || cudaMalloc(&flags_dev, ntiles) != cudaSuccess ||
         cudaMalloc(&counters, 3 * sizeof(unsigned long long)) != cudaSuccess) {
         cudaGetLastError();
-        return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)h->packed_bytes));
+        return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
     }
+    // tensor maps of the packed bytes viewed as rows of 64 bf16 (128 bytes):
+    // dense slab / dense image (128 rows), 2:4 values (64 rows), metadata (16 rows)
+    const int64_t rows = std::max<int64_t>(p.bytes, 2048) / 128;
+    if ((st = encode_2d(&h->tm_a16, h->packed, 64, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
+        (st = encode_2d(&h->tm_a8, h->packed, 64, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
+        (st = encode_2d(&h->tm_e, h->packed, 64, rows, 64, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK)
+        return cleanup(st);
     cudaError_t e;
-    if ((e = cudaMemcpyAsync(h->table_dev, h->table.data(), sizeof(uint32_t) * h->table.size(),
-                             cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+    if ((e = cudaMemcpyAsync(h->slab_dev, p.slab.data(), sizeof(uint32_t) * p.slab.size(), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(h->meta_dev, p.meta.data(), sizeof(uint32_t) * p.meta.size(), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(h->gemm_dev, p.gemm.data(), sizeof(uint32_t) * p.gemm.size(), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(flags_dev, tile_flags, ntiles, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
         (e = cudaMemsetAsync(counters, 0, 3 * sizeof(unsigned long long), s)) != cudaSuccess ||
         (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess)
@@ -365,14 +488,17 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     a.bits = mask_bits;
     a.bitorder = bitorder;
     a.flags = flags_dev;
-    a.table = h->table_dev;
+    a.slab = h->slab_dev;
+    a.meta = h->meta_dev;
+    a.gemm = h->gemm_dev;
     a.out = h->packed;
     a.K = K;
     a.R = tile_rows;
     a.C = tile_cols;
-    a.KB = h->KB;
+    a.KB = p.KB;
+    a.KC = p.KC;
     a.counters = counters;
-    pack_kernel<<<h->S * h->KB, 256, 0, s>>>(a);
+    pack_kernel<<<p.S * p.KB, 256, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return cleanup(cuda_fail(e, "pack kernel launch"));
     unsigned long long cnt[3] = {0, 0, 0};
     if ((e = cudaMemcpyAsync(cnt, counters, sizeof(cnt), cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
@@ -380,16 +506,22 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         return cleanup(cuda_fail(e, "pack kernel"));
     if (cnt[0] != 0)
         return cleanup(fail(PATCH_ERR_MASK, "%llu groups inside 2:4 tiles do not keep exactly two of four", cnt[0]));
-    h->info.N = N;
-    h->info.K = K;
-    h->info.tile_rows = tile_rows;
-    h->info.tile_cols = tile_cols;
-    h->info.tiles_total = ntiles;
-    h->info.tiles_sparse = tiles_sparse;
-    h->info.packed_bytes = h->packed_bytes;
-    h->info.pruned = (int64_t)cnt[2];
-    h->info.stray_zeros = (int64_t)cnt[1];
-    h->info.sparsity = (double)cnt[2] / (double)(N * K);
+    patch_info_t& info = h->info;
+    info.N = N;
+    info.K = K;
+    info.tile_rows = tile_rows;
+    info.tile_cols = tile_cols;
+    info.tiles_total = ntiles;
+    info.tiles_sparse = tiles_sparse;
+    info.slabs_total = (int64_t)p.S * p.KB;
+    info.slabs_sparse = p.sparse;
+    info.slabs_pair_sparse = p.pair_sparse;
+    info.meta_blocks = p.meta_blocks;
+    info.dense_images = p.images;
+    info.packed_bytes = p.bytes;
+    info.pruned = (int64_t)cnt[2];
+    info.stray_zeros = (int64_t)cnt[1];
+    info.sparsity = (double)cnt[2] / (double)(N * K);
     *out = h;
     return cleanup(PATCH_OK);
 }
@@ -398,10 +530,10 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
                                void* stream) {
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_PAIR) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     if (!X_bf16 || !Y_bf16) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
     if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMV) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     patch_status st = check_handle_device(h);
     if (st != PATCH_OK) return st;
     return run_linear(h, X_bf16, M, Y_bf16, path, static_cast<cudaStream_t>(stream));
@@ -424,14 +556,20 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
         cudaFree(h->stage_x);
         h->stage_x = nullptr;
         h->stage_x_bytes = 0;
-        if (cudaMalloc(&h->stage_x, xb) != cudaSuccess) return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+        if (cudaMalloc(&h->stage_x, xb) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+        }
         h->stage_x_bytes = xb;
     }
     if (yb > h->stage_y_bytes) {
         cudaFree(h->stage_y);
         h->stage_y = nullptr;
         h->stage_y_bytes = 0;
-        if (cudaMalloc(&h->stage_y, yb) != cudaSuccess) return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+        if (cudaMalloc(&h->stage_y, yb) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+        }
         h->stage_y_bytes = yb;
     }
     PATCH_CUDA(cudaMemcpyAsync(h->stage_x, X_host, xb, cudaMemcpyHostToDevice, s));
@@ -447,8 +585,8 @@ patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream) {
     if (!aligned16(W_masked_bf16)) return fail(PATCH_ERR_ALIGN, "output must be 16-byte aligned");
     patch_status st = check_handle_device(h);
     if (st != PATCH_OK) return st;
-    unpack_kernel<<<h->S * h->KB, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        h->packed, h->table_dev, h->KB, h->K, static_cast<uint16_t*>(W_masked_bf16));
+    unpack_kernel<<<h->plan.S * h->plan.KB, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        h->packed, h->slab_dev, h->meta_dev, h->plan.KB, h->plan.KC, h->K, static_cast<uint16_t*>(W_masked_bf16));
     PATCH_CUDA(cudaGetLastError());
     return PATCH_OK;
 }
@@ -459,17 +597,18 @@ patch_status patch_info(patch_handle h, patch_info_t* info) {
     return PATCH_OK;
 }
 
-patch_status patch_copy_packed(patch_handle h, void* packed_host, int64_t packed_cap, uint32_t* table_host,
-                               int64_t table_cap) {
+patch_status patch_copy_packed(patch_handle h, void* packed_host, int64_t packed_cap, uint32_t* slab_host,
+                               int64_t slab_cap, uint32_t* meta_host, int64_t meta_cap, uint32_t* gemm_host,
+                               int64_t gemm_cap) {
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
-    if (packed_host) {
-        if (packed_cap < h->packed_bytes) return fail(PATCH_ERR_ARG, "packed buffer too small");
-        PATCH_CUDA(cudaMemcpy(packed_host, h->packed, h->packed_bytes, cudaMemcpyDeviceToHost));
-    }
-    if (table_host) {
-        if (table_cap < (int64_t)h->table.size()) return fail(PATCH_ERR_ARG, "table buffer too small");
-        memcpy(table_host, h->table.data(), sizeof(uint32_t) * h->table.size());
-    }
+    const Plan& p = h->plan;
+    if ((packed_host && packed_cap < p.bytes) || (slab_host && slab_cap < (int64_t)p.slab.size()) ||
+        (meta_host && meta_cap < (int64_t)p.meta.size()) || (gemm_host && gemm_cap < (int64_t)p.gemm.size()))
+        return fail(PATCH_ERR_ARG, "a destination buffer is too small");
+    if (packed_host) PATCH_CUDA(cudaMemcpy(packed_host, h->packed, p.bytes, cudaMemcpyDeviceToHost));
+    if (slab_host) memcpy(slab_host, p.slab.data(), sizeof(uint32_t) * p.slab.size());
+    if (meta_host) memcpy(meta_host, p.meta.data(), sizeof(uint32_t) * p.meta.size());
+    if (gemm_host) memcpy(gemm_host, p.gemm.data(), sizeof(uint32_t) * p.gemm.size());
     return PATCH_OK;
 }
 
@@ -488,27 +627,5 @@ patch_status patch_check(patch_handle h, void* stream) {
 }
 
 void patch_free(patch_handle h) { free_handle(h); }
-
-patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
-                        uint32_t* table_host, int64_t* packed_bytes) {
-    g_err.clear();
-    if (!tile_flags) return fail(PATCH_ERR_ARG, "tile_flags is NULL");
-    patch_status st = check_shape(N, K, tile_rows, tile_cols);
-    if (st != PATCH_OK) return st;
-    const int64_t ntiles = (N / tile_rows) * (K / tile_cols);
-    for (int64_t i = 0; i < ntiles; ++i)
-        if (tile_flags[i] > 1) return fail(PATCH_ERR_ARG, "tile flag %lld is %d, must be 0 or 1", (long long)i, (int)tile_flags[i]);
-    patch_handle_s tmp;
-    tmp.N = N;
-    tmp.K = K;
-    tmp.R = tile_rows;
-    tmp.C = tile_cols;
-    tmp.S = (int)(N / kStrip);
-    tmp.KB = (int)(K / kSlabK);
-    const int64_t bytes = build_table(&tmp, tile_flags);
-    if (table_host) memcpy(table_host, tmp.table.data(), sizeof(uint32_t) * tmp.table.size());
-    if (packed_bytes) *packed_bytes = bytes;
-    return PATCH_OK;
-}
 
 }  // extern "C"

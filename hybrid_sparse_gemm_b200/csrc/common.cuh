@@ -10,20 +10,27 @@
 namespace patch {
 
 // ---- packed weight format --------------------------------------------------
-// A strip is 128 rows of W, a slab is a strip times 64 columns; slabs are
-// stored strip-major with K ascending. A dense slab is the 128x64 bf16 block
-// in the 128-byte-swizzled K-major layout the tensor core reads; a sparse
-// slab is 128x32 kept values in the 64-byte-swizzled layout. A 2048-byte
-// metadata block per 128-column chunk follows the values of the chunk's first
-// sparse slab, laid out lane-major (16 bytes per TMEM lane) so one
-// tcgen05.cp.128x128b moves it into four TMEM columns.
+// A strip is 128 rows of W, a slab is a strip times 64 columns, a chunk two
+// slabs. Strips 2p and 2p+1 are partners (an odd last strip is its own).
+// Region V holds every slab, strip-major with K ascending: a dense slab is the
+// 128x64 bf16 block in the 128-byte-swizzled K-major layout the tensor core
+// reads; a sparse slab is 128x32 kept values in the 64-byte-swizzled layout.
+// Region E holds one 2048-byte metadata block per chunk with a sparse slab,
+// lane-major (16 bytes per TMEM lane) so one tcgen05.cp.128x128b moves it
+// into four TMEM columns. Region D holds a dense image of each sparse slab
+// whose partner's slab is dense, for the CTA-pair kernel (one MMA instruction
+// spans both strips, so both must be of one kind).
+// Tables of uint32: slab = (V offset/16)<<2 | first<<1 | sparse (first: the
+// chunk's first sparse slab); meta = E offset/16 or kNoMeta; gemm = (offset/16)<<2
+// | first<<1 | pair_sparse, pointing at the record the CTA-pair kernel loads.
 constexpr int kStrip = 128;
 constexpr int kSlabK = 64;
 constexpr int kDenseSlabBytes = kStrip * kSlabK * 2;   // 16384
 constexpr int kSparseValBytes = kStrip * kSlabK;       // 8192
 constexpr int kMetaBytes = 2048;
 constexpr uint32_t kSlabSparse = 1u;
-constexpr uint32_t kSlabHasMeta = 2u;
+constexpr uint32_t kSlabFirst = 2u;
+constexpr uint32_t kNoMeta = 0xFFFFFFFFu;
 
 __host__ __device__ inline uint64_t slab_offset_bytes(uint32_t d) { return (uint64_t)(d >> 2) * 16; }
 

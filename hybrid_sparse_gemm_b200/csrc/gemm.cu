@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
                 const int s = u / a.MB, j = u % a.MB;
-                const uint32_t* trow = a.table + (size_t)s * a.KB;
+                const uint32_t* trow = a.slab + (size_t)s * a.KB;
+                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
                 for (int b = 0; b < a.KB; ++b) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ab.raise();
@@ -116,12 +117,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const uint32_t d = trow[b];
-                    const uint32_t bytes_a = (d & kSlabSparse)
-                                                 ? (kSparseValBytes + ((d & kSlabHasMeta) ? kMetaBytes : 0))
-                                                 : kDenseSlabBytes;
-                    mbar_arrive_expect_tx(&full[stage], bytes_a + C::kStageBBytes);
-                    bulk_load(sA + stage * kStageABytes, a.packed + slab_offset_bytes(d), bytes_a,
-                              &full[stage]);
+                    const bool sp = d & kSlabSparse, first = d & kSlabFirst;
+                    const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
+                    mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + C::kStageBBytes);
+                    bulk_load(sA + stage * kStageABytes, a.packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    if (first)
+                        bulk_load(sA + stage * kStageABytes + kSparseValBytes,
+                                  a.packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes, &full[stage]);
                     tma_load_2d(sB + stage * C::kStageBBytes, &tmap_x, &full[stage], b * kSlabK, j * BN);
                     ++issued;
                     if (++stage == C::kStages) {
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
                 const int s = u / a.MB;
-                const uint32_t* trow = a.table + (size_t)s * a.KB;
+                const uint32_t* trow = a.slab + (size_t)s * a.KB;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
                     ab.raise();
                     break;
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a_addr = smem_u32(sA + stage * kStageABytes);
                     const uint32_t b_addr = smem_u32(sB + stage * C::kStageBBytes);
                     if (d & kSlabSparse) {
-                        if (d & kSlabHasMeta)
+                        if (d & kSlabFirst)
                             tc_cp_128x128b(tmem_base + C::kECol,
                                            smem_desc(a_addr + kSparseValBytes, 16, 128, kLayoutNone));
 #pragma unroll
@@ -276,25 +278,10 @@ cudaError_t set_attr() {
 
 }  // namespace
 
-int gemm_bn_for(int M) {
-    (void)M;
-    return 128;
-}
+cudaError_t gemm_prepare_single() { return set_attr<kGemmBN>(); }
 
-cudaError_t gemm_prepare() {
-    cudaError_t e = set_attr<128>();
-    if (e != cudaSuccess) return e;
-    return cudaSuccess;
-}
-
-cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmArgs& a, int grid, int bn, cudaStream_t st) {
-    switch (bn) {
-        case 128:
-            hybrid_gemm_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, st>>>(tmap_x, a);
-            break;
-        default:
-            return cudaErrorInvalidValue;
-    }
+cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmArgs& a, int grid, cudaStream_t st) {
+    hybrid_gemm_kernel<kGemmBN><<<grid, kThreads, Cfg<kGemmBN>::kSmemBytes, st>>>(tmap_x, a);
     return cudaGetLastError();
 }
 

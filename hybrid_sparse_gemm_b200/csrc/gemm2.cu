@@ -1,0 +1,390 @@
+// Hybrid dense / 2:4 GEMM on a CTA pair (cta_group::2): Y = X . (W (.) Mask)^T.
+//
+// Same method as the single-CTA kernel (dense slabs on tcgen05.mma, 2:4 slabs
+// on tcgen05.mma.sp; PATCH abstract, "PATCH: Learnable Tile-level Hybrid
+// Sparsity for LLMs"), on the unit Blackwell's tensor core is built around:
+// two CTAs on neighbouring SMs form one 256 x 256 MMA. CTA r holds the 128
+// weight rows of strip 2p+r (operand A) and tokens [128r, 128r+128) of the
+// block (operand B); each MMA multiplies both A halves by both B halves, so an
+// SM loads half the activations it would need alone. The leader CTA (rank 0)
+// issues every MMA; both CTAs' TMA loads complete on the leader's barriers,
+// and the leader's commits arrive on both CTAs' barriers.
+//
+// TMEM: each CTA holds its 128 rows x 256 tokens in one of two 256-column
+// accumulators. The 2:4 metadata of the running tile lives in the last four
+// columns of the other accumulator: its epilogue drains those columns first
+// and releases them early (e_free) so the next tile's tcgen05.cp can land.
+//
+// Both strips of a pair load the same kind of record at every slab (dense
+// images stand in for 2:4 slabs whose partner is dense), so one MMA
+// instruction always covers both. An odd last strip pairs with itself; its
+// second CTA computes a duplicate and stores nothing.
+#include "kernels.cuh"
+
+namespace patch {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kHalf = 128;                    // tokens per CTA
+constexpr int kStages = 6;
+constexpr int kStageA = 18432;                // 16 KB dense, or 8 KB values + 2 KB metadata
+constexpr int kStageB = kHalf * 128;          // 16 KB
+constexpr int kSmemData = kStages * (kStageA + kStageB);
+constexpr int kSmemBytes = kSmemData + 1024 + 256;
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 512;
+constexpr int kETail = kAccCols - 4;          // metadata columns inside the idle accumulator
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 2-D TMA load whose completion is counted on the leader CTA's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void mma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma2_sp_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t e_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+        : "memory");
+}
+__device__ __forceinline__ void cp2_128x128b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Commit of the leader's MMAs, arriving on the barrier at this offset in both CTAs.
+__device__ __forceinline__ void commit2_both(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void commit2_local(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    hybrid_gemm2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a16,
+                        const __grid_constant__ CUtensorMap tm_a8, const __grid_constant__ CUtensorMap tm_e,
+                        const Gemm2Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kStageA;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
+    uint64_t* full = bars;                  // leader: both CTAs' bytes of a stage
+    uint64_t* empty = bars + kStages;       // both: stage consumed by the MMAs
+    uint64_t* acc_full = bars + 2 * kStages;  // both: accumulator ready
+    uint64_t* acc_empty = acc_full + 2;     // leader: 8 epilogue warps drained it
+    uint64_t* e_free = acc_full + 4;        // leader: 8 epilogue warps read its tail
+    uint64_t* drain = acc_full + 6;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int cl = blockIdx.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 8);
+            mbar_init(&e_free[i], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_a16);
+        prefetch_tmap(&tm_a8);
+        prefetch_tmap(&tm_e);
+    }
+    if (warp == 1) {
+        tmem_alloc2(tmem_slot, kTmemCols);
+        tmem_relinquish2();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    auto raise = [&]() {
+        *abort_flag = 1;
+        atomicCAS(a.status, 0, kStatusTimeout);
+    };
+
+    const int w_begin = a.work_off[cl];
+    const int w_end = a.work_off[cl + 1];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer (both CTAs) ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int it = w_begin; it < w_end && ok; ++it) {
+                const int u = a.work[it];
+                const int p = u / a.MB, j = u % a.MB;
+                int s = 2 * p + (int)rank;
+                if (s >= a.S) s = 2 * p;  // odd last strip: duplicate
+                const uint32_t* trow = a.gemm + (size_t)s * a.KB;
+                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
+                for (int b = 0; b < a.KB; ++b) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t d = trow[b];
+                    const bool sp = d & kSlabSparse, first = d & kSlabFirst;
+                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&full[stage],
+                                              2u * ((sp ? kSparseValBytes : kDenseSlabBytes) +
+                                                    (first ? kMetaBytes : 0) + kStageB));
+                    const uint32_t dst_a = smem_u32(sA + stage * kStageA);
+                    const int row = (int)(slab_offset_bytes(d) >> 7);
+                    tma_load_2d_pair(dst_a, sp ? &tm_a8 : &tm_a16, bar, 0, row);
+                    if (first)
+                        tma_load_2d_pair(dst_a + kSparseValBytes, &tm_e, bar, 0, (int)(mrow[b >> 1] >> 3));
+                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tm_x, bar, b * kSlabK,
+                                     j * kGemm2BN + (int)rank * kHalf);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (rank == 0) {
+                // Bounded wait for the loads of the last stages, whatever the
+                // abort flag says, so none lands after the pair exits.
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < kStages && i < issued; ++i) {
+                    if (--st < 0) {
+                        st = kStages - 1;
+                        ph ^= 1u;
+                    }
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&full[st], ph) && globaltimer() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (leader) ----------------
+            const uint32_t idesc_d = idesc_bf16(256, kGemm2BN, false);
+            const uint32_t idesc_s = idesc_bf16(256, kGemm2BN, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, any_mma = false;
+            int t = 0;
+            for (int it = w_begin; it < w_end && ok; ++it, ++t) {
+                const int u = a.work[it];
+                const int p = u / a.MB;
+                const uint32_t* trow = a.gemm + (size_t)(2 * p) * a.KB;
+                const int acc = t & 1;
+                if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
+                    raise();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+                const uint32_t e_base = tmem_base + (uint32_t)((1 - acc) * kAccCols + kETail);
+                bool e_ready = (t == 0);
+                for (int b = 0; b < a.KB; ++b) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = trow[b];
+                    const uint32_t a_addr = smem_u32(sA + stage * kStageA);
+                    const uint32_t b_addr = smem_u32(sB + stage * kStageB);
+                    if (d & kSlabSparse) {
+                        if (d & kSlabFirst) {
+                            if (!e_ready) {
+                                if (!mbar_wait(&e_free[1 - acc], ((t - 1) >> 1) & 1, abort_flag)) {
+                                    raise();
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
+                                e_ready = true;
+                            }
+                            cp2_128x128b(e_base, smem_desc(a_addr + kSparseValBytes, 16, 128, kLayoutNone));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 512, kLayoutSw64);
+                            const uint64_t bd = smem_desc(b_addr + i * 64, 16, 1024, kLayoutSw128);
+                            const uint32_t ecol = e_base + (uint32_t)((b & 1) * 2 + i);
+                            mma2_sp_bf16(d_tmem, ad, bd, idesc_s | (ecol & 1u), ecol & ~1u, (b | i) != 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 1024, kLayoutSw128);
+                            const uint64_t bd = smem_desc(b_addr + i * 32, 16, 1024, kLayoutSw128);
+                            mma2_bf16(d_tmem, ad, bd, idesc_d, (b | i) != 0);
+                        }
+                    }
+                    any_mma = true;
+                    commit2_both(&empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                commit2_both(&acc_full[acc]);
+            }
+            if (*abort_flag && any_mma) {
+                commit2_local(drain);
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+        const int q = warp & 3;
+        int t = 0;
+        for (int it = w_begin; it < w_end; ++it, ++t) {
+            const int u = a.work[it];
+            const int p = u / a.MB, j = u % a.MB;
+            const int s = 2 * p + (int)rank;
+            const bool store = s < a.S;
+            const int acc = t & 1;
+            if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
+                if (lane == 0) raise();
+                break;
+            }
+            tc_fence_after();
+            const int n = s * kStrip + q * 32 + lane;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
+            __nv_bfloat16* yc = a.Y + n;
+#pragma unroll 1
+            for (int c0 = kAccCols - 32; c0 >= 0; c0 -= 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(taddr + c0, v);
+                tc_wait_ld();
+                if (c0 == kAccCols - 32) {
+                    // The tail (metadata columns of the next tile) is read: release it.
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) remote_arrive(map_to_rank(smem_u32(&e_free[acc]), 0));
+                }
+                if (!store) continue;
+                const int m0 = j * kGemm2BN + c0;
+                if (m0 + 32 <= a.M) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (m0 + c < a.M)
+                            yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[acc]), 0));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its partner may still signal it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc2(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t gemm_prepare_pair(int* max_clusters) {
+    cudaError_t e =
+        cudaFuncSetAttribute(hybrid_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm2_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    *max_clusters = n;
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm2(const CUtensorMap& tmap_x, const CUtensorMap& tm_a16, const CUtensorMap& tm_a8,
+                         const CUtensorMap& tm_e, const Gemm2Args& a, int clusters, cudaStream_t st) {
+    hybrid_gemm2_kernel<<<2 * clusters, kThreads, kSmemBytes, st>>>(tmap_x, tm_a16, tm_a8, tm_e, a);
+    return cudaGetLastError();
+}
+
+}  // namespace patch

@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(256) hybrid_gemv_kernel(const GemvArgs a) {
     const int s = blockIdx.x >> 3, h = blockIdx.x & 7;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = lane & 7, rg = lane >> 3;
-    const uint32_t* trow = a.table + (size_t)s * a.KB;
+    const uint32_t* trow = a.slab + (size_t)s * a.KB;
+    const uint32_t* mrow = a.meta + (size_t)s * a.KC;
 
     float acc[4][MT];
 #pragma unroll
@@ -75,9 +76,7 @@ __global__ void __launch_bounds__(256) hybrid_gemv_kernel(const GemvArgs a) {
                 }
             }
         } else {
-            const uint8_t* meta = (d & kSlabHasMeta)
-                                      ? base + kSparseValBytes
-                                      : a.packed + slab_offset_bytes(__ldg(trow + b - 1)) + kSparseValBytes;
+            const uint8_t* meta = a.packed + (uint64_t)__ldg(mrow + (b >> 1)) * 16;
             const int kc = (b & 1) * kSlabK + 8 * L;
             uint2 cv[4];
             uint32_t code8[4];

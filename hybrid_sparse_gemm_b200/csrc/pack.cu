@@ -1,12 +1,13 @@
 // Pack and unpack kernels: bit-packed keep/prune mask + frozen bf16 weights ->
-// per-slab dense blocks or compressed 2:4 values with 2-bit position codes.
+// per-slab dense blocks or compressed 2:4 values, 2-bit position codes, and
+// dense images of 2:4 slabs whose partner strip is dense.
 //
 // Semantics: the PATCH model cards ("llama_3.2_1b-PATCH-45Sparse", release
 // paragraph and "How to use") ship only a bit-packed keep/prune mask and apply
 // it by zeroing pruned weights; each tile is dense or 2:4 (method paragraph).
-// The stored layout is this library's own; it is the shared-memory image the
-// tcgen05 GEMM feeds to the tensor core, so the GEMM loads it with plain bulk
-// copies.
+// The stored layout is this library's own: every record is the shared-memory
+// image the tcgen05 kernels feed to the tensor core, so they load records
+// with plain bulk or TMA copies.
 #include "kernels.cuh"
 
 namespace patch {
@@ -17,22 +18,48 @@ __device__ __forceinline__ int keep_bit(uint32_t byte, int e, int bitorder) {
     return bitorder == 0 ? (byte >> (7 - e)) & 1 : (byte >> e) & 1;
 }
 
-// Metadata block of the 128-column chunk containing slab b, or nullptr.
-__device__ __forceinline__ uint8_t* chunk_meta(const PackArgs& a, int s, int b) {
-    const int c0 = b & ~1;
-    const uint32_t d0 = a.table[s * a.KB + c0];
-    if ((d0 & 3u) == 3u) return a.out + slab_offset_bytes(d0) + kSparseValBytes;
-    if (c0 + 1 < a.KB) {
-        const uint32_t d1 = a.table[s * a.KB + c0 + 1];
-        if ((d1 & 3u) == 3u) return a.out + slab_offset_bytes(d1) + kSparseValBytes;
-    }
-    return nullptr;
-}
-
-// Zero the two metadata words (columns j, j+1) of every lane.
+// Zero the two metadata words (columns j, j+1) of every lane of a block.
 __device__ __forceinline__ void zero_meta_words(uint8_t* meta, int j) {
     for (int lane = threadIdx.x; lane < 128; lane += blockDim.x)
         *reinterpret_cast<uint2*>(meta + lane * 16 + j * 4) = make_uint2(0u, 0u);
+}
+
+// Dense image of slab (s, b) of W (.) Mask at dst. When `count` is set the
+// validation counters are updated (groups of 2:4-flagged tiles, stray zeros).
+__device__ void write_dense(const PackArgs& a, int s, int b, uint8_t* dst, bool count,
+                            unsigned long long& bad, unsigned long long& stray, unsigned long long& pruned) {
+    const int64_t K = a.K;
+    const int tiles_k = (int)(K / a.C);
+    for (int q = threadIdx.x; q < 1024; q += blockDim.x) {
+        const int r = q >> 3, L = (q & 7) ^ (r & 7);
+        const int64_t n = (int64_t)s * kStrip + r;
+        const int64_t k = (int64_t)b * kSlabK + 8 * L;
+        const int64_t e0 = n * K + k;  // multiple of 8: one mask byte
+        uint4 w = *reinterpret_cast<const uint4*>(a.W + e0);
+        const uint32_t mb = a.bits[e0 >> 3];
+        uint16_t h[8];
+        memcpy(h, &w, 16);
+        int kept = 0;
+        for (int e = 0; e < 8; ++e) {
+            const int kb = keep_bit(mb, e, a.bitorder);
+            kept += kb;
+            if (!kb) h[e] = 0;
+        }
+        if (count) {
+            pruned += 8 - kept;
+            if (a.flags[(n / a.R) * tiles_k + (k / a.C)]) {
+                for (int g = 0; g < 2; ++g) {
+                    int c = 0;
+                    for (int e = 4 * g; e < 4 * g + 4; ++e) c += keep_bit(mb, e, a.bitorder);
+                    bad += (c != 2);
+                }
+            } else {
+                stray += 8 - kept;
+            }
+        }
+        memcpy(&w, h, 16);
+        *reinterpret_cast<uint4*>(dst + sw128_off(r, L)) = w;
+    }
 }
 
 }  // namespace
@@ -44,48 +71,18 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
 
     const int s = blockIdx.x / a.KB;
     const int b = blockIdx.x % a.KB;
-    const uint32_t d = a.table[blockIdx.x];
+    const uint32_t d = a.slab[blockIdx.x];
     uint8_t* base = a.out + slab_offset_bytes(d);
-    const int64_t K = a.K;
-    const int tiles_k = (int)(K / a.C);
+    const uint32_t mo = a.meta[s * a.KC + (b >> 1)];
+    uint8_t* meta = (mo == kNoMeta) ? nullptr : a.out + (uint64_t)mo * 16;
     unsigned long long bad = 0, stray = 0, pruned = 0;
 
     if (!(d & kSlabSparse)) {
-        // 1024 chunks of 16 bytes: row r, swizzled chunk p holds columns 8L..8L+7.
-        for (int q = threadIdx.x; q < 1024; q += blockDim.x) {
-            const int r = q >> 3, p = q & 7, L = p ^ (r & 7);
-            const int64_t n = (int64_t)s * kStrip + r;
-            const int64_t k = (int64_t)b * kSlabK + 8 * L;
-            const int64_t e0 = n * K + k;  // multiple of 8: one mask byte
-            uint4 w = *reinterpret_cast<const uint4*>(a.W + e0);
-            const uint32_t mb = a.bits[e0 >> 3];
-            uint16_t h[8];
-            memcpy(h, &w, 16);
-            int kept = 0;
-            for (int e = 0; e < 8; ++e) {
-                const int kb = keep_bit(mb, e, a.bitorder);
-                kept += kb;
-                if (!kb) h[e] = 0;
-            }
-            pruned += 8 - kept;
-            const bool tile_sparse = a.flags[(n / a.R) * tiles_k + (k / a.C)] != 0;
-            if (tile_sparse) {
-                for (int g = 0; g < 2; ++g) {
-                    int c = 0;
-                    for (int e = 4 * g; e < 4 * g + 4; ++e) c += keep_bit(mb, e, a.bitorder);
-                    bad += (c != 2);
-                }
-            } else {
-                stray += 8 - kept;
-            }
-            memcpy(&w, h, 16);
-            *reinterpret_cast<uint4*>(base + sw128_off(r, L)) = w;
-        }
+        write_dense(a, s, b, base, true, bad, stray, pruned);
         // A dense slab in a chunk that has a metadata block zeroes its columns.
-        uint8_t* meta = chunk_meta(a, s, b);
         if (meta) zero_meta_words(meta, (b & 1) * 2);
     } else {
-        uint8_t* meta = chunk_meta(a, s, b);
+        const int64_t K = a.K;
         // 512 items: row r, logical 16-column quarter L (4 groups, 8 kept values).
         for (int q = threadIdx.x; q < 512; q += blockDim.x) {
             const int r = q >> 2, L = q & 3;
@@ -122,9 +119,16 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
             *reinterpret_cast<uint16_t*>(meta + meta_lane(r, kc) * 16 + (kc >> 5) * 4 +
                                          (meta_bit(r, kc) >> 3)) = (uint16_t)code;
         }
-        // The first slab of a chunk that has no partner slab (K % 128 == 64)
+        // The first slab of a chunk without a partner slab (K % 128 == 64)
         // zeroes the partner's columns.
         if (!(b & 1) && b + 1 >= a.KB) zero_meta_words(meta, 2);
+        // A 2:4 slab whose partner strip is dense also gets a dense image for
+        // the CTA-pair kernel.
+        const uint32_t g = a.gemm[blockIdx.x];
+        if (!(g & kSlabSparse)) {
+            unsigned long long x0 = 0, x1 = 0, x2 = 0;
+            write_dense(a, s, b, a.out + slab_offset_bytes(g), false, x0, x1, x2);
+        }
     }
 
     // block reduction of the counters
@@ -142,13 +146,14 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
     if (threadIdx.x < 3 && s_cnt[threadIdx.x]) atomicAdd(&a.counters[threadIdx.x], s_cnt[threadIdx.x]);
 }
 
-// Decode packed slabs back to W (.) Mask, row-major N x K.
+// Decode the per-strip records back to W (.) Mask, row-major N x K.
 __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed,
-                                                     const uint32_t* __restrict__ table, int KB,
+                                                     const uint32_t* __restrict__ slab,
+                                                     const uint32_t* __restrict__ meta_tab, int KB, int KC,
                                                      int64_t K, uint16_t* __restrict__ Wm) {
     const int s = blockIdx.x / KB;
     const int b = blockIdx.x % KB;
-    const uint32_t d = table[blockIdx.x];
+    const uint32_t d = slab[blockIdx.x];
     const uint8_t* base = packed + slab_offset_bytes(d);
     if (!(d & kSlabSparse)) {
         for (int q = threadIdx.x; q < 1024; q += blockDim.x) {
@@ -159,9 +164,7 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
         }
         return;
     }
-    const uint8_t* meta = (d & kSlabHasMeta) ? base + kSparseValBytes
-                                              : packed + slab_offset_bytes(table[blockIdx.x - 1]) +
-                                                    kSparseValBytes;
+    const uint8_t* meta = packed + (uint64_t)meta_tab[s * KC + (b >> 1)] * 16;
     for (int q = threadIdx.x; q < 512; q += blockDim.x) {
         const int r = q >> 2, L = q & 3;
         const int64_t n = (int64_t)s * kStrip + r;

@@ -55,8 +55,10 @@ typedef enum {
 /* Which kernel patch_linear_path runs. AUTO picks by M. */
 typedef enum {
     PATCH_PATH_AUTO = 0,
-    PATCH_PATH_GEMM = 1,  /* tcgen05 tensor-core kernel (TMA, TMEM accumulators) */
-    PATCH_PATH_GEMV = 2   /* CUDA-core kernel for decode-sized M (M <= 16) */
+    PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core kernel, variant chosen by M */
+    PATCH_PATH_GEMV = 2,         /* CUDA-core kernel for decode-sized M (M <= 16) */
+    PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
+    PATCH_PATH_GEMM_PAIR = 4     /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
 } patch_path;
 
 typedef struct {
@@ -66,6 +68,9 @@ typedef struct {
     int64_t tiles_sparse;       /* tiles flagged 2:4 */
     int64_t slabs_total;        /* (N/128) * (K/64) storage slabs */
     int64_t slabs_sparse;       /* slabs stored compressed */
+    int64_t slabs_pair_sparse;  /* slabs the CTA-pair kernel runs on the sparse MMA */
+    int64_t meta_blocks;        /* 2048-byte metadata blocks */
+    int64_t dense_images;       /* dense images of 2:4 slabs whose partner strip is dense */
     int64_t packed_bytes;       /* device bytes of the packed weights */
     int64_t pruned;             /* mask zeros over all N*K elements */
     int64_t stray_zeros;        /* mask zeros inside tiles flagged dense */
@@ -102,17 +107,20 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
                         int tile_cols, void* stream, patch_handle* out);
 
 /*
- * patch_plan - the slab table and packed size patch_pack would produce for
- * these tile flags, computed on the host without touching any device.
+ * patch_plan - the tables and packed size patch_pack would produce for these
+ * tile flags, computed on the host without touching any device.
  *
  *   N, K, tile_flags, tile_rows, tile_cols  as for patch_pack.
- *   table_host    host, (N/128)*(K/64) uint32 (layout as for
- *                 patch_copy_packed), or NULL.
+ *   slab_table  host, (N/128)*(K/64) uint32, or NULL.
+ *   meta_table  host, (N/128)*ceil(K/128) uint32, or NULL.
+ *   gemm_table  host, (N/128)*(K/64) uint32, or NULL.
  *   packed_bytes  receives the device bytes of the packed weights, or NULL.
- * Same shape rules and errors as patch_pack; no mask is read.
+ * Table layouts: see patch_copy_packed. Same shape rules and errors as
+ * patch_pack; no mask is read.
  */
 patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
-                        uint32_t* table_host, int64_t* packed_bytes);
+                        uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table,
+                        int64_t* packed_bytes);
 
 /*
  * patch_linear - Y = X . (W (.) Mask)^T for the packed weights of h.
@@ -129,7 +137,7 @@ patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y
                           void* stream);
 
 /* patch_linear with an explicit kernel choice (patch_path). GEMV requires
- * M <= 16. */
+ * M <= 16. Any M works on the tensor-core variants. */
 patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                                int path, void* stream);
 
@@ -152,15 +160,24 @@ patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream);
 patch_status patch_info(patch_handle h, patch_info_t* info);
 
 /*
- * patch_copy_packed - copy the packed bytes and the slab table to the host.
- *   packed_host  host, packed_cap bytes (>= info.packed_bytes) or NULL.
- *   table_host   host, table_cap uint32 (>= info.slabs_total) or NULL.
- * Table entry per (strip s, slab b), index s*(K/64)+b:
- *   (byte_offset/16) << 2 | has_metadata << 1 | sparse.
+ * patch_copy_packed - copy the packed bytes and the three tables to the host.
+ *   packed_host  host, packed_cap bytes (>= info.packed_bytes), or NULL.
+ *   slab_host, meta_host, gemm_host  host tables with their capacities in
+ *                entries, or NULL. A too-small buffer gives PATCH_ERR_ARG.
+ * With S = N/128 strips, KB = K/64 slabs and KC = ceil(KB/2) chunks:
+ *   slab[s*KB+b] = (offset/16)<<2 | first<<1 | sparse: the slab's own record,
+ *     a 16384-byte dense block or 8192 bytes of kept 2:4 values; first marks
+ *     the first 2:4 slab of its 128-column chunk.
+ *   meta[s*KC+c] = offset/16 of the chunk's 2048-byte metadata block, or
+ *     0xFFFFFFFF when the chunk has no 2:4 slab.
+ *   gemm[s*KB+b] = (offset/16)<<2 | first<<1 | pair_sparse: the record the
+ *     CTA-pair kernel loads (strips 2p and 2p+1 agree on every slab; a 2:4
+ *     slab whose partner is dense points at its dense image).
  * Synchronous.
  */
 patch_status patch_copy_packed(patch_handle h, void* packed_host, int64_t packed_cap,
-                               uint32_t* table_host, int64_t table_cap);
+                               uint32_t* slab_host, int64_t slab_cap, uint32_t* meta_host,
+                               int64_t meta_cap, uint32_t* gemm_host, int64_t gemm_cap);
 
 /*
  * patch_check - synchronise the stream and report device-side failures of

@@ -40,7 +40,7 @@ def test_exports_every_header_symbol(hsg):
 
 
 def test_version(hsg):
-    assert hsg.version() == 1
+    assert hsg.version() == 2
 
 
 def _pack_status(hsg, W=0x1000, N=256, K=256, bits=0x2000, bitorder=0, flags=None, R=128, C=128):
@@ -73,6 +73,8 @@ def test_linear_rejects_bad_arguments(hsg):
     assert lib.patch_linear_host(None, 0x1000, 4, 0x2000, None) == 1
     assert lib.patch_unpack(None, 0x1000, None) == 1
     assert lib.patch_check(None, None) == 1
+    assert lib.patch_copy_packed(None, None, 0, None, 0, None, 0, None, 0) == 1
+    assert lib.patch_linear_path(None, 0x1000, 4, 0x2000, 9, None) == 1
     info = hsg.patch_info_t()
     assert lib.patch_info(None, ctypes.byref(info)) == 1
     lib.patch_free(None)  # ignored
@@ -90,26 +92,29 @@ def test_pack_without_device_reports_cuda_or_unsupported(hsg):
 
 @pytest.mark.parametrize("R,C", [(128, 128), (128, 64), (64, 128), (64, 64)])
 @pytest.mark.parametrize("N,K,frac", [(256, 384, 0.5), (512, 448, 0.9), (128, 64, 1.0),
-                                      (384, 1024, 0.0), (1024, 512, 0.3)])
-def test_plan_matches_oracle_table(hsg, oracle_lib, R, C, N, K, frac):
+                                      (384, 1024, 0.0), (1024, 512, 0.3), (640, 320, 0.7)])
+def test_plan_matches_oracle_tables(hsg, oracle_lib, R, C, N, K, frac):
     if N % R or K % C:
         pytest.skip("shape not divisible by tile")
     flags = synth.tile_flags(N, K, R, C, frac, "plan").numpy().reshape(-1)
-    table, nbytes = hsg.patch_plan(N, K, flags, R, C)
-    otable, obytes = oracle_lib.pack_table(N, K, flags, R, C)
-    assert nbytes == obytes
-    assert np.array_equal(table.numpy().astype(np.uint32), otable)
+    (slab, meta, gemm), nbytes = hsg.patch_plan(N, K, flags, R, C)
+    t = oracle_lib.pack_table(N, K, flags, R, C)
+    assert nbytes == t.nbytes
+    assert np.array_equal(slab, t.slab)
+    assert np.array_equal(meta, t.meta)
+    assert np.array_equal(gemm, t.gemm)
 
 
 def test_plan_checkerboard_and_llama_sizes(hsg, oracle_lib):
     # checkerboard of 64x64 tiles: no 128x64 slab is all-2:4, so nothing compresses
     N, K = 256, 256
     fl = np.indices((N // 64, K // 64)).sum(0) % 2
-    table, nbytes = hsg.patch_plan(N, K, fl.astype(np.uint8), 64, 64)
-    assert nbytes == N * K * 2 and int((table & 1).sum()) == 0
-    # all-2:4 Llama-3.2-1B q projection: 1.125 bytes per weight
-    table, nbytes = hsg.patch_plan(2048, 2048, np.ones(256, np.uint8), 128, 128)
+    (slab, meta, gemm), nbytes = hsg.patch_plan(N, K, fl.astype(np.uint8), 64, 64)
+    assert nbytes == N * K * 2 and int((slab & 1).sum()) == 0 and (meta == 0xFFFFFFFF).all()
+    # all-2:4 Llama-3.2-1B q projection: 1.125 bytes per weight, no dense images
+    (slab, meta, gemm), nbytes = hsg.patch_plan(2048, 2048, np.ones(256, np.uint8), 128, 128)
     assert nbytes == 2048 * 2048 * 9 // 8
+    assert np.array_equal(slab, gemm)
 
 
 def test_plan_errors(hsg):

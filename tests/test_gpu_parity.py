@@ -60,12 +60,12 @@ def pack(hsg, p):
 
 
 def check_pack(hsg, oracle_lib, p, lin):
-    packed, table = lin.packed()
+    packed, (slab, meta, gemm) = lin.packed()
     keep = p.keep.cpu().numpy().astype(np.uint8)
     op, ot = oracle_lib.pack(p.W.cpu(), keep, p.flags.cpu().numpy().reshape(-1), p.R, p.C)
-    assert np.array_equal(table.numpy().astype(np.uint32), ot)
-    assert packed.numel() == op.size
-    diff = np.flatnonzero(packed.numpy() != op)
+    assert np.array_equal(slab, ot.slab) and np.array_equal(meta, ot.meta) and np.array_equal(gemm, ot.gemm)
+    assert packed.size == op.size
+    diff = np.flatnonzero(packed != op)
     assert diff.size == 0, f"{diff.size} packed bytes differ, first at {diff[:8]}"
 
 
@@ -74,8 +74,9 @@ def check_pack(hsg, oracle_lib, p, lin):
 @pytest.mark.parametrize("R,C", [(128, 128), (128, 64), (64, 128), (64, 64)])
 @pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
 @pytest.mark.parametrize("bitorder", [0, 1])
-def test_pack_bit_exact(hsg, oracle_lib, R, C, frac, bitorder):
-    N, K = 256, (448 if C == 64 else 384)
+@pytest.mark.parametrize("N", [256, 384])
+def test_pack_bit_exact(hsg, oracle_lib, R, C, frac, bitorder, N):
+    K = 448 if C == 64 else 384
     p = synth.make_problem(N, K, 0, R=R, C=C, frac=frac, seed=7, device="cuda", bitorder=bitorder)
     lin = pack(hsg, p)
     check_pack(hsg, oracle_lib, p, lin)
@@ -121,16 +122,38 @@ def test_stray_zeros_in_dense_tiles(hsg, oracle_lib):
 SMALL = [(256, 384, 128, 128), (384, 448, 128, 64), (256, 512, 64, 128), (384, 320, 64, 64)]
 
 
-@pytest.mark.parametrize("N,K,R,C", SMALL)
+SMALL_ODD = SMALL + [(640, 320, 128, 64), (128, 256, 128, 128)]  # odd strip counts
+
+
+@pytest.mark.parametrize("N,K,R,C", SMALL_ODD)
 @pytest.mark.parametrize("frac", [0.0, 0.6, 1.0])
 @pytest.mark.parametrize("M", [1, 5, 16, 17, 128, 129, 300])
-def test_gemm_small(hsg, oracle_lib, N, K, R, C, frac, M):
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+def test_gemm_small(hsg, oracle_lib, N, K, R, C, frac, M, kernel):
     p = synth.make_problem(N, K, M, R=R, C=C, frac=frac, seed=M, device="cuda")
     lin = pack(hsg, p)
-    Y = lin(p.X, path=hsg.PATH_GEMM)
+    path = hsg.PATH_GEMM_SINGLE if kernel == "single" else hsg.PATH_GEMM_PAIR
+    Y = lin(p.X, path=path)
     torch.cuda.synchronize()
     lin.check()
-    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"gemm M={M}")
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"{kernel} M={M}")
+    lin.free()
+
+
+@pytest.mark.parametrize("M", [256, 511, 700, 1024])
+@pytest.mark.parametrize("frac", [0.3, 0.9])
+def test_pair_tiles_several_blocks(hsg, oracle_lib, M, frac):
+    """Several 256-token blocks and strip pairs per CTA pair, mixed kinds in a pair."""
+    p = synth.make_problem(1152, 1024, M, R=128, C=128, frac=frac, seed=M, device="cuda")
+    lin = pack(hsg, p)
+    info = lin.info()
+    assert info.dense_images == info.slabs_sparse - info.slabs_pair_sparse
+    for path in (hsg.PATH_GEMM_PAIR, hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM):
+        Y = lin(p.X, path=path)
+        torch.cuda.synchronize()
+        lin.check()
+        assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(M, 96, M),
+                     what=f"pair blocks path {path}")
     lin.free()
 
 
@@ -150,7 +173,7 @@ def test_single_strip_single_slab(hsg, oracle_lib):
     for frac in (0.0, 1.0):
         p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")
         lin = pack(hsg, p)
-        for path in (hsg.PATH_GEMM, hsg.PATH_GEMV):
+        for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV):
             Y = lin(p.X, path=path)
             torch.cuda.synchronize()
             assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"single slab {path}")
@@ -165,7 +188,7 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
     bits = synth.pack_bits(keep)
     X = synth.normal_bf16((40, K), 1.0, "cuda", "zero", "X")
     lin = hsg.PackedLinear.pack(W, bits, fl, 64, 64)
-    for path, M in ((hsg.PATH_GEMM, 40), (hsg.PATH_GEMV, 16)):
+    for path, M in ((hsg.PATH_GEMM_SINGLE, 40), (hsg.PATH_GEMM_PAIR, 40), (hsg.PATH_GEMV, 16)):
         Y = lin(X[:M].contiguous(), path=path)
         torch.cuda.synchronize()
         assert torch.count_nonzero(Y.float()) == 0
@@ -176,16 +199,17 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
     bits = synth.pack_bits(keep)
     lin = hsg.PackedLinear.pack(p.W, bits, fl, 64, 64)
     assert lin.info().slabs_sparse == 0
-    Y = lin(p.X, path=hsg.PATH_GEMM)
-    torch.cuda.synchronize()
-    assert_close(Y, oracle_lib, p.X, p.W, bits, keep, what="checkerboard")
+    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR):
+        Y = lin(p.X, path=path)
+        torch.cuda.synchronize()
+        assert_close(Y, oracle_lib, p.X, p.W, bits, keep, what="checkerboard")
     lin.free()
 
 
 def test_one_sparse_tile(hsg, oracle_lib):
     p = synth.make_problem(512, 512, 50, R=128, C=128, n_sparse=1, seed=5, device="cuda")
     lin = pack(hsg, p)
-    for path, M in ((hsg.PATH_GEMM, 50), (hsg.PATH_GEMV, 16)):
+    for path, M in ((hsg.PATH_GEMM_SINGLE, 50), (hsg.PATH_GEMM_PAIR, 50), (hsg.PATH_GEMV, 16)):
         X = p.X[:M].contiguous()
         Y = lin(X, path=path)
         torch.cuda.synchronize()
@@ -212,10 +236,13 @@ def test_empty_and_misaligned(hsg):
 def test_deterministic_and_host_path(hsg):
     p = synth.make_problem(512, 1024, 300, R=128, C=64, frac=0.7, seed=8, device="cuda")
     lin = pack(hsg, p)
-    Y1 = lin(p.X, path=hsg.PATH_GEMM)
-    Y2 = lin(p.X, path=hsg.PATH_GEMM)
+    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMM):
+        Ya = lin(p.X, path=path)
+        Yb = lin(p.X, path=path)
+        torch.cuda.synchronize()
+        assert torch.equal(Ya, Yb)
+    Y1 = lin(p.X)
     torch.cuda.synchronize()
-    assert torch.equal(Y1, Y2)
     Yh = lin.host(p.X.cpu().pin_memory())
     assert torch.equal(Yh, Y1.cpu())
     Xs = p.X[:5].contiguous()
@@ -230,7 +257,7 @@ def test_gemm_and_gemv_agree_with_oracle_on_config_1(hsg, oracle_lib):
     lin = pack(hsg, p)
     check_pack(hsg, oracle_lib, p, lin)
     assert abs(lin.info().sparsity - 0.25) < 1e-12
-    for path in (hsg.PATH_GEMM, hsg.PATH_GEMV, hsg.PATH_AUTO):
+    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV, hsg.PATH_AUTO):
         Y = lin(p.X, path=path)
         torch.cuda.synchronize()
         assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"config1 {path}")
