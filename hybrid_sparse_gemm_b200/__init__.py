@@ -17,7 +17,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpatch_hybrid.so")
+LIB_PATH = os.environ.get("PATCH_HYBRID_LIB") or os.path.join(_HERE, "libpatch_hybrid.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hybrid_sparse_gemm_b200.build`")
