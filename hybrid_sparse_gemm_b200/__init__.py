@@ -32,7 +32,7 @@ PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR = 0, 1, 2, 3, 
 
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
-            "patch_version", "patch_plan"]
+            "patch_version", "patch_plan", "patch_linear_noalloc"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -52,6 +52,7 @@ _lib.patch_pack.argtypes = [_P, _I64, _I64, _P, _I, _P, _I, _I, _P, ctypes.POINT
 _lib.patch_linear.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_linear_path.argtypes = [_P, _P, _I64, _P, _I, _P]
 _lib.patch_linear_host.argtypes = [_P, _P, _I64, _P, _P]
+_lib.patch_linear_noalloc.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_unpack.argtypes = [_P, _P, _P]
 _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]
 _lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
@@ -62,7 +63,7 @@ _lib.patch_free.restype = None
 _lib.patch_last_error.restype = ctypes.c_char_p
 _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
-           "patch_info", "patch_copy_packed", "patch_check", "patch_plan"]:
+           "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -131,6 +132,11 @@ def patch_linear_path(h: int, X: torch.Tensor, Y: torch.Tensor, path: int = PATH
 
 def patch_linear(h: int, X: torch.Tensor, Y: torch.Tensor, stream=None):
     _check(_lib.patch_linear(h, X.data_ptr(), X.shape[0], Y.data_ptr(), _stream(stream)))
+
+
+def patch_linear_noalloc(h: int, X: torch.Tensor, Y: torch.Tensor, stream=None):
+    """patch_linear that allocates no device memory (see the header)."""
+    _check(_lib.patch_linear_noalloc(h, X.data_ptr(), X.shape[0], Y.data_ptr(), _stream(stream)))
 
 
 def patch_linear_host(h: int, X: torch.Tensor, Y: torch.Tensor, stream=None):

@@ -629,3 +629,152 @@ patch_status patch_check(patch_handle h, void* stream) {
 void patch_free(patch_handle h) { free_handle(h); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of patch_linear.
+//
+// The tensor-core kernels read their per-launch schedule (which output tiles
+// each persistent CTA or CTA pair takes) from device memory that patch_linear
+// allocates and caches per handle on the first call for each M. Callers that
+// must not allocate device memory during the call (an allocator that is frozen
+// after start-up, a memory pool owned by another framework, a host thread
+// that may not touch the CUDA allocator) use patch_linear_noalloc instead: it
+// writes the schedule into one fixed array that lives in this library's
+// device image, so the call itself allocates nothing.
+namespace {
+
+constexpr int kNoAllocMaxSlots = 256;      // persistent CTAs or CTA pairs
+constexpr int kNoAllocMaxUnits = 65536;    // output tiles of one call
+constexpr int kNoAllocInts = (kNoAllocMaxSlots + 1) + kNoAllocMaxUnits;
+
+// Schedule scratch shared by every call on a device: [0, slots] offsets, then
+// the tile list. Host code must not pass this symbol to a kernel: its device
+// address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) int g_noalloc_sched[kNoAllocInts];
+
+std::mutex g_noalloc_mu;
+std::map<int, int*> g_noalloc_addr;  // device -> device address of g_noalloc_sched
+
+patch_status noalloc_scratch(int dev, int** out) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_addr.find(dev);
+    if (it == g_noalloc_addr.end()) {
+        int* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_sched);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the schedule scratch");
+        it = g_noalloc_addr.emplace(dev, p).first;
+    }
+    *out = it->second;
+    return PATCH_OK;
+}
+
+// Same greedy LPT rule as the cached schedules, on the host only.
+void noalloc_schedule(patch_handle h, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
+    const std::vector<double>& cost = kernel == 0 ? h->plan.strip_cost : h->plan.pair_cost;
+    const int units = (int)cost.size() * mb;
+    const int slots = kernel == 0 ? h->dev.sms : h->dev.pair_clusters;
+    const int grid = std::max(1, std::min(slots, units));
+    std::vector<int> order(units);
+    for (int u = 0; u < units; ++u) order[u] = u;
+    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x / mb] > cost[y / mb]; });
+    using Item = std::pair<double, int>;
+    std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
+    for (int c = 0; c < grid; ++c) pq.push({0.0, c});
+    std::vector<std::vector<int>> lists(grid);
+    for (int u : order) {
+        Item top = pq.top();
+        pq.pop();
+        lists[top.second].push_back(u);
+        top.first += cost[u / mb] + 1.0;
+        pq.push(top);
+    }
+    off.assign(grid + 1, 0);
+    work.clear();
+    for (int c = 0; c < grid; ++c) {
+        off[c] = (int)work.size();
+        work.insert(work.end(), lists[c].begin(), lists[c].end());
+    }
+    off[grid] = (int)work.size();
+}
+
+}  // namespace
+
+extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
+                                             void* stream) {
+    if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
+    if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
+    if (M == 0) return PATCH_OK;
+    if (!X_bf16 || !Y_bf16) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
+    if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
+    if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Decode sizes use no scratch at all.
+    if (M <= 8) {
+        patch_status s = check_handle_device(h);
+        if (s != PATCH_OK) return s;
+        return run_linear(h, X_bf16, M, Y_bf16, PATCH_PATH_GEMV, st);
+    }
+    const bool pair = M >= kPairMinM;
+    const int bn = pair ? kGemm2BN : kGemmBN;
+    const int64_t mb = (M + bn - 1) / bn;
+    const int64_t rows = pair ? (int64_t)h->plan.pair_cost.size() : (int64_t)h->plan.strip_cost.size();
+    const int slots = pair ? h->dev.pair_clusters : h->dev.sms;
+    if (rows * mb > kNoAllocMaxUnits || slots > kNoAllocMaxSlots)
+        return fail(PATCH_ERR_SHAPE,
+                    "patch_linear_noalloc handles at most %d output tiles per call (this call needs %lld); "
+                    "use patch_linear",
+                    kNoAllocMaxUnits, (long long)(rows * mb));
+    int dev = -1;
+    PATCH_CUDA(cudaGetDevice(&dev));
+    if (dev != h->device) return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", h->device, dev);
+    int* sched = nullptr;
+    patch_status s = noalloc_scratch(dev, &sched);
+    if (s != PATCH_OK) return s;
+    std::vector<int> off, work;
+    noalloc_schedule(h, pair ? 1 : 0, (int)mb, off, work);
+    const int grid = (int)off.size() - 1;
+    int* d_off = sched;
+    int* d_work = sched + kNoAllocMaxSlots + 1;
+    PATCH_CUDA(cudaMemcpyAsync(d_off, off.data(), sizeof(int) * off.size(), cudaMemcpyHostToDevice, st));
+    PATCH_CUDA(cudaMemcpyAsync(d_work, work.data(), sizeof(int) * std::max<size_t>(work.size(), 1),
+                               cudaMemcpyHostToDevice, st));
+    CUtensorMap map;
+    if (!pair) {
+        s = encode_2d(&map, X_bf16, h->K, M, kSlabK, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s != PATCH_OK) return s;
+        GemmArgs a;
+        a.packed = h->packed;
+        a.slab = h->slab_dev;
+        a.meta = h->meta_dev;
+        a.work_off = d_off;
+        a.work = d_work;
+        a.M = (int)M;
+        a.N = (int)h->N;
+        a.KB = h->plan.KB;
+        a.KC = h->plan.KC;
+        a.MB = (int)mb;
+        a.Y = static_cast<__nv_bfloat16*>(Y_bf16);
+        a.status = h->status_dev;
+        cudaError_t e = launch_gemm(map, a, grid, st);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+        return PATCH_OK;
+    }
+    s = encode_2d(&map, X_bf16, h->K, M, kSlabK, kGemm2BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != PATCH_OK) return s;
+    Gemm2Args a;
+    a.gemm = h->gemm_dev;
+    a.meta = h->meta_dev;
+    a.work_off = d_off;
+    a.work = d_work;
+    a.M = (int)M;
+    a.N = (int)h->N;
+    a.S = h->plan.S;
+    a.KB = h->plan.KB;
+    a.KC = h->plan.KC;
+    a.MB = (int)mb;
+    a.Y = static_cast<__nv_bfloat16*>(Y_bf16);
+    a.status = h->status_dev;
+    cudaError_t e = launch_gemm2(map, h->tm_a16, h->tm_a8, h->tm_e, a, grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "CTA-pair tensor-core kernel launch");
+    return PATCH_OK;
+}

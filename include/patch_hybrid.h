@@ -152,6 +152,31 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
 patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, void* Y_host,
                                void* stream);
 
+/*
+ * patch_linear_noalloc - patch_linear for callers that cannot allocate device
+ * memory during the call.
+ *
+ * The pages describe no counterpart; this entry point exists for deployment.
+ * patch_linear uploads each new M's tile schedule into device memory it
+ * allocates on first use. Callers whose device memory is owned by someone
+ * else (a frozen allocator, another framework's memory pool, a thread that
+ * may not call cudaMalloc) use this call instead: it allocates nothing and
+ * keeps the schedule in one fixed array inside this library's device image,
+ * sized for at most 65536 output tiles per call (256-token tiles for
+ * M >= 256, 128-token tiles below; PATCH_ERR_SHAPE beyond that). Every GPU
+ * that loads the library holds that array (about 257 KiB) until the process
+ * exits.
+ *
+ *   Arguments, layouts and results as for patch_linear (AUTO path).
+ * The first call on a device looks up the array's device address; make that
+ * first call before capturing later calls in a CUDA graph. All calls share
+ * the one array and each overwrites it, so calls that overlap on the GPU
+ * (different streams, or several handles at once) race: order them on one
+ * stream or synchronise between them.
+ */
+patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
+                                  void* stream);
+
 /* patch_unpack - write W (.) Mask (N*K bf16, dev, row-major, 16-byte aligned)
  * decoded from the packed weights. */
 patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream);
