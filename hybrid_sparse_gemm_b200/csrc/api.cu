@@ -91,6 +91,7 @@ patch_status prepare_device(int* dev_out, DeviceInfo* info_out) {
         di.sms = sms;
         PATCH_CUDA(gemm_prepare_single());
         PATCH_CUDA(gemm_prepare_pair(&di.pair_clusters));
+        PATCH_CUDA(decode_prepare());
         if (di.pair_clusters <= 0) di.pair_clusters = 1;
         it = g_dev.emplace(dev, di).first;
     }
@@ -142,6 +143,7 @@ struct Plan {
     int S = 0, KB = 0, KC = 0;
     std::vector<uint32_t> slab, meta, gemm;
     std::vector<double> strip_cost, pair_cost;
+    std::vector<double> strip_bytes;  // bytes the decode kernel streams per strip
     int64_t bytes = 0, sparse = 0, pair_sparse = 0, meta_blocks = 0, images = 0;
 };
 
@@ -168,6 +170,7 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
     p.gemm.assign((size_t)p.S * p.KB, 0u);
     p.strip_cost.assign(p.S, 0.0);
     p.pair_cost.assign((p.S + 1) / 2, 0.0);
+    p.strip_bytes.assign(p.S, 0.0);
     int64_t off = 0;
     for (int s = 0; s < p.S; ++s)
         for (int b = 0; b < p.KB; ++b) {
@@ -178,6 +181,7 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
             off += x ? kSparseValBytes : kDenseSlabBytes;
             p.sparse += x;
             p.strip_cost[s] += x ? 0.5 : 1.0;
+            p.strip_bytes[s] += x ? kSparseValBytes : kDenseSlabBytes;
         }
     for (int s = 0; s < p.S; ++s)
         for (int c = 0; c < p.KC; ++c) {
@@ -186,6 +190,7 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
                 p.meta[(size_t)s * p.KC + c] = (uint32_t)(off / 16);
                 off += kMetaBytes;
                 ++p.meta_blocks;
+                p.strip_bytes[s] += kMetaBytes;
             }
         }
     for (int s = 0; s < p.S; ++s)
@@ -221,6 +226,9 @@ struct patch_handle_s {
     uint32_t* meta_dev = nullptr;
     uint32_t* gemm_dev = nullptr;
     int* status_dev = nullptr;
+    int decode_parts = 1;              // K-parts per strip for the decode kernel
+    float* decode_partial = nullptr;   // [S][parts][128][16] fp32 workspace
+    unsigned* decode_counters = nullptr;  // [S], zero between calls
     CUtensorMap tm_a16, tm_a8, tm_e;
     patch_info_t info{};
     std::mutex mu;
@@ -241,6 +249,8 @@ void free_handle(patch_handle h) {
     cudaFree(h->meta_dev);
     cudaFree(h->gemm_dev);
     cudaFree(h->status_dev);
+    cudaFree(h->decode_partial);
+    cudaFree(h->decode_counters);
     for (auto& kv : h->work) {
         cudaFree(kv.second.off);
         cudaFree(kv.second.work);
@@ -261,14 +271,15 @@ patch_status get_worklist(patch_handle h, int kernel, int mb, WorkList** out) {
         *out = &it->second;
         return PATCH_OK;
     }
-    const std::vector<double>& cost = kernel == 0 ? h->plan.strip_cost : h->plan.pair_cost;
+    const std::vector<double>& cost =
+        kernel == 0 ? h->plan.strip_cost : kernel == 1 ? h->plan.pair_cost : h->plan.strip_bytes;
     const int rows = (int)cost.size();
     const int units = rows * mb;
-    const int slots = kernel == 0 ? h->dev.sms : h->dev.pair_clusters;
+    const int slots = kernel == 1 ? h->dev.pair_clusters : h->dev.sms;
     const int grid = std::max(1, std::min(slots, units));
     std::vector<int> order(units);
     for (int u = 0; u < units; ++u) order[u] = u;
-    const double epi = 1.0;
+    const double epi = kernel == 2 ? 0.0 : 1.0;
     std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x / mb] > cost[y / mb]; });
     using Item = std::pair<double, int>;  // (load, slot)
     std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
@@ -314,10 +325,37 @@ patch_status check_handle_device(patch_handle h) {
 constexpr int64_t kPairMinM = 256;  // below this the single-CTA tiles keep more SMs busy
 
 patch_status run_linear(patch_handle h, const void* X, int64_t M, void* Y, int path, cudaStream_t st) {
-    if (path == PATCH_PATH_AUTO) path = (M <= 8) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
+    if (path == PATCH_PATH_AUTO) path = (M <= kDecodeBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
     if (path == PATCH_PATH_GEMM) path = (M >= kPairMinM) ? PATCH_PATH_GEMM_PAIR : PATCH_PATH_GEMM_SINGLE;
     if (path == PATCH_PATH_GEMV) {
-        if (M > 16) return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
+        if (M > kDecodeBN) return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
+        WorkList* wl = nullptr;
+        patch_status s = get_worklist(h, 2, h->decode_parts, &wl);
+        if (s != PATCH_OK) return s;
+        CUtensorMap map;
+        s = encode_2d(&map, X, h->K, M, kSlabK, kDecodeBN, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s != PATCH_OK) return s;
+        DecodeArgs a;
+        a.packed = h->packed;
+        a.slab = h->slab_dev;
+        a.meta = h->meta_dev;
+        a.work_off = wl->off;
+        a.work = wl->work;
+        a.M = (int)M;
+        a.N = (int)h->N;
+        a.KB = h->plan.KB;
+        a.KC = h->plan.KC;
+        a.P = h->decode_parts;
+        a.partial = h->decode_partial;
+        a.counters = h->decode_counters;
+        a.Y = static_cast<__nv_bfloat16*>(Y);
+        a.status = h->status_dev;
+        cudaError_t e = launch_decode(map, a, wl->grid, st);
+        if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+        return PATCH_OK;
+    }
+    if (path == PATCH_PATH_GEMV_SIMT) {
+        if (M > 16) return fail(PATCH_ERR_SHAPE, "the CUDA-core decode kernel takes M <= 16 (got %lld)", (long long)M);
         GemvArgs a;
         a.packed = h->packed;
         a.slab = h->slab_dev;
@@ -330,7 +368,7 @@ patch_status run_linear(patch_handle h, const void* X, int64_t M, void* Y, int p
         a.KB = h->plan.KB;
         a.KC = h->plan.KC;
         cudaError_t e = launch_gemv(a, st);
-        if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+        if (e != cudaSuccess) return cuda_fail(e, "CUDA-core decode kernel launch");
         return PATCH_OK;
     }
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
@@ -465,6 +503,13 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         cudaGetLastError();
         return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
     }
+    // decode workspace: K split into parts so that strips x parts ~ 2.5 units per SM
+    h->decode_parts = std::max(1, std::min(p.KC, (int)((2.5 * di.sms) / p.S + 0.5)));
+    if (cudaMalloc(&h->decode_partial, sizeof(float) * (size_t)p.S * h->decode_parts * 128 * kDecodeBN) != cudaSuccess ||
+        cudaMalloc(&h->decode_counters, sizeof(unsigned) * p.S) != cudaSuccess) {
+        cudaGetLastError();
+        return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
+    }
     // tensor maps of the packed bytes viewed as rows of 64 bf16 (128 bytes):
     // dense slab / dense image (128 rows), 2:4 values (64 rows), metadata (16 rows)
     const int64_t rows = std::max<int64_t>(p.bytes, 2048) / 128;
@@ -481,7 +526,8 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(flags_dev, tile_flags, ntiles, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
         (e = cudaMemsetAsync(counters, 0, 3 * sizeof(unsigned long long), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess)
+        (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(h->decode_counters, 0, sizeof(unsigned) * p.S, s)) != cudaSuccess)
         return cleanup(cuda_fail(e, "pack set-up copies"));
     PackArgs a;
     a.W = static_cast<const uint16_t*>(W_bf16);
@@ -530,7 +576,7 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
                                void* stream) {
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_PAIR) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMV_SIMT) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     if (!X_bf16 || !Y_bf16) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
     if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
@@ -620,6 +666,8 @@ patch_status patch_check(patch_handle h, void* stream) {
     PATCH_CUDA(cudaMemcpy(&word, h->status_dev, sizeof(int), cudaMemcpyDeviceToHost));
     if (word != 0) {
         PATCH_CUDA(cudaMemset(h->status_dev, 0, sizeof(int)));
+        // an abandoned decode call may leave strip counters part-way: re-arm them
+        PATCH_CUDA(cudaMemset(h->decode_counters, 0, sizeof(unsigned) * h->plan.S));
         if (word == kStatusTimeout) return fail(PATCH_ERR_TIMEOUT, "a device-side wait ran past its limit");
         return fail(PATCH_ERR_CUDA, "device status word %d", word);
     }
@@ -708,11 +756,11 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // Decode sizes use no scratch at all.
+    // Decode sizes: the CUDA-core kernel needs no schedule and no scratch.
     if (M <= 8) {
         patch_status s = check_handle_device(h);
         if (s != PATCH_OK) return s;
-        return run_linear(h, X_bf16, M, Y_bf16, PATCH_PATH_GEMV, st);
+        return run_linear(h, X_bf16, M, Y_bf16, PATCH_PATH_GEMV_SIMT, st);
     }
     const bool pair = M >= kPairMinM;
     const int bn = pair ? kGemm2BN : kGemmBN;

@@ -1,0 +1,283 @@
+// Decode-sized product (M <= 16 tokens) on the tensor core with split-K.
+//
+// At decode sizes the layer is bound by the bytes of W it streams; 2:4 slabs
+// carry 1.125 bytes per weight instead of 2, which is where PATCH's hybrid
+// kernel earns its speed (abstract of "PATCH: Learnable Tile-level Hybrid
+// Sparsity for LLMs"). This kernel is a streaming engine: one persistent CTA
+// per SM walks a cost-balanced list of units (strip s, K-part p); warp 0 keeps
+// up to kStages packed slab records in flight with bulk copies (plus the
+// 16-token X tile by TMA), warp 1 runs them through tcgen05.mma / .mma.sp
+// with N = 16 into one of two TMEM accumulators, and warps 2..5 write each
+// unit's fp32 partial (128 rows x 16 tokens) to a workspace. The CTA that
+// finishes the last part of a strip (per-strip arrival counter) sums the
+// strip's partials in part order, so the result does not depend on which CTA
+// finishes first, writes bf16 Y and re-arms the counter for the next call.
+#include "kernels.cuh"
+
+namespace patch {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBN = kDecodeBN;           // tokens per MMA (M <= 16)
+constexpr int kStageA = 18432;           // 16 KB dense, or 8 KB values + 2 KB metadata
+constexpr int kStageX = kBN * 128;       // 2 KB, 128-byte swizzled
+constexpr int kStageBytes = kStageA + kStageX;
+constexpr int kStages = 8;
+constexpr int kSmemData = kStages * kStageBytes;
+constexpr int kSmemBytes = kSmemData + 1024 + 256;
+constexpr int kECol = 2 * kBN;           // metadata columns after the two accumulators
+constexpr int kTmemCols = 64;
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hybrid_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const DecodeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kStages;
+    uint64_t* acc_full = bars + 2 * kStages;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_full + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = abort_flag + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    auto raise = [&]() {
+        *abort_flag = 1;
+        atomicCAS(a.status, 0, kStatusTimeout);
+    };
+    const int w_begin = a.work_off[blockIdx.x];
+    const int w_end = a.work_off[blockIdx.x + 1];
+    // part p of a strip covers chunks [p*KC/P, (p+1)*KC/P), i.e. slabs from 2x that
+    auto part_range = [&](int p, int& b0, int& b1) {
+        b0 = 2 * (int)(((int64_t)p * a.KC) / a.P);
+        b1 = min(a.KB, 2 * (int)(((int64_t)(p + 1) * a.KC) / a.P));
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int it = w_begin; it < w_end && ok; ++it) {
+                const int u = a.work[it];
+                const int s = u / a.P, p = u % a.P;
+                int b0, b1;
+                part_range(p, b0, b1);
+                const uint32_t* trow = a.slab + (size_t)s * a.KB;
+                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
+                for (int b = b0; b < b1; ++b) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t d = trow[b];
+                    const bool sp = d & kSlabSparse, first = d & kSlabFirst;
+                    const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
+                    uint8_t* st = smem + stage * kStageBytes;
+                    mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + kStageX);
+                    bulk_load(st, a.packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    if (first)
+                        bulk_load(st + kSparseValBytes, a.packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes,
+                                  &full[stage]);
+                    tma_load_2d(st + kStageA, &tmap_x, &full[stage], b * kSlabK, 0);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            int st = stage;
+            uint32_t ph = phase;
+            for (int i = 0; i < kStages && i < issued; ++i) {
+                if (--st < 0) {
+                    st = kStages - 1;
+                    ph ^= 1u;
+                }
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(&full[st], ph) && globaltimer() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t idesc_d = idesc_bf16(128, kBN, false);
+            const uint32_t idesc_s = idesc_bf16(128, kBN, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, any_mma = false;
+            int t = 0;
+            for (int it = w_begin; it < w_end && ok; ++it, ++t) {
+                const int u = a.work[it];
+                const int s = u / a.P, p = u % a.P;
+                int b0, b1;
+                part_range(p, b0, b1);
+                const uint32_t* trow = a.slab + (size_t)s * a.KB;
+                const int acc = t & 1;
+                if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
+                    raise();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+                for (int b = b0; b < b1; ++b) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = trow[b];
+                    const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t x_addr = a_addr + kStageA;
+                    const uint32_t first_mma = (b == b0) ? 0u : 1u;
+                    if (d & kSlabSparse) {
+                        if (d & kSlabFirst)
+                            tc_cp_128x128b(tmem_base + kECol,
+                                           smem_desc(a_addr + kSparseValBytes, 16, 128, kLayoutNone));
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 512, kLayoutSw64);
+                            const uint64_t bd = smem_desc(x_addr + i * 64, 16, 1024, kLayoutSw128);
+                            const uint32_t ecol = kECol + (b & 1) * 2 + i;
+                            mma_sp_bf16(d_tmem, ad, bd, idesc_s | (ecol & 1u), tmem_base + (ecol & ~1u),
+                                        first_mma | (uint32_t)i);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 1024, kLayoutSw128);
+                            const uint64_t bd = smem_desc(x_addr + i * 32, 16, 1024, kLayoutSw128);
+                            mma_bf16(d_tmem, ad, bd, idesc_d, first_mma | (uint32_t)i);
+                        }
+                    }
+                    any_mma = true;
+                    tc_commit(&empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+            }
+            if (*abort_flag && any_mma) {
+                tc_commit(drain);
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int t = 0;
+        for (int it = w_begin; it < w_end; ++it, ++t) {
+            const int u = a.work[it];
+            const int s = u / a.P, p = u % a.P;
+            const int acc = t & 1;
+            if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
+                if (lane == 0) raise();
+                break;
+            }
+            tc_fence_after();
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN), v);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            // this unit's partial: workspace[s][p][row][0..15]
+            float4* dst = reinterpret_cast<float4*>(a.partial + (((size_t)s * a.P + p) * 128 + row) * kBN);
+#pragma unroll
+            for (int c = 0; c < kBN / 4; ++c)
+                dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                     __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+            __threadfence();
+            epi_bar();
+            if (threadIdx.x == 64) {
+                const unsigned old = atomicAdd(&a.counters[s], 1u);
+                *last_flag = (old == (unsigned)(a.P - 1));
+            }
+            epi_bar();
+            if (*last_flag) {
+                __threadfence();
+                float sum[kBN];
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) sum[c] = 0.f;
+                for (int pp = 0; pp < a.P; ++pp) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        a.partial + (((size_t)s * a.P + pp) * 128 + row) * kBN);
+#pragma unroll
+                    for (int c = 0; c < kBN / 4; ++c) {
+                        const float4 f = __ldcg(src + c);
+                        sum[4 * c] += f.x;
+                        sum[4 * c + 1] += f.y;
+                        sum[4 * c + 2] += f.z;
+                        sum[4 * c + 3] += f.w;
+                    }
+                }
+                __nv_bfloat16* yc = a.Y + (size_t)s * kStrip + row;
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (c < a.M) yc[(size_t)c * a.N] = __float2bfloat16_rn(sum[c]);
+                if (threadIdx.x == 64) a.counters[s] = 0u;  // re-armed for the next call
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t decode_prepare() {
+    return cudaFuncSetAttribute(hybrid_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t launch_decode(const CUtensorMap& tmap_x, const DecodeArgs& a, int grid, cudaStream_t st) {
+    hybrid_decode_kernel<<<grid, kThreads, kSmemBytes, st>>>(tmap_x, a);
+    return cudaGetLastError();
+}
+
+}  // namespace patch

@@ -56,14 +56,32 @@ struct GemvArgs {
     int M, N, K, KB, KC;
 };
 
+// Decode kernel (M <= 16): split-K over persistent CTAs, partials reduced by
+// the last CTA of each strip.
+struct DecodeArgs {
+    const uint8_t* packed;
+    const uint32_t* slab;
+    const uint32_t* meta;
+    const int* work_off;     // per CTA
+    const int* work;         // unit = strip * P + part
+    int M, N, KB, KC, P;
+    float* partial;          // [S][P][128][16] fp32 workspace
+    unsigned* counters;      // [S] arrivals per strip, zero between calls
+    __nv_bfloat16* Y;
+    int* status;
+};
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemm2(const CUtensorMap& tmap_x, const CUtensorMap& tm_a16, const CUtensorMap& tm_a8,
                          const CUtensorMap& tm_e, const Gemm2Args& a, int clusters, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
+cudaError_t launch_decode(const CUtensorMap& tmap_x, const DecodeArgs& a, int grid, cudaStream_t st);
+cudaError_t decode_prepare();
 cudaError_t gemm_prepare(int* max_pair_clusters);  // one-time function attributes, cluster occupancy
 
 constexpr int kGemmBN = 128;   // tokens per CTA tile (single-CTA kernel)
 constexpr int kGemm2BN = 256;  // tokens per CTA-pair tile
+constexpr int kDecodeBN = 16;  // tokens per decode MMA (M <= 16)
 
 }  // namespace patch

@@ -56,9 +56,10 @@ typedef enum {
 typedef enum {
     PATCH_PATH_AUTO = 0,
     PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core kernel, variant chosen by M */
-    PATCH_PATH_GEMV = 2,         /* CUDA-core kernel for decode-sized M (M <= 16) */
+    PATCH_PATH_GEMV = 2,         /* decode kernel (M <= 16): tcgen05 N=16, split-K */
     PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
-    PATCH_PATH_GEMM_PAIR = 4     /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
+    PATCH_PATH_GEMM_PAIR = 4,    /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
+    PATCH_PATH_GEMV_SIMT = 5     /* decode on CUDA cores (M <= 16), no workspace */
 } patch_path;
 
 typedef struct {

@@ -157,15 +157,34 @@ def test_pair_tiles_several_blocks(hsg, oracle_lib, M, frac):
     lin.free()
 
 
-@pytest.mark.parametrize("N,K,R,C", SMALL)
+@pytest.mark.parametrize("N,K,R,C", SMALL_ODD)
 @pytest.mark.parametrize("frac", [0.0, 0.6, 1.0])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 8, 12, 16])
-def test_gemv_small(hsg, oracle_lib, N, K, R, C, frac, M):
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
+def test_gemv_small(hsg, oracle_lib, N, K, R, C, frac, M, kernel):
     p = synth.make_problem(N, K, M, R=R, C=C, frac=frac, seed=M + 100, device="cuda")
     lin = pack(hsg, p)
-    Y = lin(p.X, path=hsg.PATH_GEMV)
+    Y = lin(p.X, path=hsg.PATH_GEMV if kernel == "tc" else hsg.PATH_GEMV_SIMT)
     torch.cuda.synchronize()
-    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"gemv M={M}")
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"gemv {kernel} M={M}")
+    lin.free()
+
+
+def test_decode_repeat_and_interleave(hsg, oracle_lib):
+    """The split-K decode re-arms its per-strip counters: repeated and
+    interleaved calls on one handle give identical bits."""
+    p = synth.make_problem(1152, 2048, 16, R=128, C=128, frac=0.7, seed=9, device="cuda")
+    lin = pack(hsg, p)
+    outs = []
+    for M in (16, 1, 16, 5, 16):
+        X = p.X[:M].contiguous()
+        outs.append((M, lin(X, path=hsg.PATH_GEMV)))
+    torch.cuda.synchronize()
+    lin.check()
+    assert torch.equal(outs[0][1], outs[2][1]) and torch.equal(outs[0][1], outs[4][1])
+    for M, Y in outs:
+        assert_close(Y, oracle_lib, p.X[:M].contiguous(), p.W, p.bits, p.keep, what=f"decode repeat M={M}")
     lin.free()
 
 
@@ -173,7 +192,7 @@ def test_single_strip_single_slab(hsg, oracle_lib):
     for frac in (0.0, 1.0):
         p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")
         lin = pack(hsg, p)
-        for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV):
+        for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV, hsg.PATH_GEMV_SIMT):
             Y = lin(p.X, path=path)
             torch.cuda.synchronize()
             assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"single slab {path}")
@@ -188,7 +207,8 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
     bits = synth.pack_bits(keep)
     X = synth.normal_bf16((40, K), 1.0, "cuda", "zero", "X")
     lin = hsg.PackedLinear.pack(W, bits, fl, 64, 64)
-    for path, M in ((hsg.PATH_GEMM_SINGLE, 40), (hsg.PATH_GEMM_PAIR, 40), (hsg.PATH_GEMV, 16)):
+    for path, M in ((hsg.PATH_GEMM_SINGLE, 40), (hsg.PATH_GEMM_PAIR, 40), (hsg.PATH_GEMV, 16),
+                    (hsg.PATH_GEMV_SIMT, 16)):
         Y = lin(X[:M].contiguous(), path=path)
         torch.cuda.synchronize()
         assert torch.count_nonzero(Y.float()) == 0
@@ -209,7 +229,8 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
 def test_one_sparse_tile(hsg, oracle_lib):
     p = synth.make_problem(512, 512, 50, R=128, C=128, n_sparse=1, seed=5, device="cuda")
     lin = pack(hsg, p)
-    for path, M in ((hsg.PATH_GEMM_SINGLE, 50), (hsg.PATH_GEMM_PAIR, 50), (hsg.PATH_GEMV, 16)):
+    for path, M in ((hsg.PATH_GEMM_SINGLE, 50), (hsg.PATH_GEMM_PAIR, 50), (hsg.PATH_GEMV, 16),
+                    (hsg.PATH_GEMV_SIMT, 16)):
         X = p.X[:M].contiguous()
         Y = lin(X, path=path)
         torch.cuda.synchronize()
@@ -257,7 +278,7 @@ def test_gemm_and_gemv_agree_with_oracle_on_config_1(hsg, oracle_lib):
     lin = pack(hsg, p)
     check_pack(hsg, oracle_lib, p, lin)
     assert abs(lin.info().sparsity - 0.25) < 1e-12
-    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV, hsg.PATH_AUTO):
+    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV, hsg.PATH_GEMV_SIMT, hsg.PATH_AUTO):
         Y = lin(p.X, path=path)
         torch.cuda.synchronize()
         assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"config1 {path}")
@@ -302,7 +323,7 @@ def test_config2_llama32_1b_m4096(hsg, oracle_lib):
 def test_config3_llama2_7b_decode(hsg, oracle_lib, M):
     shapes = synth.llama2_7b()
     _layer(hsg, oracle_lib, shapes, M, [0.7] * 7, tag="cfg3",
-           paths=[hsg.PATH_GEMV, hsg.PATH_GEMM], check_bytes=(M == 1))
+           paths=[hsg.PATH_GEMV, hsg.PATH_GEMV_SIMT, hsg.PATH_GEMM], check_bytes=(M == 1))
 
 
 @pytest.mark.parametrize("frac", [0.0, 0.5, 0.7, 0.9, 1.0])
