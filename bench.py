@@ -129,9 +129,16 @@ def model_linears(n_layers: int):
     return out
 
 
-def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1.0, rank=0):
-    """Packs every linear of the model at global 2:4 fraction `frac`. Returns
-    (list of (PackedLinear, K, N, kept_elems), inputs by K, outputs)."""
+ROLE_INPUT = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "mlp", "up": "mlp", "down": "down"}
+
+
+def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1.0, rank=0, group=True):
+    """Packs every linear of the model at global 2:4 fraction `frac`.
+
+    Returns (layers, X, Y, frac): layers is a list of per-layer launch lists;
+    each launch is (callable, [(PackedLinear, K, N, kept_weights, packed_bytes)]).
+    q/k/v read one input, gate/up another, o and down their own; every linear
+    writes its own output."""
     lins = model_linears(n_layers)
     T = [(l.N // 128) * (l.K // 128) for _, l in lins]
     if frac in (0.0, 1.0):
@@ -139,37 +146,56 @@ def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1
     else:
         counts = synth.split_fraction(T, frac, max(0.0, lo - (0.9 - frac)), min(1.0, hi - (0.9 - frac)),
                                       "model", seed, frac)
-    packed = []
+    X = {}
+    for role, K in (("attn", 2048), ("o", 2048), ("mlp", 2048), ("down", 8192)):
+        X[role] = synth.normal_bf16((M, K), 1.0, "cuda", "X", seed, rank, M, role)
+    per_layer = {}
     for (layer, l), cnt in zip(lins, counts):
         p = synth.make_problem(l.N, l.K, 0, R=128, C=128, n_sparse=cnt, seed=seed,
                                device="cuda", tag=f"L{layer}-{l.name}")
         lin = hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu())
         info = lin.info()
         kept = (info.slabs_total - info.slabs_sparse) * 128 * 64 + info.slabs_sparse * 128 * 32
-        packed.append((lin, l.K, l.N, kept, info.packed_bytes))
+        Yt = torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda")
+        per_layer.setdefault(layer, []).append((lin, l.K, l.N, kept, info.packed_bytes, X[ROLE_INPUT[l.name]], Yt))
         del p
     torch.cuda.synchronize()
-    X = {}
-    for K in sorted({l.K for _, l in lins}):
-        X[K] = synth.normal_bf16((M, K), 1.0, "cuda", "X", seed, rank, M, K)
-    Y = {}
-    for N in sorted({l.N for _, l in lins}):
-        Y[N] = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    return packed, X, Y, sum(counts) / sum(T)
+    layers = []
+    for layer in sorted(per_layer):
+        members = per_layer[layer]
+        if group:
+            g = hsg.LinearGroup([m[0] for m in members])
+            layers.append((g, members))
+        else:
+            for m in members:
+                layers.append((None, [m]))
+    return layers, X, None, sum(counts) / sum(T)
+
+
+def free_model(layers):
+    for g, members in layers:
+        if g is not None:
+            g.free()
+        for m in members:
+            m[0].free()
 
 
 def run_step(hsg, model, X, Y, stream, path=0, events=None):
-    for i, (lin, K, N, _, _) in enumerate(model):
+    for i, (g, members) in enumerate(model):
         if events is not None:
             events[i][0].record(stream)
-        hsg.patch_linear_path(lin.handle, X[K], Y[N], path, stream)
+        if g is not None:
+            g([m[5] for m in members], [m[6] for m in members], path=path, stream=stream)
+        else:
+            m = members[0]
+            hsg.patch_linear_path(m[0].handle, m[5], m[6], path, stream)
         if events is not None:
             events[i][1].record(stream)
 
 
-def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=False):
+def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=False, path=0):
     for _ in range(warmup):
-        run_step(hsg, model, X, Y, stream)
+        run_step(hsg, model, X, Y, stream, path)
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
@@ -181,7 +207,7 @@ def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=Fals
     torch.cuda.synchronize()
     start.record(stream)
     for s in range(steps):
-        run_step(hsg, model, X, Y, stream, events=ev[s] if ev else None)
+        run_step(hsg, model, X, Y, stream, path, events=ev[s] if ev else None)
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
@@ -195,8 +221,12 @@ def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=Fals
     return ms / steps, launch_ms
 
 
+def members(model):
+    return [m for _, ms in model for m in ms]
+
+
 def flops_dense(model, M):
-    return sum(2.0 * M * N * K for _, K, N, _, _ in model)
+    return sum(2.0 * M * m[2] * m[1] for m in members(model))
 
 
 def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
@@ -226,44 +256,54 @@ def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
                                        f"{t:.1f} s")
 
 
-def decode_bench(hsg, stream, steps=20):
-    """Decode kernel, Llama-2-7B layer shapes, 70% 2:4 tiles, 4 layers of
-    weights rotated so each launch streams its weights from HBM."""
+def decode_bench(hsg, stream, peaks, steps=20):
+    """Decode kernel on Llama-2-7B layer shapes, 70% 2:4 tiles: each layer's 7
+    linears in one grouped launch, 4 layers rotated (about 1.1 GB of weights,
+    far above L2) so every launch streams its weights from HBM. Bytes counted
+    are the ones the decode path must read: per-strip records (16 KB per dense
+    slab, 8 KB per 2:4 slab), metadata blocks, X and Y."""
     shapes = synth.llama2_7b()
     layers = []
     for L in range(4):
-        row = []
+        mem = []
         for l in shapes:
             p = synth.make_problem(l.N, l.K, 0, R=128, C=128, frac=0.7, seed=L, device="cuda",
                                    tag=f"dec{L}-{l.name}")
             lin = hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu())
-            row.append((lin, l.K, l.N, lin.info().packed_bytes))
+            info = lin.info()
+            algo = ((info.slabs_total - info.slabs_sparse) * 16384 + info.slabs_sparse * 8192
+                    + info.meta_blocks * 2048)
+            mem.append((lin, l.K, l.N, algo))
             del p
-        layers.append(row)
+        layers.append((hsg.LinearGroup([m[0] for m in mem]), mem))
     out = {}
     for M in (1, 4, 16):
         X = {K: synth.normal_bf16((M, K), 1.0, "cuda", "decX", M, K) for K in (4096, 11008)}
-        Y = {N: torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for N in (4096, 11008)}
-        for _ in range(3):
-            for row in layers:
-                for lin, K, N, _ in row:
-                    hsg.patch_linear_path(lin.handle, X[K], Y[N], 2, stream)
-        torch.cuda.synchronize()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        nbytes = 0
-        for _ in range(steps):
-            for row in layers:
-                for lin, K, N, pb in row:
-                    hsg.patch_linear_path(lin.handle, X[K], Y[N], 2, stream)
-                    nbytes += pb + M * K * 2 + M * N * 2
-        e.record(stream)
-        torch.cuda.synchronize()
-        ms = s.elapsed_time(e)
-        out[f"M{M}"] = {"GB_s": nbytes / (ms / 1e3) / 1e9, "us_per_layer": ms * 1e3 / (steps * len(layers))}
-    for row in layers:
-        for lin, *_ in row:
-            lin.free()
+        Y = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _, _, N, _ in mem] for _, mem in layers]
+        res = {}
+        for name, path in (("tc", 2), ("simt", 5)):
+            def step():
+                for (g, mem), ys in zip(layers, Y):
+                    g([X[K] for _, K, _, _ in mem], ys, path=path, stream=stream)
+            for _ in range(3):
+                step()
+            torch.cuda.synchronize()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            for _ in range(steps):
+                step()
+            e.record(stream)
+            torch.cuda.synchronize()
+            ms = s.elapsed_time(e)
+            nbytes = steps * sum(a + M * K * 2 + M * N * 2 for _, mem in layers for _, K, N, a in mem)
+            gbs = nbytes / (ms / 1e3) / 1e9
+            res[name] = {"GB_s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                         "us_per_layer": ms * 1e3 / (steps * len(layers))}
+        out[f"M{M}"] = res
+    for g, mem in layers:
+        g.free()
+        for m in mem:
+            m[0].free()
     return out
 
 
@@ -275,6 +315,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=16)
     ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--no-group", action="store_true", help="one launch per linear instead of per layer")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -284,7 +325,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    workload = (f"Llama-3.2-1B linears (16 layers x q,k,v,o,gate,up,down), M={args.M} tokens, "
+    workload = (f"Llama-3.2-1B linears ({args.layers} layers x q,k,v,o,gate,up,down), M={args.M} tokens, "
                 f"bf16, 128x128 tiles, 90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]")
 
     if args.impl == "reference":
@@ -319,24 +360,24 @@ def main():
     stream = torch.cuda.Stream()
     peaks = load_peaks()
     M = args.M
+    group = not args.no_group
 
     with torch.cuda.stream(stream):
-        model, X, Y, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank)
-        dense_model, _, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank)
+        model, X, _, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank, group=group)
+        dense_model, _, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank, group=group)
     torch.cuda.synchronize()
     F = flops_dense(model, M)
-    exec_flops = sum(2.0 * M * kept for _, _, _, kept, _ in model)
+    exec_flops = sum(2.0 * M * m[3] for m in members(model))
+    n_launch = len(model)
 
     with ClockSampler(torch.cuda.current_device()) as clk:
-        ms_h, launch_ms = time_steps(hsg, model, X, Y, args.steps, args.warmup, stream, dist_on,
-                                     per_launch=False)
+        ms_h, _ = time_steps(hsg, model, X, None, args.steps, args.warmup, stream, dist_on)
     clocks = clk.summary()
-    ms_d, _ = time_steps(hsg, dense_model, X, Y, args.steps, args.warmup, stream, dist_on)
-    # per-launch durations for the roofline (separate pass, events between launches)
-    _, launch_ms = time_steps(hsg, model, X, Y, max(2, args.steps // 2), 1, stream, dist_on, per_launch=True)
+    ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on)
+    # per-launch durations for the roofline (separate pass, events around each launch)
+    _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True)
     kern_ms = statistics.mean(sum(row) for row in launch_ms)
     achieved = exec_flops / (kern_ms / 1e3) / 1e12
-    n_launch = len(model)
     value = world * F / (ms_h / 1e3) / 1e12
 
     sweep = None
@@ -349,31 +390,31 @@ def main():
                 t = ms_h
             else:
                 with torch.cuda.stream(stream):
-                    mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank)
-                t, _ = time_steps(hsg, mdl, X, Y, args.steps, args.warmup, stream, dist_on)
-                for lin, *_ in mdl:
-                    lin.free()
+                    mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group)
+                t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on)
+                free_model(mdl)
                 del mdl
             sweep[str(f)] = {"tflops": world * F / (t / 1e3) / 1e12, "speedup_vs_dense": ms_d / t,
                              "ms_per_step": t}
 
     e2e = None
     if not args.no_e2e:
-        Xh = {K: X[K].cpu().pin_memory() for K in X}
-        Yh = {N: torch.empty(Y[N].shape, dtype=torch.bfloat16).pin_memory() for N in Y}
-        h2d = sum(M * K * 2 for _, K, _, _, _ in model)
-        d2h = sum(M * N * 2 for _, _, N, _, _ in model)
+        mem = members(model)
+        Xh = {id(m[5]): m[5].cpu().pin_memory() for m in mem}
+        Yh = [torch.empty(m[6].shape, dtype=torch.bfloat16).pin_memory() for m in mem]
+        h2d = sum(M * m[1] * 2 for m in mem)
+        d2h = sum(M * m[2] * 2 for m in mem)
         e2e_steps = max(1, min(args.steps, 3))
-        for lin, K, N, _, _ in model:  # warm-up
-            hsg.patch_linear_host(lin.handle, Xh[K], Yh[N], stream)
+        for m, yh in zip(mem, Yh):  # warm-up
+            hsg.patch_linear_host(m[0].handle, Xh[id(m[5])], yh, stream)
         if dist_on:
             torch.distributed.barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         s.record(stream)
         for _ in range(e2e_steps):
-            for lin, K, N, _, _ in model:
-                hsg.patch_linear_host(lin.handle, Xh[K], Yh[N], stream)
+            for m, yh in zip(mem, Yh):
+                hsg.patch_linear_host(m[0].handle, Xh[id(m[5])], yh, stream)
         e.record(stream)
         torch.cuda.synchronize()
         ms_e = s.elapsed_time(e) / e2e_steps
@@ -384,12 +425,11 @@ def main():
         e2e = {"value": world * F / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
 
+    free_model(dense_model)
+    dense_model = []
     decode = None
     if not args.no_decode:
-        for lin, *_ in dense_model:
-            lin.free()
-        dense_model = []
-        decode = decode_bench(hsg, stream)
+        decode = decode_bench(hsg, stream, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -397,30 +437,30 @@ def main():
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     if rank == 0:
+        packed_gb = sum(m[4] for m in members(model)) / 1e9
         line = {
             "metric": "hybrid dense/2:4 GEMM dense-equiv TFLOP/s and speedup vs dense bf16, per sparsity",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_h, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload, "M": M, "layers": args.layers, "linears": len(model),
+            "config": {"workload": workload, "M": M, "layers": args.layers, "linears": len(members(model)),
+                       "launches_per_step": n_launch, "grouped": group,
                        "frac_2to4": frac_real, "tile": "128x128",
-                       "l2": "inputs larger than L2 (%.2f GB of packed weights per step)" %
-                             (sum(pb for *_, pb in model) / 1e9),
+                       "l2": "inputs larger than L2 (%.2f GB of packed weights per step)" % packed_gb,
                        "parallelism": f"dp{world} (M split, replicated weights)"},
             "speedup_vs_dense": ms_d / ms_h, "dense_ms_per_step": ms_d,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
                          "traffic": None,
                          "kernel": "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
-                         "work": "2*M*(kept weights of stored slabs) per launch; sparse slabs count half",
+                         "work": "2*M per kept weight of every loaded slab (a 2:4 slab counts half)",
                          "peak_kind": f"bf16 sustained ({peaks['source']})"},
             "gpu_launches": n_launch * args.steps,
             "clocks": clocks,
             "sweep": sweep, "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
         }
         print(json.dumps(line))
-    for lin, *_ in model:
-        lin.free()
+    free_model(model)
     if dist_on:
         torch.distributed.destroy_process_group()
 

@@ -32,7 +32,8 @@ PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR, PATH_GEMV_SIM
 
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
-            "patch_version", "patch_plan", "patch_linear_noalloc"]
+            "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
+            "patch_group_linear", "patch_group_free"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -53,6 +54,10 @@ _lib.patch_linear.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_linear_path.argtypes = [_P, _P, _I64, _P, _I, _P]
 _lib.patch_linear_host.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_linear_noalloc.argtypes = [_P, _P, _I64, _P, _P]
+_lib.patch_group_create.argtypes = [_P, _I, ctypes.POINTER(_P)]
+_lib.patch_group_linear.argtypes = [_P, _P, _I64, _P, _I, _P]
+_lib.patch_group_free.argtypes = [_P]
+_lib.patch_group_free.restype = None
 _lib.patch_unpack.argtypes = [_P, _P, _P]
 _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]
 _lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
@@ -63,7 +68,8 @@ _lib.patch_free.restype = None
 _lib.patch_last_error.restype = ctypes.c_char_p
 _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
-           "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc"]:
+           "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc",
+           "patch_group_create", "patch_group_linear"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -173,6 +179,39 @@ def patch_check(h: int, stream=None):
 
 def patch_free(h: int):
     _lib.patch_free(h)
+
+
+class LinearGroup:
+    """Several packed linears run with one launch (they share M)."""
+
+    def __init__(self, linears):
+        self.linears = list(linears)
+        arr = (_P * len(self.linears))(*[l.handle for l in self.linears])
+        g = _P()
+        _check(_lib.patch_group_create(arr, len(self.linears), ctypes.byref(g)))
+        self.handle = g.value
+
+    def __call__(self, Xs, outs=None, path: int = PATH_AUTO, stream=None):
+        n = len(self.linears)
+        assert len(Xs) == n
+        M = Xs[0].shape[0]
+        if outs is None:
+            outs = [torch.empty((M, l.N), dtype=torch.bfloat16, device=Xs[0].device) for l in self.linears]
+        xs = (_P * n)(*[x.data_ptr() for x in Xs])
+        ys = (_P * n)(*[y.data_ptr() for y in outs])
+        _check(_lib.patch_group_linear(self.handle, xs, M, ys, path, _stream(stream)))
+        return outs
+
+    def free(self):
+        if self.handle:
+            _lib.patch_group_free(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
 
 
 # ---- object wrapper -----------------------------------------------------------

@@ -1,5 +1,8 @@
 // Host runtime behind the C ABI in patch_hybrid.h: argument checks, the slab
 // tables, the cost-balanced persistent schedules, tensor maps and launches.
+//
+// Every tensor-core launch runs a group of packed linears that share M; a
+// single patch_linear call runs the handle's own one-member group.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -16,11 +19,6 @@
 #include "patch_hybrid.h"
 
 using namespace patch;
-
-namespace patch {
-cudaError_t gemm_prepare_single();
-cudaError_t gemm_prepare_pair(int* max_clusters);
-}  // namespace patch
 
 namespace {
 
@@ -65,7 +63,8 @@ patch_status check_shape(int64_t N, int64_t K, int tile_rows, int tile_cols) {
 
 patch_status check_flags(const uint8_t* flags, int64_t n) {
     for (int64_t i = 0; i < n; ++i)
-        if (flags[i] > 1) return fail(PATCH_ERR_ARG, "tile flag %lld is %d, must be 0 or 1", (long long)i, (int)flags[i]);
+        if (flags[i] > 1)
+            return fail(PATCH_ERR_ARG, "tile flag %lld is %d, must be 0 or 1", (long long)i, (int)flags[i]);
     return PATCH_OK;
 }
 
@@ -117,8 +116,8 @@ patch_status get_encode() {
 
 // 2-D bf16 tensor map: `rows` rows of `cols` elements (row pitch cols*2 bytes),
 // box of box_cols x box_rows.
-patch_status encode_2d(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols,
-                       int box_rows, CUtensorMapSwizzle swizzle) {
+patch_status encode_2d(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int box_cols, int box_rows,
+                       CUtensorMapSwizzle swizzle) {
     patch_status st = get_encode();
     if (st != PATCH_OK) return st;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -133,7 +132,7 @@ patch_status encode_2d(CUtensorMap* map, const void* base, int64_t cols, int64_t
 }
 
 struct WorkList {
-    int grid = 0;         // CTAs (single kernel) or clusters (pair kernel)
+    int grid = 0;         // CTAs (single, decode) or CTA pairs (pair kernel)
     int* off = nullptr;   // device, grid + 1
     int* work = nullptr;  // device, units
 };
@@ -142,8 +141,8 @@ struct WorkList {
 struct Plan {
     int S = 0, KB = 0, KC = 0;
     std::vector<uint32_t> slab, meta, gemm;
-    std::vector<double> strip_cost, pair_cost;
-    std::vector<double> strip_bytes;  // bytes the decode kernel streams per strip
+    std::vector<double> strip_cost, pair_cost;  // tensor-core time: dense slab 1, 2:4 slab 1/2
+    std::vector<double> strip_bytes;            // bytes the decode kernel streams per strip
     int64_t bytes = 0, sparse = 0, pair_sparse = 0, meta_blocks = 0, images = 0;
 };
 
@@ -213,7 +212,28 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
     p.bytes = off;
 }
 
+// Decode K-parts per strip: the fewest parts that keep the per-CTA load within
+// a few percent of the best split, each part costing one extra epilogue.
+int choose_decode_parts(int S, int KC, int sms) {
+    double best = 1e30;
+    int best_p = 1;
+    for (int P = 1; P <= KC; ++P) {
+        const int units = S * P;
+        const int rounds = (units + sms - 1) / sms;
+        const double load = rounds * (1.0 / P + 0.01);  // strips of bytes per CTA, plus epilogue
+        if (load < best * 0.97) {
+            best = load;
+            best_p = P;
+        }
+    }
+    return best_p;
+}
+
+constexpr int64_t kPairMinM = 256;  // below this the single-CTA tiles keep more SMs busy
+
 }  // namespace
+
+struct patch_group_s;
 
 struct patch_handle_s {
     int device = 0;
@@ -226,24 +246,48 @@ struct patch_handle_s {
     uint32_t* meta_dev = nullptr;
     uint32_t* gemm_dev = nullptr;
     int* status_dev = nullptr;
-    int decode_parts = 1;              // K-parts per strip for the decode kernel
-    float* decode_partial = nullptr;   // [S][parts][128][16] fp32 workspace
+    int decode_parts = 1;                 // K-parts per strip for the decode kernel
+    float* decode_partial = nullptr;      // [S][parts][128][16] fp32 workspace
     unsigned* decode_counters = nullptr;  // [S], zero between calls
+    LinDesc desc{};                       // host copy of the device descriptor
     CUtensorMap tm_a16, tm_a8, tm_e;
     patch_info_t info{};
+    patch_group_s* self = nullptr;        // one-member group used by patch_linear
     std::mutex mu;
-    std::map<std::pair<int, int>, WorkList> work;  // (kernel, m_blocks) -> schedule
     void* stage_x = nullptr;
     size_t stage_x_bytes = 0;
     void* stage_y = nullptr;
     size_t stage_y_bytes = 0;
 };
 
+struct patch_group_s {
+    int device = 0;
+    DeviceInfo dev;
+    int n = 0;
+    patch_handle h[kMaxGroup] = {};
+    LinDesc* lins_dev = nullptr;  // n descriptors
+    int* status_dev = nullptr;    // the first member's status word
+    std::mutex mu;
+    std::map<std::pair<int, int>, WorkList> work;  // (kernel, m_blocks or 0) -> schedule
+};
+
 namespace {
+
+void free_group(patch_group g) {
+    if (!g) return;
+    cudaDeviceSynchronize();
+    cudaFree(g->lins_dev);
+    for (auto& kv : g->work) {
+        cudaFree(kv.second.off);
+        cudaFree(kv.second.work);
+    }
+    delete g;
+}
 
 void free_handle(patch_handle h) {
     if (!h) return;
     cudaDeviceSynchronize();
+    free_group(h->self);
     cudaFree(h->packed);
     cudaFree(h->slab_dev);
     cudaFree(h->meta_dev);
@@ -251,175 +295,199 @@ void free_handle(patch_handle h) {
     cudaFree(h->status_dev);
     cudaFree(h->decode_partial);
     cudaFree(h->decode_counters);
-    for (auto& kv : h->work) {
-        cudaFree(kv.second.off);
-        cudaFree(kv.second.work);
-    }
     cudaFree(h->stage_x);
     cudaFree(h->stage_y);
     delete h;
 }
 
-// Greedy longest-processing-time assignment of output tiles to persistent
-// CTAs (or CTA pairs). A tile's cost is its slab work (dense 1, sparse 1/2,
-// the ratio of tensor-core time) plus a fixed epilogue share.
-patch_status get_worklist(patch_handle h, int kernel, int mb, WorkList** out) {
-    std::lock_guard<std::mutex> lk(h->mu);
-    auto key = std::make_pair(kernel, mb);
-    auto it = h->work.find(key);
-    if (it != h->work.end()) {
-        *out = &it->second;
-        return PATCH_OK;
+patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
+    patch_group g = new (std::nothrow) patch_group_s();
+    if (!g) return fail(PATCH_ERR_NOMEM, "host allocation failed");
+    g->device = hs[0]->device;
+    g->dev = hs[0]->dev;
+    g->n = n;
+    g->status_dev = hs[0]->status_dev;
+    LinDesc d[kMaxGroup];
+    for (int i = 0; i < n; ++i) {
+        g->h[i] = hs[i];
+        d[i] = hs[i]->desc;
     }
-    const std::vector<double>& cost =
-        kernel == 0 ? h->plan.strip_cost : kernel == 1 ? h->plan.pair_cost : h->plan.strip_bytes;
-    const int rows = (int)cost.size();
-    const int units = rows * mb;
-    const int slots = kernel == 1 ? h->dev.pair_clusters : h->dev.sms;
-    const int grid = std::max(1, std::min(slots, units));
-    std::vector<int> order(units);
-    for (int u = 0; u < units; ++u) order[u] = u;
-    const double epi = kernel == 2 ? 0.0 : 1.0;
-    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x / mb] > cost[y / mb]; });
-    using Item = std::pair<double, int>;  // (load, slot)
+    if (cudaMalloc(&g->lins_dev, sizeof(LinDesc) * n) != cudaSuccess) {
+        cudaGetLastError();
+        delete g;
+        return fail(PATCH_ERR_NOMEM, "group descriptor allocation failed");
+    }
+    if (cudaMemcpy(g->lins_dev, d, sizeof(LinDesc) * n, cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(g->lins_dev);
+        delete g;
+        return fail(PATCH_ERR_CUDA, "group descriptor upload failed");
+    }
+    *out = g;
+    return PATCH_OK;
+}
+
+// Greedy longest-processing-time assignment of the group's units to
+// persistent CTAs (or CTA pairs). kernel 0: (strip, token block), cost = slab
+// work (dense 1, 2:4 1/2) + one epilogue; kernel 1: (strip pair, token block),
+// same costs; kernel 2: (strip, K-part), cost = streamed bytes of the part.
+void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
+    struct Unit {
+        double cost;
+        int id;
+    };
+    std::vector<Unit> units;
+    for (int l = 0; l < g->n; ++l) {
+        const Plan& p = g->h[l]->plan;
+        if (kernel == 0 || kernel == 1) {
+            const std::vector<double>& c = kernel == 0 ? p.strip_cost : p.pair_cost;
+            for (int r = 0; r < (int)c.size(); ++r)
+                for (int j = 0; j < mb; ++j) units.push_back({c[r] + 1.0, (l << kUnitShift) | (r * mb + j)});
+        } else {
+            const int P = g->h[l]->decode_parts;
+            for (int s = 0; s < p.S; ++s)
+                for (int q = 0; q < P; ++q)
+                    units.push_back({p.strip_bytes[s] / P + 16384.0, (l << kUnitShift) | (s * P + q)});
+        }
+    }
+    std::stable_sort(units.begin(), units.end(), [](const Unit& x, const Unit& y) { return x.cost > y.cost; });
+    const int slots = kernel == 1 ? g->dev.pair_clusters : g->dev.sms;
+    const int grid = std::max(1, std::min(slots, (int)units.size()));
+    using Item = std::pair<double, int>;
     std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
     for (int c = 0; c < grid; ++c) pq.push({0.0, c});
     std::vector<std::vector<int>> lists(grid);
-    for (int u : order) {
+    for (const Unit& u : units) {
         Item top = pq.top();
         pq.pop();
-        lists[top.second].push_back(u);
-        top.first += cost[u / mb] + epi;
+        lists[top.second].push_back(u.id);
+        top.first += u.cost;
         pq.push(top);
     }
-    std::vector<int> off(grid + 1, 0), work;
-    work.reserve(units);
+    off.assign(grid + 1, 0);
+    work.clear();
     for (int c = 0; c < grid; ++c) {
         off[c] = (int)work.size();
         work.insert(work.end(), lists[c].begin(), lists[c].end());
     }
     off[grid] = (int)work.size();
+}
+
+patch_status get_worklist(patch_group g, int kernel, int mb, WorkList** out) {
+    std::lock_guard<std::mutex> lk(g->mu);
+    auto key = std::make_pair(kernel, mb);
+    auto it = g->work.find(key);
+    if (it != g->work.end()) {
+        *out = &it->second;
+        return PATCH_OK;
+    }
+    std::vector<int> off, work;
+    lpt_schedule(g, kernel, mb, off, work);
     WorkList wl;
-    wl.grid = grid;
-    if (cudaMalloc(&wl.off, sizeof(int) * (grid + 1)) != cudaSuccess ||
-        cudaMalloc(&wl.work, sizeof(int) * std::max(units, 1)) != cudaSuccess) {
+    wl.grid = (int)off.size() - 1;
+    if (cudaMalloc(&wl.off, sizeof(int) * off.size()) != cudaSuccess ||
+        cudaMalloc(&wl.work, sizeof(int) * std::max<size_t>(work.size(), 1)) != cudaSuccess) {
         cudaFree(wl.off);
         cudaGetLastError();
         return fail(PATCH_ERR_NOMEM, "schedule allocation failed");
     }
-    PATCH_CUDA(cudaMemcpy(wl.off, off.data(), sizeof(int) * (grid + 1), cudaMemcpyHostToDevice));
-    PATCH_CUDA(cudaMemcpy(wl.work, work.data(), sizeof(int) * units, cudaMemcpyHostToDevice));
-    auto res = h->work.emplace(key, wl);
+    PATCH_CUDA(cudaMemcpy(wl.off, off.data(), sizeof(int) * off.size(), cudaMemcpyHostToDevice));
+    PATCH_CUDA(cudaMemcpy(wl.work, work.data(), sizeof(int) * work.size(), cudaMemcpyHostToDevice));
+    auto res = g->work.emplace(key, wl);
     *out = &res.first->second;
     return PATCH_OK;
 }
 
-patch_status check_handle_device(patch_handle h) {
+patch_status check_device_is(int device) {
     int dev = -1;
     PATCH_CUDA(cudaGetDevice(&dev));
-    if (dev != h->device)
-        return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", h->device, dev);
+    if (dev != device) return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", device, dev);
     return PATCH_OK;
 }
 
-constexpr int64_t kPairMinM = 256;  // below this the single-CTA tiles keep more SMs busy
-
-patch_status run_linear(patch_handle h, const void* X, int64_t M, void* Y, int path, cudaStream_t st) {
+// Resolves AUTO / GEMM to a concrete kernel for this M.
+int resolve_path(int path, int64_t M) {
     if (path == PATCH_PATH_AUTO) path = (M <= kDecodeBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
     if (path == PATCH_PATH_GEMM) path = (M >= kPairMinM) ? PATCH_PATH_GEMM_PAIR : PATCH_PATH_GEMM_SINGLE;
-    if (path == PATCH_PATH_GEMV) {
-        if (M > kDecodeBN) return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
-        WorkList* wl = nullptr;
-        patch_status s = get_worklist(h, 2, h->decode_parts, &wl);
-        if (s != PATCH_OK) return s;
-        CUtensorMap map;
-        s = encode_2d(&map, X, h->K, M, kSlabK, kDecodeBN, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (s != PATCH_OK) return s;
-        DecodeArgs a;
-        a.packed = h->packed;
-        a.slab = h->slab_dev;
-        a.meta = h->meta_dev;
-        a.work_off = wl->off;
-        a.work = wl->work;
-        a.M = (int)M;
-        a.N = (int)h->N;
-        a.KB = h->plan.KB;
-        a.KC = h->plan.KC;
-        a.P = h->decode_parts;
-        a.partial = h->decode_partial;
-        a.counters = h->decode_counters;
-        a.Y = static_cast<__nv_bfloat16*>(Y);
-        a.status = h->status_dev;
-        cudaError_t e = launch_decode(map, a, wl->grid, st);
-        if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-        return PATCH_OK;
-    }
-    if (path == PATCH_PATH_GEMV_SIMT) {
-        if (M > 16) return fail(PATCH_ERR_SHAPE, "the CUDA-core decode kernel takes M <= 16 (got %lld)", (long long)M);
-        GemvArgs a;
-        a.packed = h->packed;
-        a.slab = h->slab_dev;
-        a.meta = h->meta_dev;
-        a.X = static_cast<const __nv_bfloat16*>(X);
-        a.Y = static_cast<__nv_bfloat16*>(Y);
-        a.M = (int)M;
-        a.N = (int)h->N;
-        a.K = (int)h->K;
-        a.KB = h->plan.KB;
-        a.KC = h->plan.KC;
-        cudaError_t e = launch_gemv(a, st);
-        if (e != cudaSuccess) return cuda_fail(e, "CUDA-core decode kernel launch");
-        return PATCH_OK;
-    }
-    if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
-    if (path == PATCH_PATH_GEMM_SINGLE) {
-        const int mb = (int)((M + kGemmBN - 1) / kGemmBN);
-        WorkList* wl = nullptr;
-        patch_status s = get_worklist(h, 0, mb, &wl);
-        if (s != PATCH_OK) return s;
-        CUtensorMap map;
-        s = encode_2d(&map, X, h->K, M, kSlabK, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (s != PATCH_OK) return s;
-        GemmArgs a;
-        a.packed = h->packed;
-        a.slab = h->slab_dev;
-        a.meta = h->meta_dev;
-        a.work_off = wl->off;
-        a.work = wl->work;
-        a.M = (int)M;
-        a.N = (int)h->N;
-        a.KB = h->plan.KB;
-        a.KC = h->plan.KC;
-        a.MB = mb;
-        a.Y = static_cast<__nv_bfloat16*>(Y);
-        a.status = h->status_dev;
-        cudaError_t e = launch_gemm(map, a, wl->grid, st);
-        if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
-        return PATCH_OK;
-    }
-    if (path != PATCH_PATH_GEMM_PAIR) return fail(PATCH_ERR_ARG, "unknown path %d", path);
-    const int mb = (int)((M + kGemm2BN - 1) / kGemm2BN);
-    WorkList* wl = nullptr;
-    patch_status s = get_worklist(h, 1, mb, &wl);
-    if (s != PATCH_OK) return s;
-    CUtensorMap map;
-    s = encode_2d(&map, X, h->K, M, kSlabK, kGemm2BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (s != PATCH_OK) return s;
-    Gemm2Args a;
-    a.gemm = h->gemm_dev;
+    return path;
+}
+
+patch_status run_simt(patch_handle h, const void* X, int64_t M, void* Y, cudaStream_t st) {
+    if (M > 16) return fail(PATCH_ERR_SHAPE, "the CUDA-core decode kernel takes M <= 16 (got %lld)", (long long)M);
+    GemvArgs a;
+    a.packed = h->packed;
+    a.slab = h->slab_dev;
     a.meta = h->meta_dev;
-    a.work_off = wl->off;
-    a.work = wl->work;
+    a.X = static_cast<const __nv_bfloat16*>(X);
+    a.Y = static_cast<__nv_bfloat16*>(Y);
     a.M = (int)M;
     a.N = (int)h->N;
-    a.S = h->plan.S;
+    a.K = (int)h->K;
     a.KB = h->plan.KB;
     a.KC = h->plan.KC;
+    cudaError_t e = launch_gemv(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "CUDA-core decode kernel launch");
+    return PATCH_OK;
+}
+
+// One launch over every member of the group. `sched` (off, work) may point at
+// caller-provided device memory; otherwise the group's cached schedule is used.
+patch_status run_group(patch_group g, const void* const* X, int64_t M, void* const* Y, int path, cudaStream_t st,
+                       const int* sched_off = nullptr, const int* sched_work = nullptr, int sched_grid = 0) {
+    path = resolve_path(path, M);
+    if (path == PATCH_PATH_GEMV_SIMT) {
+        for (int l = 0; l < g->n; ++l) {
+            patch_status s = run_simt(g->h[l], X[l], M, Y[l], st);
+            if (s != PATCH_OK) return s;
+        }
+        return PATCH_OK;
+    }
+    if (path != PATCH_PATH_GEMV && path != PATCH_PATH_GEMM_SINGLE && path != PATCH_PATH_GEMM_PAIR)
+        return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path == PATCH_PATH_GEMV && M > kDecodeBN)
+        return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
+    if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
+    const int kernel = path == PATCH_PATH_GEMM_SINGLE ? 0 : path == PATCH_PATH_GEMM_PAIR ? 1 : 2;
+    const int bn = kernel == 0 ? kGemmBN : kernel == 1 ? kGemm2BN : kDecodeBN;
+    const int mb = kernel == 2 ? 0 : (int)((M + bn - 1) / bn);
+    const int box_rows = kernel == 1 ? kGemm2BN / 2 : bn;
+    GroupMaps maps;
+    GroupArgs a;
+    memset(&maps, 0, sizeof(maps));
+    memset(&a, 0, sizeof(a));
+    for (int l = 0; l < g->n; ++l) {
+        patch_handle h = g->h[l];
+        patch_status s = encode_2d(&maps.x[l], X[l], h->K, M, kSlabK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (s != PATCH_OK) return s;
+        maps.a16[l] = h->tm_a16;
+        maps.a8[l] = h->tm_a8;
+        maps.e[l] = h->tm_e;
+        a.Y[l] = static_cast<__nv_bfloat16*>(Y[l]);
+    }
+    int grid = sched_grid;
+    if (!sched_off) {
+        WorkList* wl = nullptr;
+        patch_status s = get_worklist(g, kernel, mb, &wl);
+        if (s != PATCH_OK) return s;
+        sched_off = wl->off;
+        sched_work = wl->work;
+        grid = wl->grid;
+    }
+    a.lins = g->lins_dev;
+    a.work_off = sched_off;
+    a.work = sched_work;
+    a.M = (int)M;
     a.MB = mb;
-    a.Y = static_cast<__nv_bfloat16*>(Y);
-    a.status = h->status_dev;
-    cudaError_t e = launch_gemm2(map, h->tm_a16, h->tm_a8, h->tm_e, a, wl->grid, st);
-    if (e != cudaSuccess) return cuda_fail(e, "CTA-pair tensor-core kernel launch");
+    a.status = g->status_dev;
+    cudaError_t e = kernel == 0 ? launch_gemm(maps, a, grid, st)
+                  : kernel == 1 ? launch_gemm2(maps, a, grid, st)
+                                : launch_decode(maps, a, grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+    return PATCH_OK;
+}
+
+patch_status check_xy(const void* X, const void* Y) {
+    if (!X || !Y) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
+    if (!aligned16(X) || !aligned16(Y)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
     return PATCH_OK;
 }
 
@@ -429,7 +497,7 @@ extern "C" {
 
 const char* patch_last_error(void) { return g_err.c_str(); }
 
-int patch_version(void) { return 2; }
+int patch_version(void) { return 3; }
 
 patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                         uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table, int64_t* packed_bytes) {
@@ -485,6 +553,7 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     }
     int64_t tiles_sparse = 0;
     for (int64_t i = 0; i < ntiles; ++i) tiles_sparse += tile_flags[i];
+    h->decode_parts = choose_decode_parts(p.S, p.KC, di.sms);
 
     uint8_t* flags_dev = nullptr;
     unsigned long long* counters = nullptr;
@@ -498,15 +567,12 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         cudaMalloc(&h->slab_dev, sizeof(uint32_t) * p.slab.size()) != cudaSuccess ||
         cudaMalloc(&h->meta_dev, sizeof(uint32_t) * p.meta.size()) != cudaSuccess ||
         cudaMalloc(&h->gemm_dev, sizeof(uint32_t) * p.gemm.size()) != cudaSuccess ||
-        cudaMalloc(&h->status_dev, sizeof(int)) != cudaSuccess || cudaMalloc(&flags_dev, ntiles) != cudaSuccess ||
+        cudaMalloc(&h->status_dev, sizeof(int)) != cudaSuccess ||
+        cudaMalloc(&h->decode_partial, sizeof(float) * (size_t)p.S * h->decode_parts * 128 * kDecodeBN) !=
+            cudaSuccess ||
+        cudaMalloc(&h->decode_counters, sizeof(unsigned) * p.S) != cudaSuccess ||
+        cudaMalloc(&flags_dev, ntiles) != cudaSuccess ||
         cudaMalloc(&counters, 3 * sizeof(unsigned long long)) != cudaSuccess) {
-        cudaGetLastError();
-        return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
-    }
-    // decode workspace: K split into parts so that strips x parts ~ 2.5 units per SM
-    h->decode_parts = std::max(1, std::min(p.KC, (int)((2.5 * di.sms) / p.S + 0.5)));
-    if (cudaMalloc(&h->decode_partial, sizeof(float) * (size_t)p.S * h->decode_parts * 128 * kDecodeBN) != cudaSuccess ||
-        cudaMalloc(&h->decode_counters, sizeof(unsigned) * p.S) != cudaSuccess) {
         cudaGetLastError();
         return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
     }
@@ -552,6 +618,19 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         return cleanup(cuda_fail(e, "pack kernel"));
     if (cnt[0] != 0)
         return cleanup(fail(PATCH_ERR_MASK, "%llu groups inside 2:4 tiles do not keep exactly two of four", cnt[0]));
+    h->desc.packed = h->packed;
+    h->desc.slab = h->slab_dev;
+    h->desc.meta = h->meta_dev;
+    h->desc.gemm = h->gemm_dev;
+    h->desc.partial = h->decode_partial;
+    h->desc.counters = h->decode_counters;
+    h->desc.N = (int)N;
+    h->desc.S = p.S;
+    h->desc.KB = p.KB;
+    h->desc.KC = p.KC;
+    h->desc.P = h->decode_parts;
+    patch_handle self[1] = {h};
+    if ((st = make_group(self, 1, &h->self)) != PATCH_OK) return cleanup(st);
     patch_info_t& info = h->info;
     info.N = N;
     info.K = K;
@@ -578,11 +657,12 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
     if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMV_SIMT) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
-    if (!X_bf16 || !Y_bf16) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
-    if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
-    patch_status st = check_handle_device(h);
+    patch_status st = check_xy(X_bf16, Y_bf16);
     if (st != PATCH_OK) return st;
-    return run_linear(h, X_bf16, M, Y_bf16, path, static_cast<cudaStream_t>(stream));
+    if ((st = check_device_is(h->device)) != PATCH_OK) return st;
+    const void* xs[1] = {X_bf16};
+    void* ys[1] = {Y_bf16};
+    return run_group(h->self, xs, M, ys, path, static_cast<cudaStream_t>(stream));
 }
 
 patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16, void* stream) {
@@ -594,9 +674,10 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
     if (M == 0) return PATCH_OK;
     if (!X_host || !Y_host) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
-    patch_status st = check_handle_device(h);
+    patch_status st = check_device_is(h->device);
     if (st != PATCH_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lk(h->mu);
     const size_t xb = (size_t)M * h->K * 2, yb = (size_t)M * h->N * 2;
     if (xb > h->stage_x_bytes) {
         cudaFree(h->stage_x);
@@ -619,17 +700,51 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
         h->stage_y_bytes = yb;
     }
     PATCH_CUDA(cudaMemcpyAsync(h->stage_x, X_host, xb, cudaMemcpyHostToDevice, s));
-    st = run_linear(h, h->stage_x, M, h->stage_y, PATCH_PATH_AUTO, s);
+    const void* xs[1] = {h->stage_x};
+    void* ys[1] = {h->stage_y};
+    st = run_group(h->self, xs, M, ys, PATCH_PATH_AUTO, s);
     if (st != PATCH_OK) return st;
     PATCH_CUDA(cudaMemcpyAsync(Y_host, h->stage_y, yb, cudaMemcpyDeviceToHost, s));
     PATCH_CUDA(cudaStreamSynchronize(s));
     return PATCH_OK;
 }
 
+patch_status patch_group_create(const patch_handle* handles, int n, patch_group* out) {
+    g_err.clear();
+    if (!out) return fail(PATCH_ERR_ARG, "out is NULL");
+    *out = nullptr;
+    if (!handles || n < 1 || n > kMaxGroup) return fail(PATCH_ERR_ARG, "a group takes 1 to %d handles", kMaxGroup);
+    for (int i = 0; i < n; ++i) {
+        if (!handles[i]) return fail(PATCH_ERR_ARG, "handle %d is NULL", i);
+        if (handles[i]->device != handles[0]->device) return fail(PATCH_ERR_ARG, "handles live on different devices");
+    }
+    patch_status st = check_device_is(handles[0]->device);
+    if (st != PATCH_OK) return st;
+    return make_group(handles, n, out);
+}
+
+patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, void* const* Y, int path,
+                                void* stream) {
+    if (!g) return fail(PATCH_ERR_ARG, "group is NULL");
+    if (!X || !Y) return fail(PATCH_ERR_ARG, "X and Y arrays must be non-NULL");
+    if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMV_SIMT) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (M == 0) return PATCH_OK;
+    for (int l = 0; l < g->n; ++l) {
+        patch_status st = check_xy(X[l], Y[l]);
+        if (st != PATCH_OK) return st;
+    }
+    patch_status st = check_device_is(g->device);
+    if (st != PATCH_OK) return st;
+    return run_group(g, X, M, Y, path, static_cast<cudaStream_t>(stream));
+}
+
+void patch_group_free(patch_group g) { free_group(g); }
+
 patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream) {
     if (!h || !W_masked_bf16) return fail(PATCH_ERR_ARG, "handle and output must be non-NULL");
     if (!aligned16(W_masked_bf16)) return fail(PATCH_ERR_ALIGN, "output must be 16-byte aligned");
-    patch_status st = check_handle_device(h);
+    patch_status st = check_device_is(h->device);
     if (st != PATCH_OK) return st;
     unpack_kernel<<<h->plan.S * h->plan.KB, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         h->packed, h->slab_dev, h->meta_dev, h->plan.KB, h->plan.KC, h->K, static_cast<uint16_t*>(W_masked_bf16));
@@ -716,35 +831,6 @@ patch_status noalloc_scratch(int dev, int** out) {
     return PATCH_OK;
 }
 
-// Same greedy LPT rule as the cached schedules, on the host only.
-void noalloc_schedule(patch_handle h, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
-    const std::vector<double>& cost = kernel == 0 ? h->plan.strip_cost : h->plan.pair_cost;
-    const int units = (int)cost.size() * mb;
-    const int slots = kernel == 0 ? h->dev.sms : h->dev.pair_clusters;
-    const int grid = std::max(1, std::min(slots, units));
-    std::vector<int> order(units);
-    for (int u = 0; u < units; ++u) order[u] = u;
-    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x / mb] > cost[y / mb]; });
-    using Item = std::pair<double, int>;
-    std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
-    for (int c = 0; c < grid; ++c) pq.push({0.0, c});
-    std::vector<std::vector<int>> lists(grid);
-    for (int u : order) {
-        Item top = pq.top();
-        pq.pop();
-        lists[top.second].push_back(u);
-        top.first += cost[u / mb] + 1.0;
-        pq.push(top);
-    }
-    off.assign(grid + 1, 0);
-    work.clear();
-    for (int c = 0; c < grid; ++c) {
-        off[c] = (int)work.size();
-        work.insert(work.end(), lists[c].begin(), lists[c].end());
-    }
-    off[grid] = (int)work.size();
-}
-
 }  // namespace
 
 extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
@@ -752,17 +838,15 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
     if (M == 0) return PATCH_OK;
-    if (!X_bf16 || !Y_bf16) return fail(PATCH_ERR_ARG, "X and Y must be non-NULL");
-    if (!aligned16(X_bf16) || !aligned16(Y_bf16)) return fail(PATCH_ERR_ALIGN, "X and Y must be 16-byte aligned");
+    patch_status s = check_xy(X_bf16, Y_bf16);
+    if (s != PATCH_OK) return s;
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = check_device_is(h->device)) != PATCH_OK) return s;
     // Decode sizes: the CUDA-core kernel needs no schedule and no scratch.
-    if (M <= 8) {
-        patch_status s = check_handle_device(h);
-        if (s != PATCH_OK) return s;
-        return run_linear(h, X_bf16, M, Y_bf16, PATCH_PATH_GEMV_SIMT, st);
-    }
-    const bool pair = M >= kPairMinM;
+    if (M <= 8) return run_simt(h, X_bf16, M, Y_bf16, st);
+    const int path = resolve_path(PATCH_PATH_GEMM, M);
+    const bool pair = path == PATCH_PATH_GEMM_PAIR;
     const int bn = pair ? kGemm2BN : kGemmBN;
     const int64_t mb = (M + bn - 1) / bn;
     const int64_t rows = pair ? (int64_t)h->plan.pair_cost.size() : (int64_t)h->plan.strip_cost.size();
@@ -772,57 +856,16 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
                     "patch_linear_noalloc handles at most %d output tiles per call (this call needs %lld); "
                     "use patch_linear",
                     kNoAllocMaxUnits, (long long)(rows * mb));
-    int dev = -1;
-    PATCH_CUDA(cudaGetDevice(&dev));
-    if (dev != h->device) return fail(PATCH_ERR_ARG, "handle lives on device %d, current device is %d", h->device, dev);
     int* sched = nullptr;
-    patch_status s = noalloc_scratch(dev, &sched);
-    if (s != PATCH_OK) return s;
+    if ((s = noalloc_scratch(h->device, &sched)) != PATCH_OK) return s;
     std::vector<int> off, work;
-    noalloc_schedule(h, pair ? 1 : 0, (int)mb, off, work);
-    const int grid = (int)off.size() - 1;
+    lpt_schedule(h->self, pair ? 1 : 0, (int)mb, off, work);
     int* d_off = sched;
     int* d_work = sched + kNoAllocMaxSlots + 1;
     PATCH_CUDA(cudaMemcpyAsync(d_off, off.data(), sizeof(int) * off.size(), cudaMemcpyHostToDevice, st));
     PATCH_CUDA(cudaMemcpyAsync(d_work, work.data(), sizeof(int) * std::max<size_t>(work.size(), 1),
                                cudaMemcpyHostToDevice, st));
-    CUtensorMap map;
-    if (!pair) {
-        s = encode_2d(&map, X_bf16, h->K, M, kSlabK, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (s != PATCH_OK) return s;
-        GemmArgs a;
-        a.packed = h->packed;
-        a.slab = h->slab_dev;
-        a.meta = h->meta_dev;
-        a.work_off = d_off;
-        a.work = d_work;
-        a.M = (int)M;
-        a.N = (int)h->N;
-        a.KB = h->plan.KB;
-        a.KC = h->plan.KC;
-        a.MB = (int)mb;
-        a.Y = static_cast<__nv_bfloat16*>(Y_bf16);
-        a.status = h->status_dev;
-        cudaError_t e = launch_gemm(map, a, grid, st);
-        if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
-        return PATCH_OK;
-    }
-    s = encode_2d(&map, X_bf16, h->K, M, kSlabK, kGemm2BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (s != PATCH_OK) return s;
-    Gemm2Args a;
-    a.gemm = h->gemm_dev;
-    a.meta = h->meta_dev;
-    a.work_off = d_off;
-    a.work = d_work;
-    a.M = (int)M;
-    a.N = (int)h->N;
-    a.S = h->plan.S;
-    a.KB = h->plan.KB;
-    a.KC = h->plan.KC;
-    a.MB = (int)mb;
-    a.Y = static_cast<__nv_bfloat16*>(Y_bf16);
-    a.status = h->status_dev;
-    cudaError_t e = launch_gemm2(map, h->tm_a16, h->tm_a8, h->tm_e, a, grid, st);
-    if (e != cudaSuccess) return cuda_fail(e, "CTA-pair tensor-core kernel launch");
-    return PATCH_OK;
+    const void* xs[1] = {X_bf16};
+    void* ys[1] = {Y_bf16};
+    return run_group(h->self, xs, M, ys, path, st, d_off, d_work, (int)off.size() - 1);
 }

@@ -32,7 +32,7 @@ constexpr int kTmemCols = 64;
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    hybrid_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const DecodeArgs a) {
+    hybrid_decode_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -61,7 +61,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -78,9 +77,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int w_begin = a.work_off[blockIdx.x];
     const int w_end = a.work_off[blockIdx.x + 1];
     // part p of a strip covers chunks [p*KC/P, (p+1)*KC/P), i.e. slabs from 2x that
-    auto part_range = [&](int p, int& b0, int& b1) {
-        b0 = 2 * (int)(((int64_t)p * a.KC) / a.P);
-        b1 = min(a.KB, 2 * (int)(((int64_t)(p + 1) * a.KC) / a.P));
+    auto part_range = [](const LinDesc& L, int p, int& b0, int& b1) {
+        b0 = 2 * (int)(((int64_t)p * L.KC) / L.P);
+        b1 = min(L.KB, 2 * (int)(((int64_t)(p + 1) * L.KC) / L.P));
     };
 
     if (warp == 0) {
@@ -92,11 +91,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
-                const int s = u / a.P, p = u % a.P;
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int s = lu / L.P, p = lu % L.P;
                 int b0, b1;
-                part_range(p, b0, b1);
-                const uint32_t* trow = a.slab + (size_t)s * a.KB;
-                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
+                part_range(L, p, b0, b1);
+                const uint32_t* trow = L.slab + (size_t)s * L.KB;
+                const uint32_t* mrow = L.meta + (size_t)s * L.KC;
+                const uint8_t* packed = L.packed;
+                const CUtensorMap* tmap_x = &maps.x[l];
                 for (int b = b0; b < b1; ++b) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         raise();
@@ -108,11 +111,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
                     uint8_t* st = smem + stage * kStageBytes;
                     mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + kStageX);
-                    bulk_load(st, a.packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    bulk_load(st, packed + slab_offset_bytes(d), bytes_a, &full[stage]);
                     if (first)
-                        bulk_load(st + kSparseValBytes, a.packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes,
+                        bulk_load(st + kSparseValBytes, packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes,
                                   &full[stage]);
-                    tma_load_2d(st + kStageA, &tmap_x, &full[stage], b * kSlabK, 0);
+                    tma_load_2d(st + kStageA, tmap_x, &full[stage], b * kSlabK, 0);
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -143,10 +146,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
-                const int s = u / a.P, p = u % a.P;
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int s = lu / L.P, p = lu % L.P;
                 int b0, b1;
-                part_range(p, b0, b1);
-                const uint32_t* trow = a.slab + (size_t)s * a.KB;
+                part_range(L, p, b0, b1);
+                const uint32_t* trow = L.slab + (size_t)s * L.KB;
                 const int acc = t & 1;
                 if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
                     raise();
@@ -209,7 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
             const int u = a.work[it];
-            const int s = u / a.P, p = u % a.P;
+            const int l = u >> kUnitShift, lu = u & kUnitMask;
+            const LinDesc& L = a.lins[l];
+            const int P = L.P;
+            const int s = lu / P, p = lu % P;
             const int acc = t & 1;
             if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
                 if (lane == 0) raise();
@@ -222,17 +230,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
+            if (P == 1) {
+                // whole strip in one unit: no partial sums
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                continue;
+            }
             // this unit's partial: workspace[s][p][row][0..15]
-            float4* dst = reinterpret_cast<float4*>(a.partial + (((size_t)s * a.P + p) * 128 + row) * kBN);
+            float4* dst = reinterpret_cast<float4*>(L.partial + (((size_t)s * P + p) * 128 + row) * kBN);
 #pragma unroll
             for (int c = 0; c < kBN / 4; ++c)
                 dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
                                      __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
-            __threadfence();
             epi_bar();
             if (threadIdx.x == 64) {
-                const unsigned old = atomicAdd(&a.counters[s], 1u);
-                *last_flag = (old == (unsigned)(a.P - 1));
+                // the barrier orders the other epilogue threads' stores before
+                // this fence, which releases them with the arrival
+                __threadfence();
+                const unsigned old = atomicAdd(&L.counters[s], 1u);
+                *last_flag = (old == (unsigned)(P - 1));
             }
             epi_bar();
             if (*last_flag) {
@@ -240,9 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float sum[kBN];
 #pragma unroll
                 for (int c = 0; c < kBN; ++c) sum[c] = 0.f;
-                for (int pp = 0; pp < a.P; ++pp) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        a.partial + (((size_t)s * a.P + pp) * 128 + row) * kBN);
+                for (int pp = 0; pp < P; ++pp) {
+                    const float4* src =
+                        reinterpret_cast<const float4*>(L.partial + (((size_t)s * P + pp) * 128 + row) * kBN);
 #pragma unroll
                     for (int c = 0; c < kBN / 4; ++c) {
                         const float4 f = __ldcg(src + c);
@@ -252,11 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sum[4 * c + 3] += f.w;
                     }
                 }
-                __nv_bfloat16* yc = a.Y + (size_t)s * kStrip + row;
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
-                    if (c < a.M) yc[(size_t)c * a.N] = __float2bfloat16_rn(sum[c]);
-                if (threadIdx.x == 64) a.counters[s] = 0u;  // re-armed for the next call
+                    if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(sum[c]);
+                if (threadIdx.x == 64) L.counters[s] = 0u;  // re-armed for the next call
             }
         }
     }
@@ -275,8 +292,8 @@ cudaError_t decode_prepare() {
     return cudaFuncSetAttribute(hybrid_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-cudaError_t launch_decode(const CUtensorMap& tmap_x, const DecodeArgs& a, int grid, cudaStream_t st) {
-    hybrid_decode_kernel<<<grid, kThreads, kSmemBytes, st>>>(tmap_x, a);
+cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st) {
+    hybrid_decode_kernel<<<grid, kThreads, kSmemBytes, st>>>(maps, a);
     return cudaGetLastError();
 }
 

@@ -52,7 +52,7 @@ struct Abort {
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs a) {
+    hybrid_gemm_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
     using C = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -83,7 +83,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -107,10 +106,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
-                const int s = u / a.MB, j = u % a.MB;
-                const uint32_t* trow = a.slab + (size_t)s * a.KB;
-                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
-                for (int b = 0; b < a.KB; ++b) {
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int s = lu / a.MB, j = lu % a.MB;
+                const uint32_t* trow = L.slab + (size_t)s * L.KB;
+                const uint32_t* mrow = L.meta + (size_t)s * L.KC;
+                const uint8_t* packed = L.packed;
+                const CUtensorMap* tmap_x = &maps.x[l];
+                const int KB = L.KB;
+                for (int b = 0; b < KB; ++b) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ab.raise();
                         ok = false;
@@ -120,11 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
                     const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
                     mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + C::kStageBBytes);
-                    bulk_load(sA + stage * kStageABytes, a.packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    bulk_load(sA + stage * kStageABytes, packed + slab_offset_bytes(d), bytes_a, &full[stage]);
                     if (first)
                         bulk_load(sA + stage * kStageABytes + kSparseValBytes,
-                                  a.packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes, &full[stage]);
-                    tma_load_2d(sB + stage * C::kStageBBytes, &tmap_x, &full[stage], b * kSlabK, j * BN);
+                                  packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes, &full[stage]);
+                    tma_load_2d(sB + stage * C::kStageBBytes, tmap_x, &full[stage], b * kSlabK, j * BN);
                     ++issued;
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -159,15 +163,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool any_mma = false;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
-                const int s = u / a.MB;
-                const uint32_t* trow = a.slab + (size_t)s * a.KB;
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int s = lu / a.MB;
+                const uint32_t* trow = L.slab + (size_t)s * L.KB;
+                const int KB = L.KB;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
                     ab.raise();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int b = 0; b < a.KB; ++b) {
+                for (int b = 0; b < KB; ++b) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) {
                         ab.raise();
                         ok = false;
@@ -226,7 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         for (int it = w_begin; it < w_end; ++it) {
             const int u = a.work[it];
-            const int s = u / a.MB, j = u % a.MB;
+            const int l = u >> kUnitShift, lu = u & kUnitMask;
+            const int N = a.lins[l].N;
+            const int s = lu / a.MB, j = lu % a.MB;
             if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag)) {
                 if (lane == 0) ab.raise();
                 break;
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int n = s * kStrip + q * 32 + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            __nv_bfloat16* yc = a.Y + n;
+            __nv_bfloat16* yc = a.Y[l] + n;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
@@ -244,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (m0 + 32 <= a.M) {
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
-                        yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                        yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
                 } else {
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
                         if (m0 + c < a.M)
-                            yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                            yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
                 }
             }
             tc_fence_before();
@@ -280,8 +289,8 @@ cudaError_t set_attr() {
 
 cudaError_t gemm_prepare_single() { return set_attr<kGemmBN>(); }
 
-cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmArgs& a, int grid, cudaStream_t st) {
-    hybrid_gemm_kernel<kGemmBN><<<grid, kThreads, Cfg<kGemmBN>::kSmemBytes, st>>>(tmap_x, a);
+cudaError_t launch_gemm(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st) {
+    hybrid_gemm_kernel<kGemmBN><<<grid, kThreads, Cfg<kGemmBN>::kSmemBytes, st>>>(maps, a);
     return cudaGetLastError();
 }
 

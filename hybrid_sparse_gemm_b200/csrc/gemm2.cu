@@ -108,9 +108,7 @@ __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    hybrid_gemm2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a16,
-                        const __grid_constant__ CUtensorMap tm_a8, const __grid_constant__ CUtensorMap tm_e,
-                        const Gemm2Args a) {
+    hybrid_gemm2_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -144,10 +142,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tm_x);
-        prefetch_tmap(&tm_a16);
-        prefetch_tmap(&tm_a8);
-        prefetch_tmap(&tm_e);
     }
     if (warp == 1) {
         tmem_alloc2(tmem_slot, kTmemCols);
@@ -175,12 +169,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
-                const int p = u / a.MB, j = u % a.MB;
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int p = lu / a.MB, j = lu % a.MB;
                 int s = 2 * p + (int)rank;
-                if (s >= a.S) s = 2 * p;  // odd last strip: duplicate
-                const uint32_t* trow = a.gemm + (size_t)s * a.KB;
-                const uint32_t* mrow = a.meta + (size_t)s * a.KC;
-                for (int b = 0; b < a.KB; ++b) {
+                if (s >= L.S) s = 2 * p;  // odd last strip: duplicate
+                const uint32_t* trow = L.gemm + (size_t)s * L.KB;
+                const uint32_t* mrow = L.meta + (size_t)s * L.KC;
+                const int KB = L.KB;
+                const CUtensorMap* tm_x = &maps.x[l];
+                const CUtensorMap* tm_a16 = &maps.a16[l];
+                const CUtensorMap* tm_a8 = &maps.a8[l];
+                const CUtensorMap* tm_e = &maps.e[l];
+                for (int b = 0; b < KB; ++b) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         raise();
                         ok = false;
@@ -195,10 +196,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                     (first ? kMetaBytes : 0) + kStageB));
                     const uint32_t dst_a = smem_u32(sA + stage * kStageA);
                     const int row = (int)(slab_offset_bytes(d) >> 7);
-                    tma_load_2d_pair(dst_a, sp ? &tm_a8 : &tm_a16, bar, 0, row);
+                    tma_load_2d_pair(dst_a, sp ? tm_a8 : tm_a16, bar, 0, row);
                     if (first)
-                        tma_load_2d_pair(dst_a + kSparseValBytes, &tm_e, bar, 0, (int)(mrow[b >> 1] >> 3));
-                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tm_x, bar, b * kSlabK,
+                        tma_load_2d_pair(dst_a + kSparseValBytes, tm_e, bar, 0, (int)(mrow[b >> 1] >> 3));
+                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), tm_x, bar, b * kSlabK,
                                      j * kGemm2BN + (int)rank * kHalf);
                     ++issued;
                     if (++stage == kStages) {
@@ -234,8 +235,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
-                const int p = u / a.MB;
-                const uint32_t* trow = a.gemm + (size_t)(2 * p) * a.KB;
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int p = lu / a.MB;
+                const uint32_t* trow = L.gemm + (size_t)(2 * p) * L.KB;
+                const int KB = L.KB;
                 const int acc = t & 1;
                 if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
                     raise();
@@ -245,7 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
                 const uint32_t e_base = tmem_base + (uint32_t)((1 - acc) * kAccCols + kETail);
                 bool e_ready = (t == 0);
-                for (int b = 0; b < a.KB; ++b) {
+                for (int b = 0; b < KB; ++b) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) {
                         raise();
                         ok = false;
@@ -306,9 +310,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
             const int u = a.work[it];
-            const int p = u / a.MB, j = u % a.MB;
+            const int l = u >> kUnitShift, lu = u & kUnitMask;
+            const int N = a.lins[l].N;
+            const int p = lu / a.MB, j = lu % a.MB;
             const int s = 2 * p + (int)rank;
-            const bool store = s < a.S;
+            const bool store = s < a.lins[l].S;
             const int acc = t & 1;
             if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
                 if (lane == 0) raise();
@@ -317,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int n = s * kStrip + q * 32 + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
-            __nv_bfloat16* yc = a.Y + n;
+            __nv_bfloat16* yc = a.Y[l] + n;
 #pragma unroll 1
             for (int c0 = kAccCols - 32; c0 >= 0; c0 -= 32) {
                 uint32_t v[32];
@@ -334,12 +340,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (m0 + 32 <= a.M) {
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
-                        yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                        yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
                 } else {
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
                         if (m0 + c < a.M)
-                            yc[(size_t)(m0 + c) * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                            yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
                 }
             }
             tc_fence_before();
@@ -381,9 +387,8 @@ cudaError_t gemm_prepare_pair(int* max_clusters) {
     return cudaSuccess;
 }
 
-cudaError_t launch_gemm2(const CUtensorMap& tmap_x, const CUtensorMap& tm_a16, const CUtensorMap& tm_a8,
-                         const CUtensorMap& tm_e, const Gemm2Args& a, int clusters, cudaStream_t st) {
-    hybrid_gemm2_kernel<<<2 * clusters, kThreads, kSmemBytes, st>>>(tmap_x, tm_a16, tm_a8, tm_e, a);
+cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
+    hybrid_gemm2_kernel<<<2 * clusters, kThreads, kSmemBytes, st>>>(maps, a);
     return cudaGetLastError();
 }
 

@@ -24,28 +24,41 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, const uint32_t
                               const uint32_t* __restrict__ meta_tab, int KB, int KC, int64_t K,
                               uint16_t* __restrict__ Wm);
 
-// Tensor-core kernel, one CTA per 128-row strip x 128-token block.
-struct GemmArgs {
+// The tensor-core kernels run a group of packed linears (one or more weights
+// sharing M, e.g. the projections of one layer) in one persistent launch.
+constexpr int kMaxGroup = 8;
+
+// Static description of one packed linear (device memory, built at pack).
+struct LinDesc {
     const uint8_t* packed;
-    const uint32_t* slab;    // per-strip slab table
-    const uint32_t* meta;    // metadata block table
-    const int* work_off;     // per CTA: [work_off[c], work_off[c+1]) into work
-    const int* work;         // unit = strip * MB + m_block
-    int M, N, KB, KC, MB;
-    __nv_bfloat16* Y;
-    int* status;             // device status word (timeouts)
+    const uint32_t* slab;      // per-strip slab table
+    const uint32_t* meta;      // metadata block table
+    const uint32_t* gemm;      // CTA-pair slab table
+    float* partial;            // decode workspace [S][P][128][16] fp32
+    unsigned* counters;        // decode arrivals per strip, zero between calls
+    int N, S, KB, KC, P;       // P: decode K-parts per strip
 };
 
-// Tensor-core kernel, one CTA pair per 256-row strip pair x 256-token block.
-struct Gemm2Args {
-    const uint32_t* gemm;    // CTA-pair slab table
-    const uint32_t* meta;
-    const int* work_off;     // per cluster
-    const int* work;         // unit = pair * MB + m_block
-    int M, N, S, KB, KC, MB;
-    __nv_bfloat16* Y;
-    int* status;
+// Tensor maps: X of every member (per call) and the packed bytes of every
+// member viewed as 128-byte rows with 128-, 64- and 16-row boxes.
+struct GroupMaps {
+    CUtensorMap x[kMaxGroup];
+    CUtensorMap a16[kMaxGroup], a8[kMaxGroup], e[kMaxGroup];
 };
+
+// Per-call arguments. A work unit is (member << 24) | local index, the local
+// index being strip*MB + token block (single-CTA), pair*MB + token block
+// (CTA pair) or strip*P + part (decode).
+struct GroupArgs {
+    const LinDesc* lins;
+    __nv_bfloat16* Y[kMaxGroup];
+    const int* work_off;       // per CTA (or per CTA pair): [work_off[c], work_off[c+1])
+    const int* work;
+    int M, MB;
+    int* status;               // device status word (timeouts)
+};
+constexpr int kUnitShift = 24;
+constexpr int kUnitMask = (1 << kUnitShift) - 1;
 
 struct GemvArgs {
     const uint8_t* packed;
@@ -56,29 +69,14 @@ struct GemvArgs {
     int M, N, K, KB, KC;
 };
 
-// Decode kernel (M <= 16): split-K over persistent CTAs, partials reduced by
-// the last CTA of each strip.
-struct DecodeArgs {
-    const uint8_t* packed;
-    const uint32_t* slab;
-    const uint32_t* meta;
-    const int* work_off;     // per CTA
-    const int* work;         // unit = strip * P + part
-    int M, N, KB, KC, P;
-    float* partial;          // [S][P][128][16] fp32 workspace
-    unsigned* counters;      // [S] arrivals per strip, zero between calls
-    __nv_bfloat16* Y;
-    int* status;
-};
-
 // Launchers (return cudaError_t of the launch).
-cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmArgs& a, int grid, cudaStream_t st);
-cudaError_t launch_gemm2(const CUtensorMap& tmap_x, const CUtensorMap& tm_a16, const CUtensorMap& tm_a8,
-                         const CUtensorMap& tm_e, const Gemm2Args& a, int clusters, cudaStream_t st);
+cudaError_t launch_gemm(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
+cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
+cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
-cudaError_t launch_decode(const CUtensorMap& tmap_x, const DecodeArgs& a, int grid, cudaStream_t st);
+cudaError_t gemm_prepare_single();
+cudaError_t gemm_prepare_pair(int* max_clusters);
 cudaError_t decode_prepare();
-cudaError_t gemm_prepare(int* max_pair_clusters);  // one-time function attributes, cluster occupancy
 
 constexpr int kGemmBN = 128;   // tokens per CTA tile (single-CTA kernel)
 constexpr int kGemm2BN = 256;  // tokens per CTA-pair tile

@@ -39,6 +39,7 @@ extern "C" {
 #endif
 
 typedef struct patch_handle_s* patch_handle;
+typedef struct patch_group_s* patch_group;
 
 typedef enum {
     PATCH_OK = 0,
@@ -177,6 +178,35 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
  */
 patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                                   void* stream);
+
+/*
+ * patch_group_create - bind several packed linears that are run with the same
+ * token count M (for example the q, k, v, o, gate, up and down projections of
+ * one layer) so that one persistent launch computes all of them.
+ *
+ *   handles  host array of n handles, all on the current device; 1 <= n <= 8.
+ *            The handles must outlive the group.
+ *   out      receives the group.
+ * The group owns only a small device descriptor array and its cached
+ * schedules (allocated on the first call for each M, like patch_linear).
+ */
+patch_status patch_group_create(const patch_handle* handles, int n, patch_group* out);
+
+/*
+ * patch_group_linear - Y_i = X_i . (W_i (.) Mask_i)^T for every member i in
+ * one launch (the GEMV_SIMT path runs one launch per member).
+ *
+ *   X  host array of n dev pointers, X_i: M x K_i bf16, 16-byte aligned.
+ *   Y  host array of n dev pointers, Y_i: M x N_i bf16, 16-byte aligned.
+ *      Inputs may be shared between members (q, k, v read the same X).
+ *   M, path, stream as for patch_linear_path.
+ * Device timeouts are reported through patch_check on the first member.
+ */
+patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, void* const* Y, int path,
+                                void* stream);
+
+/* patch_group_free - release a group (not its handles). NULL is ignored. */
+void patch_group_free(patch_group g);
 
 /* patch_unpack - write W (.) Mask (N*K bf16, dev, row-major, 16-byte aligned)
  * decoded from the packed weights. */

@@ -337,3 +337,55 @@ def test_config5_llama2_13b_tiles(hsg, oracle_lib, R, C):
     shapes = [l for l in synth.llama2_13b() if l.name in ("q", "gate", "down")]
     _layer(hsg, oracle_lib, shapes, 8192, [0.9] * 3, R=R, C=C, tag=f"cfg5-{R}x{C}", rows_n=64,
            check_bytes=(R == 64 and C == 64))
+
+
+# --------------------------------------------------------------- groups ---
+
+@pytest.mark.parametrize("path_name,M", [("GEMM_PAIR", 300), ("GEMM_SINGLE", 130), ("GEMV", 16), ("GEMV", 3),
+                                         ("GEMV_SIMT", 5), ("AUTO", 520), ("AUTO", 1)])
+def test_group_matches_members(hsg, oracle_lib, path_name, M):
+    """One launch over several linears (shared and separate inputs, mixed tile
+    shapes and 2:4 fractions) equals the members run one by one, bit for bit,
+    and each member is within tolerance of the oracle."""
+    specs = [(384, 256, 128, 128, 0.9, "a"), (128, 256, 128, 64, 0.5, "a"), (640, 384, 64, 64, 0.7, "b"),
+             (256, 448, 128, 64, 0.0, "c")]
+    Xs = {"a": synth.normal_bf16((M, 256), 1.0, "cuda", "gx", "a", M),
+          "b": synth.normal_bf16((M, 384), 1.0, "cuda", "gx", "b", M),
+          "c": synth.normal_bf16((M, 448), 1.0, "cuda", "gx", "c", M)}
+    probs, lins, xs = [], [], []
+    for i, (N, K, R, C, f, xk) in enumerate(specs):
+        p = synth.make_problem(N, K, 0, R=R, C=C, frac=f, seed=i, device="cuda", tag=f"grp{i}")
+        probs.append(p)
+        lins.append(pack(hsg, p))
+        xs.append(Xs[xk])
+    path = getattr(hsg, "PATH_" + path_name)
+    group = hsg.LinearGroup(lins)
+    Yg = group(xs, path=path)
+    Yi = [lin(x, path=path) for lin, x in zip(lins, xs)]
+    torch.cuda.synchronize()
+    lins[0].check()
+    for i, (p, x) in enumerate(zip(probs, xs)):
+        assert torch.equal(Yg[i], Yi[i]), f"member {i} differs from its own launch"
+        assert_close(Yg[i], oracle_lib, x, p.W, p.bits, p.keep, rows=sample_rows(M, 64, i),
+                     what=f"group {path_name} member {i}")
+    # a second call reuses the cached schedule
+    Yg2 = group(xs, path=path)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(Yg, Yg2))
+    group.free()
+    for lin in lins:
+        lin.free()
+
+
+def test_group_argument_errors(hsg):
+    import ctypes
+    lib = hsg.library()
+    g = ctypes.c_void_p()
+    assert lib.patch_group_create(None, 1, ctypes.byref(g)) == 1
+    p = synth.make_problem(128, 64, 0, R=128, C=64, seed=0, device="cuda", tag="ge")
+    lin = pack(hsg, p)
+    arr = (ctypes.c_void_p * 9)(*([lin.handle] * 9))
+    assert lib.patch_group_create(arr, 9, ctypes.byref(g)) == 1
+    assert lib.patch_group_create(arr, 0, ctypes.byref(g)) == 1
+    assert lib.patch_group_linear(None, None, 4, None, 0, None) == 1
+    lin.free()
