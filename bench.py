@@ -236,14 +236,14 @@ def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
     import oracle
     oracle.build()
     shapes = synth.llama32_1b()
-    probs = [synth.make_problem(l.N, l.K, 64, R=128, C=128, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
+    probs = [synth.make_problem(l.N, l.K, 4096, R=128, C=128, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
              for l in shapes]
     # calibrate on one row of every linear
     t0 = time.perf_counter()
     for p in probs:
         oracle.linear(p.X[:1], p.W, p.bits.numpy())
     t1 = time.perf_counter() - t0
-    rows = max(min_rows, min(64, int(budget_s / max(t1, 1e-6))))
+    rows = max(min_rows, min(4096, int(budget_s / max(t1, 1e-6))))
     flops = 0.0
     t0 = time.perf_counter()
     for l, p in zip(shapes, probs):

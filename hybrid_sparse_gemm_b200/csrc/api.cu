@@ -265,6 +265,7 @@ struct patch_group_s {
     DeviceInfo dev;
     int n = 0;
     patch_handle h[kMaxGroup] = {};
+    int parts[kMaxGroup] = {};    // decode K-parts per strip of each member in this group
     LinDesc* lins_dev = nullptr;  // n descriptors
     int* status_dev = nullptr;    // the first member's status word
     std::mutex mu;
@@ -308,9 +309,26 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     g->n = n;
     g->status_dev = hs[0]->status_dev;
     LinDesc d[kMaxGroup];
+    // Decode units: a lone linear keeps its own split (enough units for every
+    // SM); in a group the members' units already fill the GPU, so parts are
+    // made large (each unit's epilogue is then hidden behind streaming).
+    double total = 0.0;
+    for (int i = 0; i < n; ++i)
+        for (double b : hs[i]->plan.strip_bytes) total += b;
+    const double target = std::max(256.0 * 1024.0, total / (4.0 * g->dev.sms));
     for (int i = 0; i < n; ++i) {
         g->h[i] = hs[i];
         d[i] = hs[i]->desc;
+        int P = hs[i]->decode_parts;
+        if (n > 1) {
+            const Plan& pl = hs[i]->plan;
+            double avg = 0.0;
+            for (double b : pl.strip_bytes) avg += b;
+            avg /= std::max(1, pl.S);
+            P = std::max(1, std::min(hs[i]->decode_parts, (int)(avg / target + 0.5)));
+        }
+        g->parts[i] = P;
+        d[i].P = P;
     }
     if (cudaMalloc(&g->lins_dev, sizeof(LinDesc) * n) != cudaSuccess) {
         cudaGetLastError();
@@ -343,7 +361,7 @@ void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std:
             for (int r = 0; r < (int)c.size(); ++r)
                 for (int j = 0; j < mb; ++j) units.push_back({c[r] + 1.0, (l << kUnitShift) | (r * mb + j)});
         } else {
-            const int P = g->h[l]->decode_parts;
+            const int P = g->parts[l];
             for (int s = 0; s < p.S; ++s)
                 for (int q = 0; q < P; ++q)
                     units.push_back({p.strip_bytes[s] / P + 16384.0, (l << kUnitShift) | (s * P + q)});

