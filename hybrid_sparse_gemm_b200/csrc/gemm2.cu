@@ -1,14 +1,20 @@
-// Hybrid dense / 2:4 GEMM on a CTA pair (cta_group::2): Y = X . (W (.) Mask)^T.
+// Hybrid dense / 2:4 GEMM on CTA pairs (cta_group::2): Y = X . (W (.) Mask)^T.
 //
 // Same method as the single-CTA kernel (dense slabs on tcgen05.mma, 2:4 slabs
 // on tcgen05.mma.sp; PATCH abstract, "PATCH: Learnable Tile-level Hybrid
 // Sparsity for LLMs"), on the unit Blackwell's tensor core is built around:
-// two CTAs on neighbouring SMs form one 256 x 256 MMA. CTA r holds the 128
-// weight rows of strip 2p+r (operand A) and tokens [128r, 128r+128) of the
-// block (operand B); each MMA multiplies both A halves by both B halves, so an
-// SM loads half the activations it would need alone. The leader CTA (rank 0)
-// issues every MMA; both CTAs' TMA loads complete on the leader's barriers,
-// and the leader's commits arrive on both CTAs' barriers.
+// two CTAs on neighbouring SMs form one 256 x 256 MMA. CTA r of a pair holds
+// the 128 weight rows of one strip (operand A) and tokens [128r, 128r+128) of
+// the block (operand B); each MMA multiplies both A halves by both B halves,
+// so an SM loads half the activations it would need alone. The pair's leader
+// (even rank) issues every MMA; both CTAs' TMA loads complete on the leader's
+// barriers, and the leader's commits arrive on the CTAs' barriers.
+//
+// With CL = 4 two pairs (four strips) share a cluster and a token block: each
+// activation sub-tile is loaded once and multicast to the CTA of each pair
+// that needs it, halving the activation bytes each SM pulls from L2. The two
+// pairs then advance through the shared stages together (a stage is free
+// when both pairs' MMAs have consumed it).
 //
 // TMEM: each CTA holds its 128 rows x 256 tokens in one of two 256-column
 // accumulators. The 2:4 metadata of the running tile lives in the last four
@@ -17,8 +23,9 @@
 //
 // Both strips of a pair load the same kind of record at every slab (dense
 // images stand in for 2:4 slabs whose partner is dense), so one MMA
-// instruction always covers both. An odd last strip pairs with itself; its
-// second CTA computes a duplicate and stores nothing.
+// instruction always covers both. Strips past the end of the weight (an odd
+// last strip, a last cluster with fewer strips) are replaced by duplicates
+// whose results are not stored.
 #include "kernels.cuh"
 
 namespace patch {
@@ -35,6 +42,7 @@ constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kETail = kAccCols - 4;          // metadata columns inside the idle accumulator
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;   // clears the CTA-in-pair bit of a shared address
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -53,13 +61,23 @@ __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// 2-D TMA load whose completion is counted on the leader CTA's barrier.
+// 2-D TMA load whose completion is counted on the pair leader's barrier.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
                                                  int c0, int c1) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+// The same load written to the same offset in every CTA of `mask`; each
+// destination's bytes complete on its own pair leader's barrier.
+__device__ __forceinline__ void tma_load_2d_pair_mc(uint32_t dst, const CUtensorMap* map, uint32_t bar_local,
+                                                    int c0, int c1, uint16_t mask) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.multicast::cluster"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(map), "r"(bar_local & kPeerMask), "r"(c0), "r"(c1), "h"(mask)
         : "memory");
 }
 __device__ __forceinline__ void mma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -83,12 +101,13 @@ __device__ __forceinline__ void mma2_sp_bf16(uint32_t d_tmem, uint64_t adesc, ui
 __device__ __forceinline__ void cp2_128x128b(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
-// Commit of the leader's MMAs, arriving on the barrier at this offset in both CTAs.
-__device__ __forceinline__ void commit2_both(uint64_t* bar) {
+// Commit of the leader's MMAs, arriving on the barrier at this offset in every
+// CTA of `mask`.
+__device__ __forceinline__ void commit2_mask(uint64_t* bar, uint16_t mask) {
     asm volatile(
-        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-            smem_u32(bar))
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(mask)
         : "memory");
 }
 __device__ __forceinline__ void commit2_local(uint64_t* bar) {
@@ -107,19 +126,22 @@ __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int CL>
+__global__ void __launch_bounds__(kThreads, 1)
     hybrid_gemm2_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
+    constexpr int kStrips = CL;            // strips per cluster (one per CTA)
+    constexpr int kPairs = CL / 2;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kStageA;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
-    uint64_t* full = bars;                  // leader: both CTAs' bytes of a stage
-    uint64_t* empty = bars + kStages;       // both: stage consumed by the MMAs
-    uint64_t* acc_full = bars + 2 * kStages;  // both: accumulator ready
-    uint64_t* acc_empty = acc_full + 2;     // leader: 8 epilogue warps drained it
-    uint64_t* e_free = acc_full + 4;        // leader: 8 epilogue warps read its tail
+    uint64_t* full = bars;                    // pair leader: both CTAs' bytes of a stage
+    uint64_t* empty = bars + kStages;         // every CTA: stage consumed by every pair's MMAs
+    uint64_t* acc_full = bars + 2 * kStages;  // both CTAs of a pair: accumulator ready
+    uint64_t* acc_empty = acc_full + 2;       // pair leader: 8 epilogue warps drained it
+    uint64_t* e_free = acc_full + 4;          // pair leader: 8 epilogue warps read its tail
     uint64_t* drain = acc_full + 6;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -127,12 +149,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
-    const int cl = blockIdx.x >> 1;
+    const uint32_t pr = rank & 1u;          // CTA within its pair
+    const uint32_t pair = rank >> 1;        // pair within the cluster
+    const uint32_t leader = rank & ~1u;
+    const uint16_t pair_mask = (uint16_t)(3u << leader);
+    const uint16_t all_mask = (uint16_t)((1u << CL) - 1u);
+    const int cl = blockIdx.x / CL;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
+            mbar_init(&empty[i], kPairs);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
@@ -149,12 +176,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();  // barriers of both CTAs initialised before any remote use
+    cluster_sync();  // barriers of every CTA initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     auto raise = [&]() {
         *abort_flag = 1;
         atomicCAS(a.status, 0, kStatusTimeout);
+    };
+    // strip this CTA loads for cluster-unit c of a member with S strips
+    auto own_strip = [&](int c, int S) {
+        int s = kStrips * c + (int)rank;
+        if (s >= S) s = kStrips * c + (int)pr;
+        if (s >= S) s = kStrips * c;
+        return s;
     };
 
     const int w_begin = a.work_off[cl];
@@ -162,7 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- producer (both CTAs) ----------------
+            // ---------------- producer (every CTA) ----------------
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -171,9 +205,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
-                const int p = lu / a.MB, j = lu % a.MB;
-                int s = 2 * p + (int)rank;
-                if (s >= L.S) s = 2 * p;  // odd last strip: duplicate
+                const int c = lu / a.MB, j = lu % a.MB;
+                const int s = own_strip(c, L.S);
                 const uint32_t* trow = L.gemm + (size_t)s * L.KB;
                 const uint32_t* mrow = L.meta + (size_t)s * L.KC;
                 const int KB = L.KB;
@@ -189,8 +222,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     const uint32_t d = trow[b];
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
-                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
-                    if (rank == 0)
+                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), leader);
+                    if (pr == 0)
                         mbar_arrive_expect_tx(&full[stage],
                                               2u * ((sp ? kSparseValBytes : kDenseSlabBytes) +
                                                     (first ? kMetaBytes : 0) + kStageB));
@@ -199,8 +232,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tma_load_2d_pair(dst_a, sp ? tm_a8 : tm_a16, bar, 0, row);
                     if (first)
                         tma_load_2d_pair(dst_a + kSparseValBytes, tm_e, bar, 0, (int)(mrow[b >> 1] >> 3));
-                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), tm_x, bar, b * kSlabK,
-                                     j * kGemm2BN + (int)rank * kHalf);
+                    const int tok = j * kGemm2BN + (int)pr * kHalf;
+                    if (CL == 2) {
+                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), tm_x, bar, b * kSlabK, tok);
+                    } else {
+                        // this CTA fetches half of its 128 activation rows and
+                        // multicasts them to the same CTA of the other pair
+                        const uint32_t off = pair * (kStageB / 2);
+                        tma_load_2d_pair_mc(smem_u32(sB + stage * kStageB) + off, tm_x, smem_u32(&full[stage]),
+                                            b * kSlabK, tok + (int)pair * (kHalf / 2),
+                                            (uint16_t)((1u << pr) | (1u << (pr + 2))));
+                    }
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -208,9 +250,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (rank == 0) {
+            if (pr == 0) {
                 // Bounded wait for the loads of the last stages, whatever the
-                // abort flag says, so none lands after the pair exits.
+                // abort flag says, so none lands after the cluster exits.
                 int st = stage;
                 uint32_t ph = phase;
                 for (int i = 0; i < kStages && i < issued; ++i) {
@@ -225,8 +267,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
-            // ---------------- MMA issuer (leader) ----------------
+        if (lane == 0 && pr == 0) {
+            // ---------------- MMA issuer (pair leader) ----------------
             const uint32_t idesc_d = idesc_bf16(256, kGemm2BN, false);
             const uint32_t idesc_s = idesc_bf16(256, kGemm2BN, true);
             int stage = 0;
@@ -237,8 +279,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
-                const int p = lu / a.MB;
-                const uint32_t* trow = L.gemm + (size_t)(2 * p) * L.KB;
+                const int c = lu / a.MB;
+                const uint32_t* trow = L.gemm + (size_t)own_strip(c, L.S) * L.KB;
                 const int KB = L.KB;
                 const int acc = t & 1;
                 if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
@@ -288,14 +330,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                     }
                     any_mma = true;
-                    commit2_both(&empty[stage]);
+                    commit2_mask(&empty[stage], all_mask);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                commit2_both(&acc_full[acc]);
+                commit2_mask(&acc_full[acc], pair_mask);
             }
             if (*abort_flag && any_mma) {
                 commit2_local(drain);
@@ -305,15 +347,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+        // ---------------- epilogue (warps 2..5, every CTA) ----------------
         const int q = warp & 3;
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const int N = a.lins[l].N;
-            const int p = lu / a.MB, j = lu % a.MB;
-            const int s = 2 * p + (int)rank;
+            const int c = lu / a.MB, j = lu % a.MB;
+            const int s = kStrips * c + (int)rank;
             const bool store = s < a.lins[l].S;
             const int acc = t & 1;
             if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
@@ -333,63 +375,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // The tail (metadata columns of the next tile) is read: release it.
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) remote_arrive(map_to_rank(smem_u32(&e_free[acc]), 0));
+                    if (lane == 0) remote_arrive(map_to_rank(smem_u32(&e_free[acc]), leader));
                 }
                 if (!store) continue;
                 const int m0 = j * kGemm2BN + c0;
                 if (m0 + 32 <= a.M) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                    for (int cc = 0; cc < 32; ++cc)
+                        yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (m0 + c < a.M)
-                            yc[(size_t)(m0 + c) * N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                    for (int cc = 0; cc < 32; ++cc)
+                        if (m0 + cc < a.M)
+                            yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[acc]), 0));
+            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[acc]), leader));
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    cluster_sync();  // no CTA leaves while its partner may still signal it
+    cluster_sync();  // no CTA leaves while another may still signal it
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc2(tmem_base, kTmemCols);
     }
 }
 
-}  // namespace
-
-cudaError_t gemm_prepare_pair(int* max_clusters) {
+template <int CL>
+cudaError_t prepare(int* max_clusters) {
     cudaError_t e =
-        cudaFuncSetAttribute(hybrid_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(hybrid_gemm2_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2, 1, 1);
+    cfg.gridDim = dim3(CL, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.x = CL;
     attr.val.clusterDim.y = 1;
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm2_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm2_kernel<CL>, &cfg);
     if (e != cudaSuccess) return e;
     *max_clusters = n;
     return cudaSuccess;
 }
 
-cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
-    hybrid_gemm2_kernel<<<2 * clusters, kThreads, kSmemBytes, st>>>(maps, a);
-    return cudaGetLastError();
+template <int CL>
+cudaError_t launch(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = CL;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, hybrid_gemm2_kernel<CL>, maps, a);
+}
+
+}  // namespace
+
+cudaError_t gemm_prepare_pair(int* max_pair_clusters, int* max_quad_clusters) {
+    cudaError_t e = prepare<2>(max_pair_clusters);
+    if (e != cudaSuccess) return e;
+    return prepare<4>(max_quad_clusters);
+}
+
+cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, int cluster_ctas, cudaStream_t st) {
+    return cluster_ctas == 4 ? launch<4>(maps, a, clusters, st) : launch<2>(maps, a, clusters, st);
 }
 
 }  // namespace patch

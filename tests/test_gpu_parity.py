@@ -188,6 +188,24 @@ def test_decode_repeat_and_interleave(hsg, oracle_lib):
     lin.free()
 
 
+@pytest.mark.parametrize("N", [512, 1024, 3200])
+@pytest.mark.parametrize("M", [256, 300, 1000])
+@pytest.mark.parametrize("R,C,frac", [(128, 128, 0.9), (64, 64, 0.3), (128, 64, 1.0)])
+def test_pair_clusters_of_four(hsg, oracle_lib, N, M, R, C, frac):
+    """Strip counts that run two CTA pairs per cluster (shared activations),
+    including a last cluster with one real strip and three duplicates."""
+    p = synth.make_problem(N, 512, M, R=R, C=C, frac=frac, seed=N + M, device="cuda")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMM_QUAD)
+    Y2 = lin(p.X, path=hsg.PATH_GEMM_QUAD)
+    Yp = lin(p.X, path=hsg.PATH_GEMM_PAIR)
+    torch.cuda.synchronize()
+    lin.check()
+    assert torch.equal(Y, Y2) and torch.equal(Y, Yp)
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(M, 96, N), what=f"quad N={N} M={M}")
+    lin.free()
+
+
 def test_single_strip_single_slab(hsg, oracle_lib):
     for frac in (0.0, 1.0):
         p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")
