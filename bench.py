@@ -197,8 +197,7 @@ def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=Fals
     for _ in range(warmup):
         run_step(hsg, model, X, Y, stream, path)
     torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
+    hdist.barrier(dist_on)
     ev = None
     if per_launch:
         ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -211,10 +210,7 @@ def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=Fals
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
-    if dist_on:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = hdist.max_over_ranks(ms, dist_on, device="cuda")
     launch_ms = None
     if ev:
         launch_ms = [[a.elapsed_time(b) for a, b in row] for row in ev]
@@ -350,13 +346,8 @@ def main():
 
     import hybrid_sparse_gemm_b200 as hsg
 
-    dist_on = world > 1
-    if dist_on:
-        torch.cuda.set_device(local_rank)
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
+    torch.cuda.set_device(local_rank if world > 1 else 0)
+    dist_on = hdist.init("nccl")
     stream = torch.cuda.Stream()
     peaks = load_peaks()
     M = args.M
@@ -378,7 +369,7 @@ def main():
     _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True)
     kern_ms = statistics.mean(sum(row) for row in launch_ms)
     achieved = exec_flops / (kern_ms / 1e3) / 1e12
-    value = world * F / (ms_h / 1e3) / 1e12
+    value = hdist.job_rate(F, world, ms_h) / 1e12
 
     sweep = None
     if not args.no_sweep:
@@ -394,7 +385,7 @@ def main():
                 t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on)
                 free_model(mdl)
                 del mdl
-            sweep[str(f)] = {"tflops": world * F / (t / 1e3) / 1e12, "speedup_vs_dense": ms_d / t,
+            sweep[str(f)] = {"tflops": hdist.job_rate(F, world, t) / 1e12, "speedup_vs_dense": ms_d / t,
                              "ms_per_step": t}
 
     e2e = None
@@ -407,8 +398,7 @@ def main():
         e2e_steps = max(1, min(args.steps, 3))
         for m, yh in zip(mem, Yh):  # warm-up
             hsg.patch_linear_host(m[0].handle, Xh[id(m[5])], yh, stream)
-        if dist_on:
-            torch.distributed.barrier()
+        hdist.barrier(dist_on)
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         s.record(stream)
@@ -418,11 +408,8 @@ def main():
         e.record(stream)
         torch.cuda.synchronize()
         ms_e = s.elapsed_time(e) / e2e_steps
-        if dist_on:
-            t = torch.tensor([ms_e], device="cuda")
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e = float(t.item())
-        e2e = {"value": world * F / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        ms_e = hdist.max_over_ranks(ms_e, dist_on, device="cuda")
+        e2e = {"value": hdist.job_rate(F, world, ms_e) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
 
     free_model(dense_model)
@@ -461,8 +448,7 @@ def main():
         }
         print(json.dumps(line))
     free_model(model)
-    if dist_on:
-        torch.distributed.destroy_process_group()
+    hdist.shutdown(dist_on)
 
 
 if __name__ == "__main__":
