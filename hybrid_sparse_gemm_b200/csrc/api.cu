@@ -71,7 +71,7 @@ patch_status check_flags(const uint8_t* flags, int64_t n) {
 struct DeviceInfo {
     int sms = 0;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
-    int quad_clusters = 0;  // co-resident 4-CTA clusters (two pairs sharing activations)
+    int wide_clusters = 0;  // co-resident CTA pairs of the two-strips-per-CTA kernel
 };
 std::mutex g_dev_mu;
 std::map<int, DeviceInfo> g_dev;
@@ -90,7 +90,9 @@ patch_status prepare_device(int* dev_out, DeviceInfo* info_out) {
         DeviceInfo di;
         di.sms = sms;
         PATCH_CUDA(gemm_prepare_single());
-        PATCH_CUDA(gemm_prepare_pair(&di.pair_clusters, &di.quad_clusters));
+        PATCH_CUDA(gemm_prepare_pair(&di.pair_clusters));
+        PATCH_CUDA(gemm_prepare_wide(&di.wide_clusters));
+        if (di.wide_clusters <= 0) di.wide_clusters = 1;
         PATCH_CUDA(decode_prepare());
         if (di.pair_clusters <= 0) di.pair_clusters = 1;
         it = g_dev.emplace(dev, di).first;
@@ -350,6 +352,23 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
 // work (dense 1, 2:4 1/2) + one epilogue; kernel 1: (strip pair, token block),
 // same costs; kernel 3: (four strips, token block), the slower pair's cost;
 // kernel 2: (strip, K-part), cost = streamed bytes of the part.
+// Per tensor-core kernel (0 single CTA, 1 CTA pair, 2 decode, 4 CTA pair with
+// two strips per CTA): tokens per tile,
+// activation rows per TMA box, weight rows of a work unit, persistent slots.
+int kernel_bn(int kernel) {
+    return kernel == 0 ? kGemmBN : kernel == 2 ? kDecodeBN : kernel == 4 ? kGemm22BN : kGemm2BN;
+}
+int kernel_box_rows(int kernel) {
+    return kernel == 1 ? kGemm2BN / 2 : kernel == 4 ? kGemm22BN / 2 : kernel_bn(kernel);
+}
+int64_t kernel_rows(const Plan& p, int kernel) {
+    const int64_t pairs = (int64_t)p.pair_cost.size();
+    return kernel == 0 ? (int64_t)p.strip_cost.size() : kernel == 1 ? pairs : (pairs + 1) / 2;
+}
+int kernel_slots(const DeviceInfo& d, int kernel) {
+    return kernel == 1 ? d.pair_clusters : kernel == 4 ? d.wide_clusters : d.sms;
+}
+
 void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
     struct Unit {
         double cost;
@@ -362,11 +381,12 @@ void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std:
             const std::vector<double>& c = kernel == 0 ? p.strip_cost : p.pair_cost;
             for (int r = 0; r < (int)c.size(); ++r)
                 for (int j = 0; j < mb; ++j) units.push_back({c[r] + 1.0, (l << kUnitShift) | (r * mb + j)});
-        } else if (kernel == 3) {
+        } else if (kernel == 4) {
+            // a strip quad issues both of its pairs' MMAs at every slab
             const std::vector<double>& c = p.pair_cost;
             for (int r = 0; r < (int)(c.size() + 1) / 2; ++r) {
-                const double cost = std::max(c[2 * r], 2 * r + 1 < (int)c.size() ? c[2 * r + 1] : 0.0);
-                for (int j = 0; j < mb; ++j) units.push_back({cost + 1.0, (l << kUnitShift) | (r * mb + j)});
+                const double cost = c[2 * r] + (2 * r + 1 < (int)c.size() ? c[2 * r + 1] : c[2 * r]);
+                for (int j = 0; j < mb; ++j) units.push_back({cost + 2.0, (l << kUnitShift) | (r * mb + j)});
             }
         } else {
             const int P = g->parts[l];
@@ -376,8 +396,7 @@ void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std:
         }
     }
     std::stable_sort(units.begin(), units.end(), [](const Unit& x, const Unit& y) { return x.cost > y.cost; });
-    const int slots = kernel == 1 ? g->dev.pair_clusters : kernel == 3 ? g->dev.quad_clusters : g->dev.sms;
-    const int grid = std::max(1, std::min(slots, (int)units.size()));
+    const int grid = std::max(1, std::min(kernel_slots(g->dev, kernel), (int)units.size()));
     using Item = std::pair<double, int>;
     std::priority_queue<Item, std::vector<Item>, std::greater<Item>> pq;
     for (int c = 0; c < grid; ++c) pq.push({0.0, c});
@@ -461,7 +480,7 @@ int choose_kernel(patch_group g, int path) {
     (void)g;
     if (path == PATCH_PATH_GEMM_SINGLE) return 0;
     if (path == PATCH_PATH_GEMV) return 2;
-    if (path == PATCH_PATH_GEMM_QUAD) return 3;
+    if (path == PATCH_PATH_GEMM_WIDE) return 4;
     return 1;
 }
 
@@ -478,17 +497,15 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
         return PATCH_OK;
     }
     if (path != PATCH_PATH_GEMV && path != PATCH_PATH_GEMM_SINGLE && path != PATCH_PATH_GEMM_PAIR &&
-        path != PATCH_PATH_GEMM_QUAD)
+        path != PATCH_PATH_GEMM_WIDE)
         return fail(PATCH_ERR_ARG, "unknown path %d", path);
-    if (path == PATCH_PATH_GEMM_QUAD && g->dev.quad_clusters <= 0)
-        return fail(PATCH_ERR_UNSUPPORTED, "no cluster of four CTA pairs fits on this device");
     if (path == PATCH_PATH_GEMV && M > kDecodeBN)
         return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
     const int kernel = choose_kernel(g, path);
-    const int bn = kernel == 0 ? kGemmBN : kernel == 2 ? kDecodeBN : kGemm2BN;
+    const int bn = kernel_bn(kernel);
     const int mb = kernel == 2 ? 0 : (int)((M + bn - 1) / bn);
-    const int box_rows = kernel == 1 ? kGemm2BN / 2 : kernel == 3 ? kGemm2BN / 4 : bn;
+    const int box_rows = kernel_box_rows(kernel);
     GroupMaps maps;
     GroupArgs a;
     memset(&maps, 0, sizeof(maps));
@@ -518,8 +535,8 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
     a.MB = mb;
     a.status = g->status_dev;
     cudaError_t e = kernel == 0   ? launch_gemm(maps, a, grid, st)
-                    : kernel == 1 ? launch_gemm2(maps, a, grid, 2, st)
-                    : kernel == 3 ? launch_gemm2(maps, a, grid, 4, st)
+                    : kernel == 1 ? launch_gemm2(maps, a, grid, st)
+                    : kernel == 4 ? launch_gemm22(maps, a, grid, st)
                                   : launch_decode(maps, a, grid, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return PATCH_OK;
@@ -695,7 +712,7 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
                                void* stream) {
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_QUAD) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     patch_status st = check_xy(X_bf16, Y_bf16);
     if (st != PATCH_OK) return st;
@@ -768,7 +785,7 @@ patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, 
     if (!g) return fail(PATCH_ERR_ARG, "group is NULL");
     if (!X || !Y) return fail(PATCH_ERR_ARG, "X and Y arrays must be non-NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_QUAD) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     for (int l = 0; l < g->n; ++l) {
         patch_status st = check_xy(X[l], Y[l]);
@@ -887,13 +904,10 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     if (M <= 8) return run_simt(h, X_bf16, M, Y_bf16, st);
     const int path = resolve_path(PATCH_PATH_GEMM, M);
     const int kernel = choose_kernel(h->self, path);
-    const bool pair = kernel != 0;
-    const int bn = pair ? kGemm2BN : kGemmBN;
+    const int bn = kernel_bn(kernel);
     const int64_t mb = (M + bn - 1) / bn;
-    const int64_t rows = kernel == 0   ? (int64_t)h->plan.strip_cost.size()
-                         : kernel == 1 ? (int64_t)h->plan.pair_cost.size()
-                                       : (int64_t)(h->plan.pair_cost.size() + 1) / 2;
-    const int slots = kernel == 0 ? h->dev.sms : kernel == 1 ? h->dev.pair_clusters : h->dev.quad_clusters;
+    const int64_t rows = kernel_rows(h->plan, kernel);
+    const int slots = kernel_slots(h->dev, kernel);
     if (rows * mb > kNoAllocMaxUnits || slots > kNoAllocMaxSlots)
         return fail(PATCH_ERR_SHAPE,
                     "patch_linear_noalloc handles at most %d output tiles per call (this call needs %lld); "

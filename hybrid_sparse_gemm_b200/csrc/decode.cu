@@ -100,23 +100,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 part_range(L, p, b0, b1);
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
                 const uint32_t* mrow = L.meta + (size_t)s * L.KC;
-                const uint8_t* packed = L.packed;
                 const CUtensorMap* tmap_x = &maps.x[l];
+                uint32_t d_next = b0 < b1 ? trow[b0] : 0u;
                 for (int b = b0; b < b1; ++b) {
+                    const uint32_t d = d_next;
+                    if (b + 1 < b1) d_next = trow[b + 1];  // fetched one slab ahead
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    const uint32_t d = trow[b];
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
                     const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
                     uint8_t* st = smem + stage * kStageBytes;
                     mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + kStageX);
-                    bulk_load(st, packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    // the packed bytes viewed as 128-byte rows: one 2-D box per record
+                    tma_load_2d(st, sp ? &maps.a8[l] : &maps.a16[l], &full[stage], 0, (int)(slab_offset_bytes(d) >> 7));
                     if (first)
-                        bulk_load(st + kSparseValBytes, packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes,
-                                  &full[stage]);
+                        tma_load_2d(st + kSparseValBytes, &maps.e[l], &full[stage], 0, (int)(mrow[b >> 1] >> 3));
                     tma_load_2d(st + kStageA, tmap_x, &full[stage], b * kSlabK, 0);
                     ++issued;
                     if (++stage == kStages) {
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, any_mma = false;
+            bool ready = false;  // full[stage] already seen complete by the look-ahead
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
@@ -161,14 +163,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+                uint32_t d = b0 < b1 ? trow[b0] : 0u;
                 for (int b = b0; b < b1; ++b) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                    // the record comes one slab ahead and the next stage is
+                    // tested before this slab's MMAs (see the pair kernel)
+                    if (!ready && !mbar_wait(&full[stage], phase, abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t d = trow[b];
+                    const uint32_t d_next = b + 1 < b1 ? trow[b + 1] : 0u;
+                    int next = stage + 1;
+                    uint32_t next_phase = phase;
+                    if (next == kStages) {
+                        next = 0;
+                        next_phase ^= 1u;
+                    }
+                    ready = mbar_test_wait(&full[next], next_phase);
                     const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
                     const uint32_t x_addr = a_addr + kStageA;
                     const uint32_t first_mma = (b == b0) ? 0u : 1u;
@@ -194,10 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     any_mma = true;
                     tc_commit(&empty[stage]);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = next;
+                    phase = next_phase;
+                    d = d_next;
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[acc]);

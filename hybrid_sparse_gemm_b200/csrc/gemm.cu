@@ -111,23 +111,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = lu / a.MB, j = lu % a.MB;
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
                 const uint32_t* mrow = L.meta + (size_t)s * L.KC;
-                const uint8_t* packed = L.packed;
                 const CUtensorMap* tmap_x = &maps.x[l];
                 const int KB = L.KB;
+                uint32_t d_next = trow[0];
                 for (int b = 0; b < KB; ++b) {
+                    const uint32_t d = d_next;
+                    if (b + 1 < KB) d_next = trow[b + 1];  // fetched one slab ahead
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ab.raise();
                         ok = false;
                         break;
                     }
-                    const uint32_t d = trow[b];
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
                     const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
                     mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + C::kStageBBytes);
-                    bulk_load(sA + stage * kStageABytes, packed + slab_offset_bytes(d), bytes_a, &full[stage]);
+                    // the packed bytes viewed as 128-byte rows: one 2-D box per record
+                    tma_load_2d(sA + stage * kStageABytes, sp ? &maps.a8[l] : &maps.a16[l], &full[stage], 0,
+                                (int)(slab_offset_bytes(d) >> 7));
                     if (first)
-                        bulk_load(sA + stage * kStageABytes + kSparseValBytes,
-                                  packed + (uint64_t)mrow[b >> 1] * 16, kMetaBytes, &full[stage]);
+                        tma_load_2d(sA + stage * kStageABytes + kSparseValBytes, &maps.e[l], &full[stage], 0,
+                                    (int)(mrow[b >> 1] >> 3));
                     tma_load_2d(sB + stage * C::kStageBBytes, tmap_x, &full[stage], b * kSlabK, j * BN);
                     ++issued;
                     if (++stage == C::kStages) {
@@ -161,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             bool any_mma = false;
+            bool ready = false;  // full[stage] already seen complete by the look-ahead
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
@@ -174,14 +178,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                uint32_t d = trow[0];
                 for (int b = 0; b < KB; ++b) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                    // the record comes one slab ahead and the next stage is
+                    // tested before this slab's MMAs (see the pair kernel)
+                    if (!ready && !mbar_wait(&full[stage], phase, abort_flag)) {
                         ab.raise();
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t d = trow[b];
+                    const uint32_t d_next = b + 1 < KB ? trow[b + 1] : 0u;
+                    int next = stage + 1;
+                    uint32_t next_phase = phase;
+                    if (next == C::kStages) {
+                        next = 0;
+                        next_phase ^= 1u;
+                    }
+                    ready = mbar_test_wait(&full[next], next_phase);
                     const uint32_t a_addr = smem_u32(sA + stage * kStageABytes);
                     const uint32_t b_addr = smem_u32(sB + stage * C::kStageBBytes);
                     if (d & kSlabSparse) {
@@ -206,10 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     any_mma = true;
                     tc_commit(&empty[stage]);
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = next;
+                    phase = next_phase;
+                    d = d_next;
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[acc]);

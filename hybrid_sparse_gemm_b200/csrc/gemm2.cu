@@ -7,14 +7,8 @@
 // the 128 weight rows of one strip (operand A) and tokens [128r, 128r+128) of
 // the block (operand B); each MMA multiplies both A halves by both B halves,
 // so an SM loads half the activations it would need alone. The pair's leader
-// (even rank) issues every MMA; both CTAs' TMA loads complete on the leader's
+// (rank 0) issues every MMA; both CTAs' TMA loads complete on the leader's
 // barriers, and the leader's commits arrive on the CTAs' barriers.
-//
-// With CL = 4 two pairs (four strips) share a cluster and a token block: each
-// activation sub-tile is loaded once and multicast to the CTA of each pair
-// that needs it, halving the activation bytes each SM pulls from L2. The two
-// pairs then advance through the shared stages together (a stage is free
-// when both pairs' MMAs have consumed it).
 //
 // TMEM: each CTA holds its 128 rows x 256 tokens in one of two 256-column
 // accumulators. The 2:4 metadata of the running tile lives in the last four
@@ -27,14 +21,21 @@
 // last strip, a last cluster with fewer strips) are replaced by duplicates
 // whose results are not stored.
 #include "kernels.cuh"
+#include "pair.cuh"
 
 namespace patch {
 
 namespace {
 
-constexpr int kThreads = 192;
+#ifndef PATCH_GEMM2_PRODUCERS
+#define PATCH_GEMM2_PRODUCERS 2
+#endif
+constexpr int kProducers = PATCH_GEMM2_PRODUCERS;  // TMA-issuing warps per CTA (slabs dealt round robin)
+constexpr int kMmaWarp = kProducers;              // MMA issuer (pair leader) and TMEM owner
+constexpr int kThreads = 32 * (kProducers + 1 + 4);
 constexpr int kHalf = 128;                    // tokens per CTA
 constexpr int kStages = 6;
+static_assert(kStages % 2 == 0 && kStages % kProducers == 0, "stages come in pairs dealt round robin");
 constexpr int kStageA = 18432;                // 16 KB dense, or 8 KB values + 2 KB metadata
 constexpr int kStageB = kHalf * 128;          // 16 KB
 constexpr int kSmemData = kStages * (kStageA + kStageB);
@@ -42,125 +43,31 @@ constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kETail = kAccCols - 4;          // metadata columns inside the idle accumulator
-constexpr uint32_t kPeerMask = 0xFEFFFFFFu;   // clears the CTA-in-pair bit of a shared address
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Address of the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// 2-D TMA load whose completion is counted on the pair leader's barrier.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
-                                                 int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1)
-        : "memory");
-}
-// The same load written to the same offset in every CTA of `mask`; each
-// destination's bytes complete on its own pair leader's barrier.
-__device__ __forceinline__ void tma_load_2d_pair_mc(uint32_t dst, const CUtensorMap* map, uint32_t bar_local,
-                                                    int c0, int c1, uint16_t mask) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.multicast::cluster"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-        "l"(map), "r"(bar_local & kPeerMask), "r"(c0), "r"(c1), "h"(mask)
-        : "memory");
-}
-__device__ __forceinline__ void mma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma2_sp_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t e_tmem, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
-        : "memory");
-}
-__device__ __forceinline__ void cp2_128x128b(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-// Commit of the leader's MMAs, arriving on the barrier at this offset in every
-// CTA of `mask`.
-__device__ __forceinline__ void commit2_mask(uint64_t* bar, uint16_t mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"(mask)
-        : "memory");
-}
-__device__ __forceinline__ void commit2_local(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish2() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-template <int CL>
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_gemm2_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
-    constexpr int kStrips = CL;            // strips per cluster (one per CTA)
-    constexpr int kPairs = CL / 2;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + kStages * kStageA;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
-    uint64_t* full = bars;                    // pair leader: both CTAs' bytes of a stage
-    uint64_t* empty = bars + kStages;         // every CTA: stage consumed by every pair's MMAs
-    uint64_t* acc_full = bars + 2 * kStages;  // both CTAs of a pair: accumulator ready
-    uint64_t* acc_empty = acc_full + 2;       // pair leader: 8 epilogue warps drained it
-    uint64_t* e_free = acc_full + 4;          // pair leader: 8 epilogue warps read its tail
+    uint64_t* full = bars;                       // pair leader: both CTAs' bytes of a stage
+    uint64_t* empty = bars + kStages;            // both CTAs: a stage pair consumed by the MMAs
+    uint64_t* acc_full = empty + kStages / 2;    // both CTAs of a pair: accumulator ready
+    uint64_t* acc_empty = acc_full + 2;          // pair leader: 8 epilogue warps drained it
+    uint64_t* e_free = acc_full + 4;             // pair leader: 8 epilogue warps read its tail
     uint64_t* drain = acc_full + 6;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    const uint32_t pr = rank & 1u;          // CTA within its pair
-    const uint32_t pair = rank >> 1;        // pair within the cluster
-    const uint32_t leader = rank & ~1u;
-    const uint16_t pair_mask = (uint16_t)(3u << leader);
-    const uint16_t all_mask = (uint16_t)((1u << CL) - 1u);
-    const int cl = blockIdx.x / CL;
+    const uint32_t pr = cluster_rank();     // CTA within the pair (0 = leader)
+    const int cl = blockIdx.x >> 1;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kPairs);
-        }
+        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < kStages / 2; ++i) mbar_init(&empty[i], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 8);
@@ -170,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc2(tmem_slot, kTmemCols);
         tmem_relinquish2();
     }
@@ -183,23 +90,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         atomicCAS(a.status, 0, kStatusTimeout);
     };
-    // strip this CTA loads for cluster-unit c of a member with S strips
+    // strip this CTA loads for pair-unit c of a member with S strips (an odd
+    // last strip is duplicated into the second CTA and not stored)
     auto own_strip = [&](int c, int S) {
-        int s = kStrips * c + (int)rank;
-        if (s >= S) s = kStrips * c + (int)pr;
-        if (s >= S) s = kStrips * c;
+        int s = 2 * c + (int)pr;
+        if (s >= S) s = 2 * c;
         return s;
     };
 
     const int w_begin = a.work_off[cl];
     const int w_end = a.work_off[cl + 1];
 
-    if (warp == 0) {
+    if (warp < kProducers) {
         if (lane == 0) {
-            // ---------------- producer (every CTA) ----------------
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued = 0;
+            // ---------------- producers (every CTA) ----------------
+            // Slab g of this CTA's sequence goes to stage g % kStages and is
+            // loaded by producer g % kProducers; a stage pair (2q, 2q+1) is
+            // released by one commit after the MMAs of its second slab.
+            const int me = warp;
+            int g0 = 0;           // sequence index of the current unit's first slab
+            int my_last = -1;     // sequence index of the last slab this producer loaded
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
@@ -214,74 +124,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const CUtensorMap* tm_a16 = &maps.a16[l];
                 const CUtensorMap* tm_a8 = &maps.a8[l];
                 const CUtensorMap* tm_e = &maps.e[l];
-                for (int b = 0; b < KB; ++b) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                const int tok = j * kGemm2BN + (int)pr * kHalf;
+                // slab b of this unit is slab g0 + b of the CTA's sequence
+                int b = ((me - g0) % kProducers + kProducers) % kProducers;
+                uint32_t d_next = b < KB ? trow[b] : 0u;
+                for (; b < KB; b += kProducers) {
+                    const uint32_t d = d_next;
+                    if (b + kProducers < KB) d_next = trow[b + kProducers];  // fetched one slab ahead
+                    const int g = g0 + b;
+                    const int q = g >> 1;
+                    if (!mbar_wait(&empty[q % (kStages / 2)], ((q / (kStages / 2)) & 1) ^ 1u, abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    const uint32_t d = trow[b];
+                    const int stage = g % kStages;
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
-                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), leader);
+                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
                     if (pr == 0)
                         mbar_arrive_expect_tx(&full[stage],
                                               2u * ((sp ? kSparseValBytes : kDenseSlabBytes) +
                                                     (first ? kMetaBytes : 0) + kStageB));
                     const uint32_t dst_a = smem_u32(sA + stage * kStageA);
-                    const int row = (int)(slab_offset_bytes(d) >> 7);
-                    tma_load_2d_pair(dst_a, sp ? tm_a8 : tm_a16, bar, 0, row);
+                    tma_load_2d_pair(dst_a, sp ? tm_a8 : tm_a16, bar, 0, (int)(slab_offset_bytes(d) >> 7));
                     if (first)
                         tma_load_2d_pair(dst_a + kSparseValBytes, tm_e, bar, 0, (int)(mrow[b >> 1] >> 3));
-                    const int tok = j * kGemm2BN + (int)pr * kHalf;
-                    if (CL == 2) {
-                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), tm_x, bar, b * kSlabK, tok);
-                    } else {
-                        // this CTA fetches half of its 128 activation rows and
-                        // multicasts them to the same CTA of the other pair
-                        const uint32_t off = pair * (kStageB / 2);
-                        tma_load_2d_pair_mc(smem_u32(sB + stage * kStageB) + off, tm_x, smem_u32(&full[stage]),
-                                            b * kSlabK, tok + (int)pair * (kHalf / 2),
-                                            (uint16_t)((1u << pr) | (1u << (pr + 2))));
-                    }
-                    ++issued;
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), tm_x, bar, b * kSlabK, tok);
+                    my_last = g;
                 }
+                g0 += KB;
             }
             if (pr == 0) {
-                // Bounded wait for the loads of the last stages, whatever the
+                // Bounded wait for the loads of my last stages, whatever the
                 // abort flag says, so none lands after the cluster exits.
-                int st = stage;
-                uint32_t ph = phase;
-                for (int i = 0; i < kStages && i < issued; ++i) {
-                    if (--st < 0) {
-                        st = kStages - 1;
-                        ph ^= 1u;
-                    }
+                for (int g = my_last - kStages + 1; g <= my_last; ++g) {
+                    if (g < 0 || g % kProducers != me) continue;
                     const uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait(&full[st], ph) && globaltimer() - t0 < kWaitLimitNs) {
+                    while (!mbar_try_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1)) &&
+                           globaltimer() - t0 < kWaitLimitNs) {
                     }
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         if (lane == 0 && pr == 0) {
             // ---------------- MMA issuer (pair leader) ----------------
             const uint32_t idesc_d = idesc_bf16(256, kGemm2BN, false);
             const uint32_t idesc_s = idesc_bf16(256, kGemm2BN, true);
             int stage = 0;
             uint32_t phase = 0;
+            int g = 0;
             bool ok = true, any_mma = false;
+            bool ready = false;  // full[stage] already seen complete by the look-ahead
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
-                const int l = u >> kUnitShift, lu = u & kUnitMask;
-                const LinDesc& L = a.lins[l];
-                const int c = lu / a.MB;
-                const uint32_t* trow = L.gemm + (size_t)own_strip(c, L.S) * L.KB;
+                const LinDesc& L = a.lins[u >> kUnitShift];
                 const int KB = L.KB;
+                const uint32_t* trow = L.gemm + (size_t)own_strip((u & kUnitMask) / a.MB, L.S) * KB;
+                uint32_t d = trow[0];
                 const int acc = t & 1;
                 if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
                     raise();
@@ -291,14 +192,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
                 const uint32_t e_base = tmem_base + (uint32_t)((1 - acc) * kAccCols + kETail);
                 bool e_ready = (t == 0);
-                for (int b = 0; b < KB; ++b) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                for (int b = 0; b < KB; ++b, ++g) {
+                    // Nothing that depends on this slab's data sits between the
+                    // wait and the MMAs: the record was fetched one slab ahead,
+                    // and the next stage is tested (without blocking) before
+                    // this slab's MMAs so that its wait is usually free.
+                    if (!ready && !mbar_wait(&full[stage], phase, abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t d = trow[b];
+                    const uint32_t d_next = b + 1 < KB ? trow[b + 1] : 0u;
+                    int next = stage + 1;
+                    uint32_t next_phase = phase;
+                    if (next == kStages) {
+                        next = 0;
+                        next_phase ^= 1u;
+                    }
+                    ready = mbar_test_wait(&full[next], next_phase);
                     const uint32_t a_addr = smem_u32(sA + stage * kStageA);
                     const uint32_t b_addr = smem_u32(sB + stage * kStageB);
                     if (d & kSlabSparse) {
@@ -330,14 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     any_mma = true;
-                    commit2_mask(&empty[stage], all_mask);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (g & 1) commit2_mask(&empty[(g >> 1) % (kStages / 2)], 3);
+                    stage = next;
+                    phase = next_phase;
+                    d = d_next;
                 }
                 if (!ok) break;
-                commit2_mask(&acc_full[acc], pair_mask);
+                commit2_mask(&acc_full[acc], 3);
             }
             if (*abort_flag && any_mma) {
                 commit2_local(drain);
@@ -347,15 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5, every CTA) ----------------
-        const int q = warp & 3;
+        // ---------------- epilogue (4 warps, every CTA) ----------------
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const int N = a.lins[l].N;
             const int c = lu / a.MB, j = lu % a.MB;
-            const int s = kStrips * c + (int)rank;
+            const int s = 2 * c + (int)pr;
             const bool store = s < a.lins[l].S;
             const int acc = t & 1;
             if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
@@ -375,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // The tail (metadata columns of the next tile) is read: release it.
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) remote_arrive(map_to_rank(smem_u32(&e_free[acc]), leader));
+                    if (lane == 0) remote_arrive(map_to_rank(smem_u32(&e_free[acc]), 0));
                 }
                 if (!store) continue;
                 const int m0 = j * kGemm2BN + c0;
@@ -392,69 +302,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[acc]), leader));
+            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[acc]), 0));
         }
     }
 
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // no CTA leaves while another may still signal it
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc2(tmem_base, kTmemCols);
     }
 }
 
-template <int CL>
-cudaError_t prepare(int* max_clusters) {
-    cudaError_t e =
-        cudaFuncSetAttribute(hybrid_gemm2_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
+cudaLaunchConfig_t config(int clusters, cudaLaunchAttribute* attr, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL, 1, 1);
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = CL;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
+    cfg.stream = st;
+    attr->id = cudaLaunchAttributeClusterDimension;
+    attr->val.clusterDim.x = 2;
+    attr->val.clusterDim.y = 1;
+    attr->val.clusterDim.z = 1;
+    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cfg;
+}
+
+}  // namespace
+
+cudaError_t gemm_prepare_pair(int* max_clusters) {
+    cudaError_t e =
+        cudaFuncSetAttribute(hybrid_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr;
+    cudaLaunchConfig_t cfg = config(1, &attr, nullptr);
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm2_kernel<CL>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm2_kernel, &cfg);
     if (e != cudaSuccess) return e;
     *max_clusters = n;
     return cudaSuccess;
 }
 
-template <int CL>
-cudaError_t launch(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL * clusters, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = st;
+cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
     cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = CL;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, hybrid_gemm2_kernel<CL>, maps, a);
-}
-
-}  // namespace
-
-cudaError_t gemm_prepare_pair(int* max_pair_clusters, int* max_quad_clusters) {
-    cudaError_t e = prepare<2>(max_pair_clusters);
-    if (e != cudaSuccess) return e;
-    return prepare<4>(max_quad_clusters);
-}
-
-cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, int cluster_ctas, cudaStream_t st) {
-    return cluster_ctas == 4 ? launch<4>(maps, a, clusters, st) : launch<2>(maps, a, clusters, st);
+    cudaLaunchConfig_t cfg = config(clusters, &attr, st);
+    return cudaLaunchKernelEx(&cfg, hybrid_gemm2_kernel, maps, a);
 }
 
 }  // namespace patch

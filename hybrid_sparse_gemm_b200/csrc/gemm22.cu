@@ -1,0 +1,356 @@
+// Hybrid dense / 2:4 GEMM on CTA pairs with two strips per CTA:
+// Y = X . (W (.) Mask)^T.
+//
+// Same method as the other tensor-core kernels (dense slabs on tcgen05.mma,
+// 2:4 slabs on tcgen05.mma.sp; PATCH abstract, "PATCH: Learnable Tile-level
+// Hybrid Sparsity for LLMs"), arranged so that each activation tile feeds twice
+// the tensor work. A cluster of two CTAs owns a strip quad (strips 4c .. 4c+3)
+// and a block of 240 tokens. Every 64-column slab issues two 256-row MMAs
+// (cta_group::2), one per strip pair: strips (4c, 4c+1) into accumulator 0 and
+// (4c+2, 4c+3) into accumulator 1. CTA r holds strips 4c+r and 4c+2+r
+// (operand A) and tokens [r*N/2, (r+1)*N/2) of the block (operand B), so each
+// activation byte loaded from L2 serves 512 weight rows, and each slab's
+// barrier wait and commit are spread over 8 dense or 4 sparse MMAs.
+//
+// TMEM (512 columns per CTA): accumulator 0 in columns [0, 240), accumulator
+// 1 in [256, 496), the 2:4 metadata of each strip in four columns at 240 and
+// 248. The accumulators are single-buffered: a tile's MMAs start once the
+// previous tile has been drained, while the producers keep filling stages.
+//
+// Partner strips (2p, 2p+1) load the same kind of record at every slab (the
+// packed format's dense images stand in for 2:4 slabs whose partner is
+// dense), so one MMA instruction always covers both halves of a pair. Strips
+// past the end of the weight are replaced by duplicates whose results are not
+// stored.
+#include "kernels.cuh"
+#include "pair.cuh"
+
+namespace patch {
+
+namespace {
+
+constexpr int kProducers = 2;                   // TMA-issuing warps (slabs dealt round robin)
+constexpr int kMmaWarp = kProducers;            // MMA issuer (leader CTA) and TMEM owner
+constexpr int kEpiWarp0 = kProducers + 1;
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter, one per accumulator
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr int kBN = kGemm22BN;                  // tokens per tile (both CTAs)
+constexpr int kHalfN = kBN / 2;                 // token rows of operand B per CTA
+constexpr int kStages = 4;
+constexpr int kStageA = 18432;                  // 16 KB dense, or 8 KB values + 2 KB metadata
+constexpr int kStageB = kHalfN * 128;           // 15 KB
+constexpr int kStageBytes = 2 * kStageA + kStageB;
+static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle atoms)");
+static_assert(kStages % 2 == 0 && kStages % kProducers == 0, "stages come in pairs dealt round robin");
+constexpr int kSmemData = kStages * kStageBytes;
+constexpr int kSmemBytes = kSmemData + 1024 + 256;
+constexpr int kAcc1 = 256;                      // first column of accumulator 1
+constexpr int kECol0 = kBN;                     // metadata columns of strip pair 0
+constexpr int kECol1 = kBN + 8;                 // ... and of strip pair 1
+constexpr int kTmemCols = 512;
+static_assert(kECol1 + 4 <= kAcc1, "metadata columns fit between the accumulators");
+
+// Tokens of tile j (a multiple of 16: the MMA's N), at most kBN.
+__device__ __forceinline__ int tile_tokens(int j, int M) {
+    const int rem = M - j * kBN;
+    return rem >= kBN ? kBN : ((rem + 15) & ~15);
+}
+
+// Record bytes of one slab (values or dense image, plus metadata at the first
+// 2:4 slab of a chunk).
+__device__ __forceinline__ uint32_t record_bytes(uint32_t d) {
+    return ((d & kSlabSparse) ? kSparseValBytes : kDenseSlabBytes) + ((d & kSlabFirst) ? kMetaBytes : 0);
+}
+
+// One strip pair's MMAs for one slab: 4 dense K=16 MMAs, or the metadata copy
+// (first 2:4 slab of a chunk) and 2 sparse K=32 MMAs.
+__device__ __forceinline__ void issue_slab(uint32_t d, int b, uint32_t a_addr, uint32_t b_addr, uint32_t d_tmem,
+                                           uint32_t e_col, uint32_t idesc_d, uint32_t idesc_s) {
+    if (d & kSlabSparse) {
+        if (d & kSlabFirst) cp2_128x128b(e_col, smem_desc(a_addr + kSparseValBytes, 16, 128, kLayoutNone));
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 512, kLayoutSw64);
+            const uint64_t bd = smem_desc(b_addr + i * 64, 16, 1024, kLayoutSw128);
+            const uint32_t ecol = e_col + (uint32_t)((b & 1) * 2 + i);
+            mma2_sp_bf16(d_tmem, ad, bd, idesc_s | (ecol & 1u), ecol & ~1u, (b | i) != 0);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint64_t ad = smem_desc(a_addr + i * 32, 16, 1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(b_addr + i * 32, 16, 1024, kLayoutSw128);
+            mma2_bf16(d_tmem, ad, bd, idesc_d, (b | i) != 0);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hybrid_gemm22_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
+    uint64_t* full = bars;                       // leader: both CTAs' bytes of a stage
+    uint64_t* empty = full + kStages;            // every CTA: a stage pair consumed by the MMAs
+    uint64_t* acc_full = empty + kStages / 2;    // both CTAs: accumulators ready
+    uint64_t* acc_empty = acc_full + 1;          // leader: all epilogue warps of both CTAs drained them
+    uint64_t* drain = acc_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t pr = cluster_rank();          // CTA within the pair (0 = leader)
+    const int cl = blockIdx.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < kStages / 2; ++i) mbar_init(&empty[i], 1);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * kEpiWarps);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc2(tmem_slot, kTmemCols);
+        tmem_relinquish2();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    auto raise = [&]() {
+        *abort_flag = 1;
+        atomicCAS(a.status, 0, kStatusTimeout);
+    };
+    // Strip this CTA loads for strip pair h of quad c (S strips in the
+    // member); missing strips fall back to a strip whose partner relation is
+    // kept, so both halves of every MMA stay one kind.
+    auto strip_of = [&](int c, int h, int S) {
+        int s = 4 * c + 2 * h + (int)pr;
+        if (s >= S) s = 4 * c + 2 * h;
+        if (s >= S) s = 4 * c + (int)pr;
+        if (s >= S) s = 4 * c;
+        return s;
+    };
+
+    const int w_begin = a.work_off[cl];
+    const int w_end = a.work_off[cl + 1];
+
+    if (warp < kProducers) {
+        if (lane == 0) {
+            // ---------------- producers (both CTAs) ----------------
+            const int me = warp;
+            int g0 = 0;         // sequence index of the current unit's first slab
+            int my_last = -1;   // sequence index of the last slab this producer loaded
+            bool ok = true;
+            for (int it = w_begin; it < w_end && ok; ++it) {
+                const int u = a.work[it];
+                const int l = u >> kUnitShift, lu = u & kUnitMask;
+                const LinDesc& L = a.lins[l];
+                const int c = lu / a.MB, j = lu % a.MB;
+                const int KB = L.KB;
+                const int s0 = strip_of(c, 0, L.S), s1 = strip_of(c, 1, L.S);
+                const uint32_t* t0 = L.gemm + (size_t)s0 * KB;
+                const uint32_t* t1 = L.gemm + (size_t)s1 * KB;
+                const uint32_t* m0 = L.meta + (size_t)s0 * L.KC;
+                const uint32_t* m1 = L.meta + (size_t)s1 * L.KC;
+                const CUtensorMap* tm_x = &maps.x[l];
+                const CUtensorMap* tm_a16 = &maps.a16[l];
+                const CUtensorMap* tm_a8 = &maps.a8[l];
+                const CUtensorMap* tm_e = &maps.e[l];
+                const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
+                for (int b = ((me - g0) % kProducers + kProducers) % kProducers; b < KB; b += kProducers) {
+                    const int g = g0 + b;
+                    const int q = g >> 1;
+                    if (!mbar_wait(&empty[q % (kStages / 2)], ((q / (kStages / 2)) & 1) ^ 1u, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    const int stage = g % kStages;
+                    const uint32_t d0 = t0[b], d1 = t1[b];
+                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
+                    if (pr == 0) mbar_arrive_expect_tx(&full[stage], 2u * (record_bytes(d0) + record_bytes(d1) + kStageB));
+                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
+                    tma_load_2d_pair(base, (d0 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0, (int)(slab_offset_bytes(d0) >> 7));
+                    if (d0 & kSlabFirst)
+                        tma_load_2d_pair(base + kSparseValBytes, tm_e, bar, 0, (int)(m0[b >> 1] >> 3));
+                    tma_load_2d_pair(base + kStageA, (d1 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0,
+                                     (int)(slab_offset_bytes(d1) >> 7));
+                    if (d1 & kSlabFirst)
+                        tma_load_2d_pair(base + kStageA + kSparseValBytes, tm_e, bar, 0, (int)(m1[b >> 1] >> 3));
+                    tma_load_2d_pair(base + 2 * kStageA, tm_x, bar, b * kSlabK, tok);
+                    my_last = g;
+                }
+                g0 += KB;
+            }
+            if (pr == 0) {
+                // Bounded wait for the loads of my last stages, whatever the
+                // abort flag says, so none lands after the cluster exits.
+                for (int g = my_last - kStages + 1; g <= my_last; ++g) {
+                    if (g < 0 || g % kProducers != me) continue;
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1)) &&
+                           globaltimer() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && pr == 0) {
+            // ---------------- MMA issuer (leader CTA) ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            int g = 0;
+            bool ok = true, any_mma = false;
+            bool ready = false;  // full[stage] already seen complete by the look-ahead
+            int t = 0;
+            for (int it = w_begin; it < w_end && ok; ++it, ++t) {
+                const int u = a.work[it];
+                const LinDesc& L = a.lins[u >> kUnitShift];
+                const int lu = u & kUnitMask;
+                const int c = lu / a.MB, j = lu % a.MB;
+                const int KB = L.KB;
+                const uint32_t* t0 = L.gemm + (size_t)strip_of(c, 0, L.S) * KB;
+                const uint32_t* t1 = L.gemm + (size_t)strip_of(c, 1, L.S) * KB;
+                const int nt = tile_tokens(j, a.M);
+                const uint32_t idesc_d = idesc_bf16(256, nt, false);
+                const uint32_t idesc_s = idesc_bf16(256, nt, true);
+                uint32_t d0 = t0[0], d1 = t1[0];
+                if (!mbar_wait(acc_empty, (t & 1) ^ 1u, abort_flag)) {
+                    raise();
+                    break;
+                }
+                tc_fence_after();
+                for (int b = 0; b < KB; ++b, ++g) {
+                    if (!ready && !mbar_wait(&full[stage], phase, abort_flag)) {
+                        raise();
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t d0n = b + 1 < KB ? t0[b + 1] : 0u;
+                    const uint32_t d1n = b + 1 < KB ? t1[b + 1] : 0u;
+                    int next = stage + 1;
+                    uint32_t next_phase = phase;
+                    if (next == kStages) {
+                        next = 0;
+                        next_phase ^= 1u;
+                    }
+                    ready = mbar_test_wait(&full[next], next_phase);
+                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t b_addr = base + 2 * kStageA;
+                    issue_slab(d0, b, base, b_addr, tmem_base, tmem_base + kECol0, idesc_d, idesc_s);
+                    issue_slab(d1, b, base + kStageA, b_addr, tmem_base + kAcc1, tmem_base + kECol1, idesc_d,
+                               idesc_s);
+                    any_mma = true;
+                    if (g & 1) commit2_mask(&empty[(g >> 1) % (kStages / 2)], 3);
+                    stage = next;
+                    phase = next_phase;
+                    d0 = d0n;
+                    d1 = d1n;
+                }
+                if (!ok) break;
+                commit2_mask(acc_full, 3);
+            }
+            if (*abort_flag && any_mma) {
+                commit2_local(drain);
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else {
+        // ---------------- epilogue (8 warps, both CTAs) ----------------
+        const int h = (warp - kEpiWarp0) >> 2;   // accumulator (strip pair) this warp drains
+        const int q = warp & 3;                  // TMEM lane quarter this warp may access
+        int t = 0;
+        for (int it = w_begin; it < w_end; ++it, ++t) {
+            const int u = a.work[it];
+            const int l = u >> kUnitShift, lu = u & kUnitMask;
+            const int N = a.lins[l].N;
+            const int c = lu / a.MB, j = lu % a.MB;
+            const int s = 4 * c + 2 * h + (int)pr;
+            const bool store = s < a.lins[l].S;
+            const int nt = tile_tokens(j, a.M);
+            if (!mbar_wait(acc_full, t & 1, abort_flag)) {
+                if (lane == 0) raise();
+                break;
+            }
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kAcc1);
+            __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + q * 32 + lane;
+            if (store) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < nt; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(taddr + c0, v);
+                    tc_wait_ld();
+                    const int m0 = j * kBN + c0;
+                    if (m0 + 16 <= a.M) {
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc)
+                            yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+                    } else {
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc)
+                            if (m0 + cc < a.M)
+                                yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) remote_arrive(map_to_rank(smem_u32(acc_empty), 0));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while the other may still signal it
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc2(tmem_base, kTmemCols);
+    }
+}
+
+cudaLaunchConfig_t config(int clusters, cudaLaunchAttribute* attr, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    attr->id = cudaLaunchAttributeClusterDimension;
+    attr->val.clusterDim.x = 2;
+    attr->val.clusterDim.y = 1;
+    attr->val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+}  // namespace
+
+cudaError_t gemm_prepare_wide(int* max_clusters) {
+    cudaError_t e =
+        cudaFuncSetAttribute(hybrid_gemm22_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr;
+    cudaLaunchConfig_t cfg = config(1, &attr, nullptr);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm22_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    *max_clusters = n;
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
+    cudaLaunchAttribute attr;
+    cudaLaunchConfig_t cfg = config(clusters, &attr, st);
+    return cudaLaunchKernelEx(&cfg, hybrid_gemm22_kernel, maps, a);
+}
+
+}  // namespace patch

@@ -71,15 +71,18 @@ struct GemvArgs {
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_gemm(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
-cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, int cluster_ctas, cudaStream_t st);
+cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
+cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
 cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 cudaError_t gemm_prepare_single();
-cudaError_t gemm_prepare_pair(int* max_pair_clusters, int* max_quad_clusters);
+cudaError_t gemm_prepare_pair(int* max_clusters);
+cudaError_t gemm_prepare_wide(int* max_clusters);
 cudaError_t decode_prepare();
 
 constexpr int kGemmBN = 128;   // tokens per CTA tile (single-CTA kernel)
 constexpr int kGemm2BN = 256;  // tokens per CTA-pair tile
+constexpr int kGemm22BN = 240; // tokens per tile of the two-strips-per-CTA pair kernel
 constexpr int kDecodeBN = 16;  // tokens per decode MMA (M <= 16)
 
 }  // namespace patch

@@ -61,9 +61,9 @@ typedef enum {
     PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
     PATCH_PATH_GEMM_PAIR = 4,    /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
     PATCH_PATH_GEMV_SIMT = 5,    /* decode on CUDA cores (M <= 16), no workspace */
-    PATCH_PATH_GEMM_QUAD = 6     /* as GEMM_PAIR, two pairs per cluster sharing each
-                                    activation tile through TMA multicast; strips are
-                                    padded to a multiple of four with duplicates */
+    PATCH_PATH_GEMM_WIDE = 6     /* tcgen05 cta_group::2, two strips per CTA: one CTA pair
+                                    per 512-row x 240-token tile (each activation tile feeds
+                                    both strip pairs); strips padded to a multiple of four */
 } patch_path;
 
 typedef struct {

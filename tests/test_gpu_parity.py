@@ -188,21 +188,32 @@ def test_decode_repeat_and_interleave(hsg, oracle_lib):
     lin.free()
 
 
-@pytest.mark.parametrize("N", [512, 1024, 3200])
-@pytest.mark.parametrize("M", [256, 300, 1000])
-@pytest.mark.parametrize("R,C,frac", [(128, 128, 0.9), (64, 64, 0.3), (128, 64, 1.0)])
-def test_pair_clusters_of_four(hsg, oracle_lib, N, M, R, C, frac):
-    """Strip counts that run two CTA pairs per cluster (shared activations),
-    including a last cluster with one real strip and three duplicates."""
-    p = synth.make_problem(N, 512, M, R=R, C=C, frac=frac, seed=N + M, device="cuda")
+@pytest.mark.parametrize("N", [128, 384, 512, 640, 1152])
+@pytest.mark.parametrize("M", [16, 100, 240, 241, 497, 1000])
+@pytest.mark.parametrize("R,C,frac", [(128, 128, 0.9), (64, 64, 0.3), (128, 64, 1.0), (64, 128, 0.0)])
+def test_wide_tiles(hsg, oracle_lib, N, M, R, C, frac):
+    """Two strips per CTA of a pair: strip counts that leave one, two or three
+    strips of the last quad as duplicates, token counts that end in a ragged
+    tile (a narrower MMA) or fill tiles exactly."""
+    p = synth.make_problem(N, 512, M, R=R, C=C, frac=frac, seed=3 * N + M, device="cuda", tag="wide")
     lin = pack(hsg, p)
-    Y = lin(p.X, path=hsg.PATH_GEMM_QUAD)
-    Y2 = lin(p.X, path=hsg.PATH_GEMM_QUAD)
-    Yp = lin(p.X, path=hsg.PATH_GEMM_PAIR)
+    Y = lin(p.X, path=hsg.PATH_GEMM_WIDE)
+    Y2 = lin(p.X, path=hsg.PATH_GEMM_WIDE)
     torch.cuda.synchronize()
     lin.check()
-    assert torch.equal(Y, Y2) and torch.equal(Y, Yp)
-    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(M, 96, N), what=f"quad N={N} M={M}")
+    assert torch.equal(Y, Y2)
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(M, 96, N), what=f"wide N={N} M={M}")
+    lin.free()
+
+
+def test_wide_long_k(hsg, oracle_lib):
+    """Many slabs per tile (K = 4096) and several tiles per CTA pair."""
+    p = synth.make_problem(1024, 4096, 2000, R=128, C=128, frac=0.7, seed=11, device="cuda", tag="widek")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMM_WIDE)
+    torch.cuda.synchronize()
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(2000, 48, 5), what="wide long K")
     lin.free()
 
 
@@ -360,7 +371,8 @@ def test_config5_llama2_13b_tiles(hsg, oracle_lib, R, C):
 # --------------------------------------------------------------- groups ---
 
 @pytest.mark.parametrize("path_name,M", [("GEMM_PAIR", 300), ("GEMM_SINGLE", 130), ("GEMV", 16), ("GEMV", 3),
-                                         ("GEMV_SIMT", 5), ("AUTO", 520), ("AUTO", 1)])
+                                         ("GEMV_SIMT", 5), ("AUTO", 520), ("AUTO", 1), ("GEMM_WIDE", 300),
+                                         ("GEMM_WIDE", 17)])
 def test_group_matches_members(hsg, oracle_lib, path_name, M):
     """One launch over several linears (shared and separate inputs, mixed tile
     shapes and 2:4 fractions) equals the members run one by one, bit for bit,
