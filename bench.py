@@ -46,6 +46,9 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 FRACS_SWEEP = [0.0, 0.5, 0.7, 0.9, 1.0]
+KERNEL_NAMES = {4: "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
+                6: "hybrid_gemm22_kernel (CTA pair, two strips per CTA, 512x240 tiles)",
+                3: "hybrid_gemm_kernel (single CTA, 128x128 tiles)"}
 
 
 def load_peaks():
@@ -194,6 +197,7 @@ def run_step(hsg, model, X, Y, stream, path=0, events=None):
 
 
 def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=False, path=0):
+    from hybrid_sparse_gemm_b200 import dist as hdist
     for _ in range(warmup):
         run_step(hsg, model, X, Y, stream, path)
     torch.cuda.synchronize()
@@ -345,6 +349,7 @@ def main():
         return
 
     import hybrid_sparse_gemm_b200 as hsg
+    from hybrid_sparse_gemm_b200 import dist as hdist
 
     torch.cuda.set_device(local_rank if world > 1 else 0)
     dist_on = hdist.init("nccl")
@@ -368,6 +373,8 @@ def main():
     # per-launch durations for the roofline (separate pass, events around each launch)
     _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True)
     kern_ms = statistics.mean(sum(row) for row in launch_ms)
+    kernel_name = KERNEL_NAMES.get(model[0][0].path(M) if model[0][0] is not None else hsg.PATH_GEMM_PAIR,
+                                   "tensor-core GEMM")
     achieved = exec_flops / (kern_ms / 1e3) / 1e12
     value = hdist.job_rate(F, world, ms_h) / 1e12
 
@@ -439,7 +446,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
                          "traffic": None,
-                         "kernel": "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
+                         "kernel": kernel_name,
                          "work": "2*M per kept weight of every loaded slab (a 2:4 slab counts half)",
                          "peak_kind": f"bf16 sustained ({peaks['source']})"},
             "gpu_launches": n_launch * args.steps,

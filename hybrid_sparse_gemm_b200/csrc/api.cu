@@ -450,10 +450,18 @@ patch_status check_device_is(int device) {
 }
 
 // Resolves AUTO / GEMM to a concrete kernel for this M.
-int resolve_path(int path, int64_t M) {
+// AUTO and GEMM pick by M; for large M the two-strips-per-CTA kernel is used
+// when the launch has enough strip quads to keep every CTA pair busy (it
+// feeds each activation tile to twice the weight rows, but a small weight
+// gives it half as many work units as the one-strip pair kernel).
+int resolve_path(patch_group g, int path, int64_t M) {
     if (path == PATCH_PATH_AUTO) path = (M <= kDecodeBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
-    if (path == PATCH_PATH_GEMM) path = (M >= kPairMinM) ? PATCH_PATH_GEMM_PAIR : PATCH_PATH_GEMM_SINGLE;
-    return path;
+    if (path != PATCH_PATH_GEMM) return path;
+    if (M < kPairMinM) return PATCH_PATH_GEMM_SINGLE;
+    int64_t quads = 0;
+    for (int l = 0; l < g->n; ++l) quads += (g->h[l]->plan.S + 3) / 4;
+    const int64_t units = quads * ((M + kGemm22BN - 1) / kGemm22BN);
+    return units >= 2 * (int64_t)g->dev.wide_clusters ? PATCH_PATH_GEMM_WIDE : PATCH_PATH_GEMM_PAIR;
 }
 
 patch_status run_simt(patch_handle h, const void* X, int64_t M, void* Y, cudaStream_t st) {
@@ -488,7 +496,7 @@ int choose_kernel(patch_group g, int path) {
 // caller-provided device memory; otherwise the group's cached schedule is used.
 patch_status run_group(patch_group g, const void* const* X, int64_t M, void* const* Y, int path, cudaStream_t st,
                        const int* sched_off = nullptr, const int* sched_work = nullptr, int sched_grid = 0) {
-    path = resolve_path(path, M);
+    path = resolve_path(g, path, M);
     if (path == PATCH_PATH_GEMV_SIMT) {
         for (int l = 0; l < g->n; ++l) {
             patch_status s = run_simt(g->h[l], X[l], M, Y[l], st);
@@ -796,6 +804,14 @@ patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, 
     return run_group(g, X, M, Y, path, static_cast<cudaStream_t>(stream));
 }
 
+patch_status patch_group_path(patch_group g, int64_t M, int path, int* out) {
+    if (!g || !out) return fail(PATCH_ERR_ARG, "group and out must be non-NULL");
+    if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    *out = resolve_path(g, path, M);
+    return PATCH_OK;
+}
+
 void patch_group_free(patch_group g) { free_group(g); }
 
 patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream) {
@@ -902,7 +918,7 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     if ((s = check_device_is(h->device)) != PATCH_OK) return s;
     // Decode sizes: the CUDA-core kernel needs no schedule and no scratch.
     if (M <= 8) return run_simt(h, X_bf16, M, Y_bf16, st);
-    const int path = resolve_path(PATCH_PATH_GEMM, M);
+    const int path = resolve_path(h->self, PATCH_PATH_GEMM, M);
     const int kernel = choose_kernel(h->self, path);
     const int bn = kernel_bn(kernel);
     const int64_t mb = (M + bn - 1) / bn;

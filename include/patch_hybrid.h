@@ -53,10 +53,13 @@ typedef enum {
     PATCH_ERR_UNSUPPORTED = 8  /* current device is not compute capability 10.x */
 } patch_status;
 
-/* Which kernel patch_linear_path runs. AUTO picks by M. */
+/* Which kernel patch_linear_path runs. AUTO picks by M: GEMV for M <= 16,
+ * GEMM_SINGLE below M = 256, and above it GEMM_WIDE when the call (or group)
+ * has at least two 512-row x 240-token tiles per co-resident CTA pair,
+ * otherwise GEMM_PAIR. GEMM is AUTO restricted to the tensor-core GEMMs. */
 typedef enum {
     PATCH_PATH_AUTO = 0,
-    PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core kernel, variant chosen by M */
+    PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core GEMM, variant chosen as for AUTO */
     PATCH_PATH_GEMV = 2,         /* decode kernel (M <= 16): tcgen05 N=16, split-K */
     PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
     PATCH_PATH_GEMM_PAIR = 4,    /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
@@ -207,6 +210,14 @@ patch_status patch_group_create(const patch_handle* handles, int n, patch_group*
  */
 patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, void* const* Y, int path,
                                 void* stream);
+
+/*
+ * patch_group_path - the explicit path (GEMV, GEMV_SIMT, GEMM_SINGLE,
+ * GEMM_PAIR or GEMM_WIDE) that patch_group_linear would run for this M and
+ * requested path; nothing is launched. *out receives the value.
+ * Errors: PATCH_ERR_ARG for a NULL group or out, M < 0 or an unknown path.
+ */
+patch_status patch_group_path(patch_group g, int64_t M, int path, int* out);
 
 /* patch_group_free - release a group (not its handles). NULL is ignored. */
 void patch_group_free(patch_group g);

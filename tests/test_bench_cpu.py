@@ -1,0 +1,29 @@
+"""bench.py's host-side pieces on the CPU: the module imports, the peak table
+loads, and the CPU baseline (the oracle on a bounded row sample) runs and
+reports a positive rate."""
+import importlib.util
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_bench_imports_and_peaks():
+    b = _bench()
+    peaks = b.load_peaks()
+    assert peaks["hbm_gbs"] > 0 and peaks["bf16_tflops"] > 0 and peaks["bf16_tflops_sustained"] > 0
+    assert peaks["source"] in ("measured", "fallback")
+    assert set(b.KERNEL_NAMES) >= {3, 4, 6}
+
+
+def test_cpu_baseline_sample():
+    b = _bench()
+    rate, threads, desc = b.cpu_sample(budget_s=0.2, min_rows=1)
+    assert rate > 0 and threads >= 1
+    assert "oracle" in desc and "token rows" in desc

@@ -411,6 +411,23 @@ def test_group_matches_members(hsg, oracle_lib, path_name, M):
         lin.free()
 
 
+def test_group_path_choice(hsg):
+    """AUTO resolves by M and by how many two-strip tiles the launch has."""
+    small = pack(hsg, synth.make_problem(512, 256, 0, seed=1, device="cuda", tag="gp1"))
+    big = pack(hsg, synth.make_problem(8192, 256, 0, seed=2, device="cuda", tag="gp2"))
+    gs, gb = hsg.LinearGroup([small]), hsg.LinearGroup([big])
+    assert gs.path(1) == hsg.PATH_GEMV and gs.path(16) == hsg.PATH_GEMV
+    assert gs.path(17) == hsg.PATH_GEMM_SINGLE and gs.path(255) == hsg.PATH_GEMM_SINGLE
+    assert gs.path(256) == hsg.PATH_GEMM_PAIR          # one strip quad: too few tiles
+    assert gb.path(4096) == hsg.PATH_GEMM_WIDE         # 16 quads x 18 token blocks
+    assert gb.path(4096, hsg.PATH_GEMM_PAIR) == hsg.PATH_GEMM_PAIR
+    assert gs.path(4, hsg.PATH_GEMV_SIMT) == hsg.PATH_GEMV_SIMT
+    for g in (gs, gb):
+        g.free()
+    small.free()
+    big.free()
+
+
 def test_group_argument_errors(hsg):
     import ctypes
     lib = hsg.library()
