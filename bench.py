@@ -238,12 +238,21 @@ def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
     shapes = synth.llama32_1b()
     probs = [synth.make_problem(l.N, l.K, 4096, R=128, C=128, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
              for l in shapes]
-    # calibrate on one row of every linear
-    t0 = time.perf_counter()
-    for p in probs:
-        oracle.linear(p.X[:1], p.W, p.bits.numpy())
-    t1 = time.perf_counter() - t0
-    rows = max(min_rows, min(4096, int(budget_s / max(t1, 1e-6))))
+    # calibrate: time 4 and 16 rows of every linear (after one untimed call
+    # that starts the thread pool) and fit time = fixed + rows * per_row; the
+    # fixed part (mask expansion over the whole weight) does not shrink with rows
+    oracle.linear(probs[0].X[:1], probs[0].W, probs[0].bits.numpy())
+
+    def one_pass(r):
+        t0 = time.perf_counter()
+        for p in probs:
+            oracle.linear(p.X[:r], p.W, p.bits.numpy())
+        return time.perf_counter() - t0
+
+    t4, t16 = one_pass(4), one_pass(16)
+    per_row = max((t16 - t4) / 12.0, 1e-6)
+    fixed = max(t4 - 4 * per_row, 0.0)
+    rows = max(min_rows, min(4096, int((budget_s - fixed) / per_row)))
     flops = 0.0
     t0 = time.perf_counter()
     for l, p in zip(shapes, probs):
@@ -316,6 +325,8 @@ def main():
     ap.add_argument("--layers", type=int, default=16)
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--no-group", action="store_true", help="one launch per linear instead of per layer")
+    ap.add_argument("--path", default="auto", choices=["auto", "pair", "wide"],
+                    help="tensor-core kernel for the timed steps (auto: the library's choice)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -355,6 +366,7 @@ def main():
     dist_on = hdist.init("nccl")
     stream = torch.cuda.Stream()
     peaks = load_peaks()
+    gpath = {"auto": hsg.PATH_AUTO, "pair": hsg.PATH_GEMM_PAIR, "wide": hsg.PATH_GEMM_WIDE}[args.path]
     M = args.M
     group = not args.no_group
 
@@ -367,13 +379,14 @@ def main():
     n_launch = len(model)
 
     with ClockSampler(torch.cuda.current_device()) as clk:
-        ms_h, _ = time_steps(hsg, model, X, None, args.steps, args.warmup, stream, dist_on)
+        ms_h, _ = time_steps(hsg, model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
     clocks = clk.summary()
-    ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on)
+    ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
     # per-launch durations for the roofline (separate pass, events around each launch)
-    _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True)
+    _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True,
+                              path=gpath)
     kern_ms = statistics.mean(sum(row) for row in launch_ms)
-    kernel_name = KERNEL_NAMES.get(model[0][0].path(M) if model[0][0] is not None else hsg.PATH_GEMM_PAIR,
+    kernel_name = KERNEL_NAMES.get(model[0][0].path(M, gpath) if model[0][0] is not None else hsg.PATH_GEMM_PAIR,
                                    "tensor-core GEMM")
     achieved = exec_flops / (kern_ms / 1e3) / 1e12
     value = hdist.job_rate(F, world, ms_h) / 1e12
@@ -389,7 +402,7 @@ def main():
             else:
                 with torch.cuda.stream(stream):
                     mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group)
-                t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on)
+                t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
                 free_model(mdl)
                 del mdl
             sweep[str(f)] = {"tflops": hdist.job_rate(F, world, t) / 1e12, "speedup_vs_dense": ms_d / t,
@@ -441,7 +454,7 @@ def main():
                        "launches_per_step": n_launch, "grouped": group,
                        "frac_2to4": frac_real, "tile": "128x128",
                        "l2": "inputs larger than L2 (%.2f GB of packed weights per step)" % packed_gb,
-                       "parallelism": f"dp{world} (M split, replicated weights)"},
+                       "parallelism": f"dp{world} (M split, replicated weights)", "path": args.path},
             "speedup_vs_dense": ms_d / ms_h, "dense_ms_per_step": ms_d,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],

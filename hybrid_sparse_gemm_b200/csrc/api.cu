@@ -318,7 +318,7 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     double total = 0.0;
     for (int i = 0; i < n; ++i)
         for (double b : hs[i]->plan.strip_bytes) total += b;
-    const double target = std::max(256.0 * 1024.0, total / (4.0 * g->dev.sms));
+    const double target = std::max(256.0 * 1024.0, total / (4.0 * kDecodeCtasPerSm * g->dev.sms));
     for (int i = 0; i < n; ++i) {
         g->h[i] = hs[i];
         d[i] = hs[i]->desc;
@@ -366,7 +366,7 @@ int64_t kernel_rows(const Plan& p, int kernel) {
     return kernel == 0 ? (int64_t)p.strip_cost.size() : kernel == 1 ? pairs : (pairs + 1) / 2;
 }
 int kernel_slots(const DeviceInfo& d, int kernel) {
-    return kernel == 1 ? d.pair_clusters : kernel == 4 ? d.wide_clusters : d.sms;
+    return kernel == 1 ? d.pair_clusters : kernel == 4 ? d.wide_clusters : kernel == 2 ? kDecodeCtasPerSm * d.sms : d.sms;
 }
 
 void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
@@ -618,7 +618,7 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     }
     int64_t tiles_sparse = 0;
     for (int64_t i = 0; i < ntiles; ++i) tiles_sparse += tile_flags[i];
-    h->decode_parts = choose_decode_parts(p.S, p.KC, di.sms);
+    h->decode_parts = choose_decode_parts(p.S, p.KC, kDecodeCtasPerSm * di.sms);
 
     uint8_t* flags_dev = nullptr;
     unsigned long long* counters = nullptr;

@@ -24,7 +24,7 @@ constexpr int kBN = kDecodeBN;           // tokens per MMA (M <= 16)
 constexpr int kStageA = 18432;           // 16 KB dense, or 8 KB values + 2 KB metadata
 constexpr int kStageX = kBN * 128;       // 2 KB, 128-byte swizzled
 constexpr int kStageBytes = kStageA + kStageX;
-constexpr int kStages = 8;
+constexpr int kStages = 5;                // two CTAs share an SM (kDecodeCtasPerSm)
 constexpr int kSmemData = kStages * kStageBytes;
 constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kECol = 2 * kBN;           // metadata columns after the two accumulators
@@ -33,7 +33,7 @@ constexpr int kTmemCols = 64;
 // Named barrier of one epilogue warpgroup (ids 1 and 2).
 __device__ __forceinline__ void epi_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
     hybrid_decode_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
