@@ -9,8 +9,9 @@
 // (cta_group::2), one per strip pair: strips (4c, 4c+1) into accumulator 0 and
 // (4c+2, 4c+3) into accumulator 1. CTA r holds strips 4c+r and 4c+2+r
 // (operand A) and tokens [r*N/2, (r+1)*N/2) of the block (operand B), so each
-// activation byte loaded from L2 serves 512 weight rows, and each slab's
-// barrier wait and commit are spread over 8 dense or 4 sparse MMAs.
+// activation byte loaded from L2 serves 512 weight rows. Each strip pair has
+// its own issuing thread, so the tensor pipe is fed by two instruction
+// streams (one thread alone cannot issue 2:4 slabs as fast as they execute).
 //
 // TMEM (512 columns per CTA): accumulator 0 in columns [0, 240), accumulator
 // 1 in [256, 496), the 2:4 metadata of each strip in four columns at 240 and
@@ -30,9 +31,10 @@ namespace patch {
 namespace {
 
 constexpr int kProducers = 2;                   // TMA-issuing warps (slabs dealt round robin)
-constexpr int kMmaWarp = kProducers;            // MMA issuer (leader CTA) and TMEM owner
-constexpr int kEpiWarp0 = kProducers + 1;
-constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter, one per accumulator
+constexpr int kMmaWarp = kProducers;            // MMA issuers (leader CTA), one per strip pair;
+constexpr int kMmaWarps = 2;                    // the first also owns TMEM
+constexpr int kEpiWarp0 = kMmaWarp + kMmaWarps;
+constexpr int kEpiWarps = 16;                   // per accumulator, two warps per TMEM lane quarter
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBN = kGemm22BN;                  // tokens per tile (both CTAs)
 constexpr int kHalfN = kBN / 2;                 // token rows of operand B per CTA
@@ -93,10 +95,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
     uint64_t* full = bars;                       // leader: both CTAs' bytes of a stage
     uint64_t* empty = full + kStages;            // every CTA: a stage pair consumed by the MMAs
-    uint64_t* acc_full = empty + kStages / 2;    // both CTAs: accumulators ready
-    uint64_t* acc_empty = acc_full + 1;          // leader: all epilogue warps of both CTAs drained them
-    uint64_t* drain = acc_empty + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* acc_full = empty + kStages / 2;    // [2] both CTAs: accumulator h ready
+    uint64_t* acc_empty = acc_full + 2;          // [2] leader: the 16 epilogue warps of accumulator h drained it
+    uint64_t* drain = acc_empty + 2;             // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -106,10 +108,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
-        for (int i = 0; i < kStages / 2; ++i) mbar_init(&empty[i], 1);
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 2 * kEpiWarps);
-        mbar_init(drain, 1);
+        for (int i = 0; i < kStages / 2; ++i) mbar_init(&empty[i], kMmaWarps);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&acc_full[h], 1);
+            mbar_init(&acc_empty[h], kEpiWarps);  // its 8 epilogue warps in each of the 2 CTAs
+            mbar_init(&drain[h], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -200,9 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp < kMmaWarp + kMmaWarps) {
         if (lane == 0 && pr == 0) {
-            // ---------------- MMA issuer (leader CTA) ----------------
+            // ---------------- MMA issuers (leader CTA), one per strip pair ----------------
+            // Both read every stage; a stage pair is free once both have
+            // committed it. Two issuing threads keep the tensor pipe fed while
+            // either one waits on a barrier or computes descriptors.
+            const int h = warp - kMmaWarp;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(h * kAcc1);
+            const uint32_t e_col = tmem_base + (uint32_t)(h ? kECol1 : kECol0);
             int stage = 0;
             uint32_t phase = 0;
             int g = 0;
@@ -215,13 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int lu = u & kUnitMask;
                 const int c = lu / a.MB, j = lu % a.MB;
                 const int KB = L.KB;
-                const uint32_t* t0 = L.gemm + (size_t)strip_of(c, 0, L.S) * KB;
-                const uint32_t* t1 = L.gemm + (size_t)strip_of(c, 1, L.S) * KB;
+                const uint32_t* trow = L.gemm + (size_t)strip_of(c, h, L.S) * KB;
                 const int nt = tile_tokens(j, a.M);
                 const uint32_t idesc_d = idesc_bf16(256, nt, false);
                 const uint32_t idesc_s = idesc_bf16(256, nt, true);
-                uint32_t d0 = t0[0], d1 = t1[0];
-                if (!mbar_wait(acc_empty, (t & 1) ^ 1u, abort_flag)) {
+                uint32_t d = trow[0];
+                if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
                     raise();
                     break;
                 }
@@ -232,8 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t d0n = b + 1 < KB ? t0[b + 1] : 0u;
-                    const uint32_t d1n = b + 1 < KB ? t1[b + 1] : 0u;
+                    const uint32_t d_next = b + 1 < KB ? trow[b + 1] : 0u;
                     int next = stage + 1;
                     uint32_t next_phase = phase;
                     if (next == kStages) {
@@ -242,30 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ready = mbar_test_wait(&full[next], next_phase);
                     const uint32_t base = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t b_addr = base + 2 * kStageA;
-                    issue_slab(d0, b, base, b_addr, tmem_base, tmem_base + kECol0, idesc_d, idesc_s);
-                    issue_slab(d1, b, base + kStageA, b_addr, tmem_base + kAcc1, tmem_base + kECol1, idesc_d,
-                               idesc_s);
+                    issue_slab(d, b, base + h * kStageA, base + 2 * kStageA, d_tmem, e_col, idesc_d, idesc_s);
                     any_mma = true;
                     if (g & 1) commit2_mask(&empty[(g >> 1) % (kStages / 2)], 3);
                     stage = next;
                     phase = next_phase;
-                    d0 = d0n;
-                    d1 = d1n;
+                    d = d_next;
                 }
                 if (!ok) break;
-                commit2_mask(acc_full, 3);
+                commit2_mask(&acc_full[h], 3);
             }
             if (*abort_flag && any_mma) {
-                commit2_local(drain);
+                commit2_local(&drain[h]);
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+                while (!mbar_try_wait(&drain[h], 0) && globaltimer() - t0 < kWaitLimitNs) {
                 }
             }
         }
     } else {
-        // ---------------- epilogue (8 warps, both CTAs) ----------------
-        const int h = (warp - kEpiWarp0) >> 2;   // accumulator (strip pair) this warp drains
+        // ---------------- epilogue (16 warps, both CTAs) ----------------
+        const int h = (warp - kEpiWarp0) >> 3;   // accumulator (strip pair) this warp drains
+        const int ch = ((warp - kEpiWarp0) >> 2) & 1;  // this warp takes every other 16-token chunk
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = 4 * c + 2 * h + (int)pr;
             const bool store = s < a.lins[l].S;
             const int nt = tile_tokens(j, a.M);
-            if (!mbar_wait(acc_full, t & 1, abort_flag)) {
+            if (!mbar_wait(&acc_full[h], t & 1, abort_flag)) {
                 if (lane == 0) raise();
                 break;
             }
@@ -285,15 +290,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + q * 32 + lane;
             if (store) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < nt; c0 += 16) {
+                for (int c0 = 16 * ch; c0 < nt; c0 += 32) {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(taddr + c0, v);
                     tc_wait_ld();
                     const int m0 = j * kBN + c0;
                     if (m0 + 16 <= a.M) {
+                        // Lanes 2i and 2i+1 hold rows 2i and 2i+1 of Y's columns;
+                        // one swap per two tokens lets each lane store both rows'
+                        // values of one token as a 4-byte pair (half the stores).
+                        __nv_bfloat16* yq = yc - lane + (lane & ~1);
+                        const bool odd = lane & 1;
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc)
-                            yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+                        for (int cc = 0; cc < 16; cc += 2) {
+                            const float x0 = __uint_as_float(v[cc]), x1 = __uint_as_float(v[cc + 1]);
+                            const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
+                            const __nv_bfloat162 two =
+                                odd ? __floats2bfloat162_rn(recv, x1) : __floats2bfloat162_rn(x0, recv);
+                            *reinterpret_cast<__nv_bfloat162*>(yq + (size_t)(m0 + cc + (odd ? 1 : 0)) * N) = two;
+                        }
                     } else {
 #pragma unroll
                         for (int cc = 0; cc < 16; ++cc)
@@ -304,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) remote_arrive(map_to_rank(smem_u32(acc_empty), 0));
+            if (lane == 0) remote_arrive(map_to_rank(smem_u32(&acc_empty[h]), 0));
         }
     }
 
