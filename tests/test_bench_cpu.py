@@ -27,3 +27,14 @@ def test_cpu_baseline_sample():
     rate, threads, desc = b.cpu_sample(budget_s=0.2, min_rows=1)
     assert rate > 0 and threads >= 1
     assert "oracle" in desc and "token rows" in desc
+
+
+def test_measured_traffic_is_pinned_to_source():
+    import hashlib
+    b = _bench()
+    for name, t in b.MEASURED_TRAFFIC.items():
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            same = hashlib.sha256(f.read()).hexdigest()[:16] == t["sha256"]
+        got = b.measured_traffic(name + " (any label)")
+        assert (got == t["bytes_per_launch"]) if same else (got is None)
+    assert b.measured_traffic("some_other_kernel") is None
