@@ -52,19 +52,19 @@ FRACS_SWEEP = [0.0, 0.5, 0.7, 0.9, 1.0]
 # that source is unchanged.
 MEASURED_TRAFFIC = {
     "hybrid_gemm22_kernel": {"source": "hybrid_sparse_gemm_b200/csrc/gemm22.cu", "sha256": "5dc947374cfc10d5",
-                             "bytes_per_launch": 407.19e6},
+                             "workload": ("llama32-1b", 4096, "128x128"), "bytes_per_launch": 407.19e6},
 }
 KERNEL_NAMES = {4: "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
                 6: "hybrid_gemm22_kernel (CTA pair, two strips per CTA, 512x240 tiles)",
                 3: "hybrid_gemm_kernel (single CTA, 128x128 tiles)"}
 
 
-def measured_traffic(kernel_name: str):
-    """ncu DRAM bytes per launch for this kernel, or None if none was taken on
-    the current source."""
+def measured_traffic(kernel_name: str, workload=("llama32-1b", 4096, "128x128")):
+    """ncu DRAM bytes per launch for this kernel on this workload, or None if
+    none was taken on the current source."""
     import hashlib
     for k, t in MEASURED_TRAFFIC.items():
-        if kernel_name.startswith(k):
+        if kernel_name.startswith(k) and tuple(t["workload"]) == tuple(workload):
             with open(os.path.join(ROOT, t["source"]), "rb") as f:
                 if hashlib.sha256(f.read()).hexdigest()[:16] == t["sha256"]:
                     return t["bytes_per_launch"]
@@ -144,10 +144,18 @@ class ClockSampler:
 
 # -------------------------------------------------------------- workload ---
 
-def model_linears(n_layers: int):
+# Model shapes the bench can run: (shape function, default tokens M, default layers).
+WORKLOADS = {
+    "llama32-1b": (synth.llama32_1b, 4096, 16, "Llama-3.2-1B"),
+    "llama2-7b": (synth.llama2_7b, 2048, 8, "Llama-2-7B"),
+    "llama2-13b": (synth.llama2_13b, 8192, 2, "Llama-2-13B"),
+}
+
+
+def model_linears(n_layers: int, shapes=synth.llama32_1b):
     out = []
     for layer in range(n_layers):
-        for l in synth.llama32_1b():
+        for l in shapes():
             out.append((layer, l))
     return out
 
@@ -155,28 +163,31 @@ def model_linears(n_layers: int):
 ROLE_INPUT = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "mlp", "up": "mlp", "down": "down"}
 
 
-def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1.0, rank=0, group=True):
+def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1.0, rank=0, group=True,
+                shapes=synth.llama32_1b, R=128, C=128):
     """Packs every linear of the model at global 2:4 fraction `frac`.
 
     Returns (layers, X, Y, frac): layers is a list of per-layer launch lists;
     each launch is (callable, [(PackedLinear, K, N, kept_weights, packed_bytes)]).
     q/k/v read one input, gate/up another, o and down their own; every linear
     writes its own output."""
-    lins = model_linears(n_layers)
-    T = [(l.N // 128) * (l.K // 128) for _, l in lins]
+    lins = model_linears(n_layers, shapes)
+    T = [(l.N // R) * (l.K // C) for _, l in lins]
     if frac in (0.0, 1.0):
         counts = [int(round(frac * t)) for t in T]
     else:
         counts = synth.split_fraction(T, frac, max(0.0, lo - (0.9 - frac)), min(1.0, hi - (0.9 - frac)),
                                       "model", seed, frac)
     X = {}
-    for role, K in (("attn", 2048), ("o", 2048), ("mlp", 2048), ("down", 8192)):
-        X[role] = synth.normal_bf16((M, K), 1.0, "cuda", "X", seed, rank, M, role)
+    for _, l in lins[:7]:
+        role = ROLE_INPUT[l.name]
+        if role not in X:
+            X[role] = synth.normal_bf16((M, l.K), 1.0, "cuda", "X", seed, rank, M, role)
     per_layer = {}
     for (layer, l), cnt in zip(lins, counts):
-        p = synth.make_problem(l.N, l.K, 0, R=128, C=128, n_sparse=cnt, seed=seed,
+        p = synth.make_problem(l.N, l.K, 0, R=R, C=C, n_sparse=cnt, seed=seed,
                                device="cuda", tag=f"L{layer}-{l.name}")
-        lin = hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu())
+        lin = hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu(), R, C)
         info = lin.info()
         kept = (info.slabs_total - info.slabs_sparse) * 128 * 64 + info.slabs_sparse * 128 * 32
         Yt = torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda")
@@ -249,14 +260,16 @@ def flops_dense(model, M):
     return sum(2.0 * M * m[2] * m[1] for m in members(model))
 
 
-def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
+def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1, workload: str = "llama32-1b",
+               M: int = 4096, R: int = 128, C: int = 128):
     """The oracle on a bounded sample of the workload: token rows of the 7
-    Llama-3.2-1B linears (one layer), as many rows as fit in about `budget_s`
-    seconds. Returns (dense-equivalent TFLOP/s, threads, description)."""
+    linears of one layer, as many rows as fit in about `budget_s` seconds.
+    Returns (dense-equivalent TFLOP/s, threads, description)."""
     import oracle
     oracle.build()
-    shapes = synth.llama32_1b()
-    probs = [synth.make_problem(l.N, l.K, 4096, R=128, C=128, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
+    shape_fn, _, _, model_name = WORKLOADS[workload]
+    shapes = shape_fn()
+    probs = [synth.make_problem(l.N, l.K, M, R=R, C=C, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
              for l in shapes]
     # calibrate: time 4 and 16 rows of every linear (after one untimed call
     # that starts the thread pool) and fit time = fixed + rows * per_row; the
@@ -272,7 +285,7 @@ def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
     t4, t16 = one_pass(4), one_pass(16)
     per_row = max((t16 - t4) / 12.0, 1e-6)
     fixed = max(t4 - 4 * per_row, 0.0)
-    rows = max(min_rows, min(4096, int((budget_s - fixed) / per_row)))
+    rows = max(min_rows, min(M, int((budget_s - fixed) / per_row)))
     flops = 0.0
     t0 = time.perf_counter()
     for l, p in zip(shapes, probs):
@@ -281,7 +294,7 @@ def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1):
     t = time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return flops / t / 1e12, threads, (f"oracle (expand mask, zero pruned weights, naive fp32 loop, OpenMP) "
-                                       f"on {rows} token rows x the 7 Llama-3.2-1B linears of one layer, "
+                                       f"on {rows} token rows x the 7 {model_name} linears of one layer, "
                                        f"{t:.1f} s")
 
 
@@ -342,8 +355,12 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=16)
-    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--workload", default="llama32-1b", choices=sorted(WORKLOADS),
+                    help="model whose linears one step runs (default: Llama-3.2-1B, M = 4096)")
+    ap.add_argument("--layers", type=int, default=None, help="layers per step (default per workload)")
+    ap.add_argument("--M", type=int, default=None, help="tokens (default per workload)")
+    ap.add_argument("--tile", default="128x128", choices=["128x128", "128x64", "64x128", "64x64"],
+                    help="mask tile shape")
     ap.add_argument("--no-group", action="store_true", help="one launch per linear instead of per layer")
     ap.add_argument("--path", default="auto", choices=["auto", "pair", "wide"],
                     help="tensor-core kernel for the timed steps (auto: the library's choice)")
@@ -356,17 +373,23 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    workload = (f"Llama-3.2-1B linears ({args.layers} layers x q,k,v,o,gate,up,down), M={args.M} tokens, "
-                f"bf16, 128x128 tiles, 90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]")
+    shape_fn, default_M, default_layers, model_name = WORKLOADS[args.workload]
+    if args.M is None:
+        args.M = default_M
+    if args.layers is None:
+        args.layers = default_layers
+    R, C = (int(v) for v in args.tile.split("x"))
+    workload = (f"{model_name} linears ({args.layers} layers x q,k,v,o,gate,up,down), M={args.M} tokens, "
+                f"bf16, {R}x{C} tiles, 90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]")
 
     if args.impl == "reference":
         if rank != 0:
             return
         steps_v = []
         for _ in range(min(args.warmup, 1)):
-            cpu_sample(budget_s=2.0)
+            cpu_sample(budget_s=2.0, workload=args.workload, M=args.M, R=R, C=C)
         for _ in range(args.steps):
-            v, threads, desc = cpu_sample(budget_s=5.0)
+            v, threads, desc = cpu_sample(budget_s=5.0, workload=args.workload, M=args.M, R=R, C=C)
             steps_v.append(v)
         val = statistics.median(steps_v)
         print(json.dumps({
@@ -391,8 +414,10 @@ def main():
     group = not args.no_group
 
     with torch.cuda.stream(stream):
-        model, X, _, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank, group=group)
-        dense_model, _, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank, group=group)
+        model, X, _, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank, group=group,
+                                             shapes=shape_fn, R=R, C=C)
+        dense_model, _, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank, group=group,
+                                           shapes=shape_fn, R=R, C=C)
     torch.cuda.synchronize()
     F = flops_dense(model, M)
     exec_flops = sum(2.0 * M * m[3] for m in members(model))
@@ -421,7 +446,8 @@ def main():
                 t = ms_h
             else:
                 with torch.cuda.stream(stream):
-                    mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group)
+                    mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group,
+                                               shapes=shape_fn, R=R, C=C)
                 t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
                 free_model(mdl)
                 del mdl
@@ -460,7 +486,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, threads, desc = cpu_sample()
+        v, threads, desc = cpu_sample(workload=args.workload, M=args.M, R=R, C=C)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     if rank == 0:
@@ -472,13 +498,13 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": workload, "M": M, "layers": args.layers, "linears": len(members(model)),
                        "launches_per_step": n_launch, "grouped": group,
-                       "frac_2to4": frac_real, "tile": "128x128",
+                       "frac_2to4": frac_real, "tile": args.tile,
                        "l2": "inputs larger than L2 (%.2f GB of packed weights per step)" % packed_gb,
                        "parallelism": f"dp{world} (M split, replicated weights)", "path": args.path},
             "speedup_vs_dense": ms_d / ms_h, "dense_ms_per_step": ms_d,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
-                         "traffic": measured_traffic(kernel_name),
+                         "traffic": measured_traffic(kernel_name, (args.workload, M, args.tile)),
                          "kernel": kernel_name,
                          "work": "2*M per kept weight of every loaded slab (a 2:4 slab counts half)",
                          "peak_kind": f"bf16 sustained ({peaks['source']})"},

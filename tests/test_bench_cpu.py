@@ -35,6 +35,7 @@ def test_measured_traffic_is_pinned_to_source():
     for name, t in b.MEASURED_TRAFFIC.items():
         with open(os.path.join(ROOT, t["source"]), "rb") as f:
             same = hashlib.sha256(f.read()).hexdigest()[:16] == t["sha256"]
-        got = b.measured_traffic(name + " (any label)")
+        got = b.measured_traffic(name + " (any label)", t["workload"])
         assert (got == t["bytes_per_launch"]) if same else (got is None)
+        assert b.measured_traffic(name, ("llama2-7b", 2048, "128x128")) is None
     assert b.measured_traffic("some_other_kernel") is None
