@@ -33,7 +33,7 @@ PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR, PATH_GEMV_SIM
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
             "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
-            "patch_group_linear", "patch_group_path", "patch_group_free"]
+            "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -58,6 +58,7 @@ _lib.patch_group_create.argtypes = [_P, _I, ctypes.POINTER(_P)]
 _lib.patch_group_linear.argtypes = [_P, _P, _I64, _P, _I, _P]
 _lib.patch_group_path.argtypes = [_P, _I64, _I, ctypes.POINTER(_I)]
 _lib.patch_group_free.argtypes = [_P]
+_lib.patch_selftest_wait.argtypes = [_P]
 _lib.patch_group_free.restype = None
 _lib.patch_unpack.argtypes = [_P, _P, _P]
 _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]

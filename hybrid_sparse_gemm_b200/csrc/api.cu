@@ -562,7 +562,7 @@ extern "C" {
 
 const char* patch_last_error(void) { return g_err.c_str(); }
 
-int patch_version(void) { return 3; }
+int patch_version(void) { return 4; }
 
 patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                         uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table, int64_t* packed_bytes) {
@@ -813,6 +813,25 @@ patch_status patch_group_path(patch_group g, int64_t M, int path, int* out) {
 }
 
 void patch_group_free(patch_group g) { free_group(g); }
+
+patch_status patch_selftest_wait(void* stream) {
+    int dev = 0;
+    PATCH_CUDA(cudaGetDevice(&dev));
+    patch_status st = check_device_is(dev);
+    if (st != PATCH_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* status = nullptr;
+    if (cudaMalloc(&status, sizeof(int)) != cudaSuccess) return fail(PATCH_ERR_NOMEM, "status word");
+    int host = 0;
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = launch_selftest_wait(status, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(status);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    if (host == kStatusTimeout) return fail(PATCH_ERR_TIMEOUT, "self-test: the bounded wait gave up as designed");
+    return PATCH_OK;
+}
 
 patch_status patch_unpack(patch_handle h, void* W_masked_bf16, void* stream) {
     if (!h || !W_masked_bf16) return fail(PATCH_ERR_ARG, "handle and output must be non-NULL");

@@ -75,6 +75,7 @@ cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters
 cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
 cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
+cudaError_t launch_selftest_wait(int* status, cudaStream_t st);
 cudaError_t gemm_prepare_single();
 cudaError_t gemm_prepare_pair(int* max_clusters);
 cudaError_t gemm_prepare_wide(int* max_clusters);

@@ -260,6 +260,18 @@ patch_status patch_check(patch_handle h, void* stream);
  * device first). NULL is ignored. */
 void patch_free(patch_handle h);
 
+/*
+ * patch_selftest_wait - exercise the device-side failure path on the current
+ * device: one CTA waits on a barrier that nothing completes, using the bounded
+ * wait every kernel uses (limit 1 s of %globaltimer). The wait gives up, the
+ * kernel records a timeout in a status word and returns; no fault, trap or
+ * hang is involved and the context stays usable. Synchronises `stream`.
+ * Returns PATCH_ERR_TIMEOUT when the path behaves as designed, PATCH_OK if the
+ * wait unexpectedly completed, PATCH_ERR_CUDA / NOMEM on a runtime failure.
+ * Not part of the product: a check for tests and deployment health probes.
+ */
+patch_status patch_selftest_wait(void* stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char* patch_last_error(void);
 

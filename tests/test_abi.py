@@ -40,7 +40,7 @@ def test_exports_every_header_symbol(hsg):
 
 
 def test_version(hsg):
-    assert hsg.version() == 3
+    assert hsg.version() == 4
 
 
 def _pack_status(hsg, W=0x1000, N=256, K=256, bits=0x2000, bitorder=0, flags=None, R=128, C=128):

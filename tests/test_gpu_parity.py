@@ -428,6 +428,22 @@ def test_group_path_choice(hsg):
     big.free()
 
 
+def test_device_wait_gives_up_and_context_survives(hsg, oracle_lib):
+    """The bounded wait every kernel uses: a barrier nothing completes makes
+    the kernel record a timeout and return (about 1 s); the error reaches the
+    host as PATCH_ERR_TIMEOUT and the next product is still correct."""
+    lib = hsg.library()
+    assert lib.patch_selftest_wait(None) == 6          # PATCH_ERR_TIMEOUT
+    assert b"gave up" in lib.patch_last_error()
+    p = synth.make_problem(512, 512, 40, frac=0.5, seed=9, device="cuda", tag="after-timeout")
+    lin = pack(hsg, p)
+    Y = lin(p.X)
+    torch.cuda.synchronize()
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what="after a device timeout")
+    lin.free()
+
+
 def test_group_argument_errors(hsg):
     import ctypes
     lib = hsg.library()
