@@ -16,7 +16,7 @@
 // TMEM (512 columns per CTA): accumulator 0 in columns [0, 240), accumulator
 // 1 in [256, 496), the 2:4 metadata of each strip in four columns at 240 and
 // 248. The accumulators are single-buffered: a tile's MMAs start once the
-// previous tile has been drained, while the producers keep filling stages.
+// previous tile has been drained, while the producers keep filling the ring.
 //
 // Partner strips (2p, 2p+1) load the same kind of record at every slab (the
 // packed format's dense images stand in for 2:4 slabs whose partner is
@@ -38,13 +38,15 @@ constexpr int kEpiWarps = 16;                   // per accumulator, two warps pe
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBN = kGemm22BN;                  // tokens per tile (both CTAs)
 constexpr int kHalfN = kBN / 2;                 // token rows of operand B per CTA
-constexpr int kStages = 4;
-constexpr int kStageA = 18432;                  // 16 KB dense, or 8 KB values + 2 KB metadata
-constexpr int kStageB = kHalfN * 128;           // 15 KB
-constexpr int kStageBytes = 2 * kStageA + kStageB;
-static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle atoms)");
-static_assert(kStages % 2 == 0 && kStages % kProducers == 0, "stages come in pairs dealt round robin");
-constexpr int kSmemData = kStages * kStageBytes;
+constexpr int kStageB = kHalfN * 128;           // 15 KB of activations per slab
+constexpr int kRecDense = 16384;                // dense slab image
+constexpr int kRecSparse = 10240;               // 2:4 values (8 KB) + room for the chunk's metadata (2 KB)
+constexpr int kRing = 208896;                   // shared-memory ring the slabs are placed in, in order
+constexpr int kQ = 8;                           // per-slab barriers: more than the slabs that fit in the ring
+static_assert(kRing % 1024 == 0 && kRecSparse % 1024 == 0 && kStageB % 1024 == 0,
+              "every record starts 1024-byte aligned (128-byte swizzle atoms)");
+static_assert(kRing / (2 * kRecSparse + kStageB) + 2 <= kQ, "slabs in flight stay within the barrier window");
+constexpr int kSmemData = kRing;
 constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kAcc1 = 256;                      // first column of accumulator 1
 constexpr int kECol0 = kBN;                     // metadata columns of strip pair 0
@@ -63,6 +65,25 @@ __device__ __forceinline__ int tile_tokens(int j, int M) {
 __device__ __forceinline__ uint32_t record_bytes(uint32_t d) {
     return ((d & kSlabSparse) ? kSparseValBytes : kDenseSlabBytes) + ((d & kSlabFirst) ? kMetaBytes : 0);
 }
+
+__device__ __forceinline__ uint32_t ring_rec(uint32_t d) { return (d & kSlabSparse) ? kRecSparse : kRecDense; }
+
+// Slabs are placed one after another in a ring of kRing bytes; a slab that
+// does not fit before the end starts again at 0. `pos` counts bytes placed so
+// far (including skipped ends); returns the ring offset of this slab.
+struct Ring {
+    uint32_t pos = 0, off = 0;
+    __device__ __forceinline__ uint32_t place(uint32_t size) {
+        if (off + size > (uint32_t)kRing) {
+            pos += (uint32_t)kRing - off;
+            off = 0;
+        }
+        const uint32_t at = off;
+        pos += size;
+        off += size;
+        return at;
+    }
+};
 
 // One strip pair's MMAs for one slab: 4 dense K=16 MMAs, or the metadata copy
 // (first 2:4 slab of a chunk) and 2 sparse K=32 MMAs.
@@ -93,9 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
-    uint64_t* full = bars;                       // leader: both CTAs' bytes of a stage
-    uint64_t* empty = full + kStages;            // every CTA: a stage pair consumed by the MMAs
-    uint64_t* acc_full = empty + kStages / 2;    // [2] both CTAs: accumulator h ready
+    uint64_t* full = bars;                       // [kQ] leader: both CTAs' bytes of slab g (at g % kQ)
+    uint64_t* empty = full + kQ;                 // [kQ] every CTA: slab g consumed by both issuers
+    uint64_t* acc_full = empty + kQ;             // [2] both CTAs: accumulator h ready
     uint64_t* acc_empty = acc_full + 2;          // [2] leader: the 16 epilogue warps of accumulator h drained it
     uint64_t* drain = acc_empty + 2;             // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
@@ -107,8 +128,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cl = blockIdx.x >> 1;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
-        for (int i = 0; i < kStages / 2; ++i) mbar_init(&empty[i], kMmaWarps);
+        for (int i = 0; i < kQ; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kMmaWarps);
+        }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&acc_full[h], 1);
             mbar_init(&acc_empty[h], kEpiWarps);  // its 8 epilogue warps in each of the 2 CTAs
@@ -147,9 +170,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kProducers) {
         if (lane == 0) {
             // ---------------- producers (both CTAs) ----------------
+            // Every producer walks the whole slab sequence to place each slab in
+            // the ring; it loads the slabs g with g % kProducers == me. Before
+            // loading, the slabs that last used those ring bytes must have been
+            // consumed (in-order, so waiting for the latest of them suffices).
             const int me = warp;
-            int g0 = 0;         // sequence index of the current unit's first slab
-            int my_last = -1;   // sequence index of the last slab this producer loaded
+            Ring ring;
+            uint32_t hist[kQ];   // ring positions where the last kQ slabs started
+            int g = 0;
+            int my_last = -1;    // sequence index of the last slab this producer loaded
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
@@ -167,38 +196,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const CUtensorMap* tm_a8 = &maps.a8[l];
                 const CUtensorMap* tm_e = &maps.e[l];
                 const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
-                for (int b = ((me - g0) % kProducers + kProducers) % kProducers; b < KB; b += kProducers) {
-                    const int g = g0 + b;
-                    const int q = g >> 1;
-                    if (!mbar_wait(&empty[q % (kStages / 2)], ((q / (kStages / 2)) & 1) ^ 1u, abort_flag)) {
-                        raise();
-                        ok = false;
-                        break;
-                    }
-                    const int stage = g % kStages;
+                for (int b = 0; b < KB; ++b, ++g) {
                     const uint32_t d0 = t0[b], d1 = t1[b];
-                    const uint32_t bar = map_to_rank(smem_u32(&full[stage]), 0);
-                    if (pr == 0) mbar_arrive_expect_tx(&full[stage], 2u * (record_bytes(d0) + record_bytes(d1) + kStageB));
-                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t r0 = ring_rec(d0), r1 = ring_rec(d1);
+                    const uint32_t off = ring.place(r0 + r1 + kStageB);
+                    hist[g % kQ] = ring.pos - (r0 + r1 + kStageB);
+                    if (g % kProducers != me) continue;
+                    if (ring.pos > (uint32_t)kRing) {
+                        const uint32_t need = ring.pos - (uint32_t)kRing;
+                        int jl = -1;
+                        for (int jj = g - 1; jj >= 0 && jj > g - kQ; --jj)
+                            if (hist[jj % kQ] < need) {
+                                jl = jj;
+                                break;
+                            }
+                        if (jl >= 0 && !mbar_wait(&empty[jl % kQ], (uint32_t)((jl / kQ) & 1), abort_flag)) {
+                            raise();
+                            ok = false;
+                            break;
+                        }
+                    }
+                    const uint32_t bar = map_to_rank(smem_u32(&full[g % kQ]), 0);
+                    if (pr == 0)
+                        mbar_arrive_expect_tx(&full[g % kQ], 2u * (record_bytes(d0) + record_bytes(d1) + kStageB));
+                    const uint32_t base = smem_u32(smem) + off;
                     tma_load_2d_pair(base, (d0 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0, (int)(slab_offset_bytes(d0) >> 7));
                     if (d0 & kSlabFirst)
                         tma_load_2d_pair(base + kSparseValBytes, tm_e, bar, 0, (int)(m0[b >> 1] >> 3));
-                    tma_load_2d_pair(base + kStageA, (d1 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0,
+                    tma_load_2d_pair(base + r0, (d1 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0,
                                      (int)(slab_offset_bytes(d1) >> 7));
                     if (d1 & kSlabFirst)
-                        tma_load_2d_pair(base + kStageA + kSparseValBytes, tm_e, bar, 0, (int)(m1[b >> 1] >> 3));
-                    tma_load_2d_pair(base + 2 * kStageA, tm_x, bar, b * kSlabK, tok);
+                        tma_load_2d_pair(base + r0 + kSparseValBytes, tm_e, bar, 0, (int)(m1[b >> 1] >> 3));
+                    tma_load_2d_pair(base + r0 + r1, tm_x, bar, b * kSlabK, tok);
                     my_last = g;
                 }
-                g0 += KB;
             }
             if (pr == 0) {
-                // Bounded wait for the loads of my last stages, whatever the
+                // Bounded wait for the loads of my last slabs, whatever the
                 // abort flag says, so none lands after the cluster exits.
-                for (int g = my_last - kStages + 1; g <= my_last; ++g) {
-                    if (g < 0 || g % kProducers != me) continue;
+                for (int gg = my_last - kQ + 1; gg <= my_last; ++gg) {
+                    if (gg < 0 || gg % kProducers != me) continue;
                     const uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1)) &&
+                    while (!mbar_try_wait(&full[gg % kQ], (uint32_t)((gg / kQ) & 1)) &&
                            globaltimer() - t0 < kWaitLimitNs) {
                     }
                 }
@@ -207,17 +246,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kMmaWarp + kMmaWarps) {
         if (lane == 0 && pr == 0) {
             // ---------------- MMA issuers (leader CTA), one per strip pair ----------------
-            // Both read every stage; a stage pair is free once both have
+            // Both read every slab; a slab's ring bytes are free once both have
             // committed it. Two issuing threads keep the tensor pipe fed while
             // either one waits on a barrier or computes descriptors.
             const int h = warp - kMmaWarp;
             const uint32_t d_tmem = tmem_base + (uint32_t)(h * kAcc1);
             const uint32_t e_col = tmem_base + (uint32_t)(h ? kECol1 : kECol0);
-            int stage = 0;
-            uint32_t phase = 0;
+            Ring ring;
             int g = 0;
             bool ok = true, any_mma = false;
-            bool ready = false;  // full[stage] already seen complete by the look-ahead
+            bool ready = false;  // full[g % kQ] already seen complete by the look-ahead
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
@@ -225,37 +263,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int lu = u & kUnitMask;
                 const int c = lu / a.MB, j = lu % a.MB;
                 const int KB = L.KB;
-                const uint32_t* trow = L.gemm + (size_t)strip_of(c, h, L.S) * KB;
+                // both strip pairs' records place the slab in the ring
+                const uint32_t* t0 = L.gemm + (size_t)strip_of(c, 0, L.S) * KB;
+                const uint32_t* t1 = L.gemm + (size_t)strip_of(c, 1, L.S) * KB;
                 const int nt = tile_tokens(j, a.M);
                 const uint32_t idesc_d = idesc_bf16(256, nt, false);
                 const uint32_t idesc_s = idesc_bf16(256, nt, true);
-                uint32_t d = trow[0];
+                uint32_t d0 = t0[0], d1 = t1[0];
                 if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
                     raise();
                     break;
                 }
                 tc_fence_after();
                 for (int b = 0; b < KB; ++b, ++g) {
-                    if (!ready && !mbar_wait(&full[stage], phase, abort_flag)) {
+                    if (!ready && !mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    const uint32_t d_next = b + 1 < KB ? trow[b + 1] : 0u;
-                    int next = stage + 1;
-                    uint32_t next_phase = phase;
-                    if (next == kStages) {
-                        next = 0;
-                        next_phase ^= 1u;
-                    }
-                    ready = mbar_test_wait(&full[next], next_phase);
-                    const uint32_t base = smem_u32(smem + stage * kStageBytes);
-                    issue_slab(d, b, base + h * kStageA, base + 2 * kStageA, d_tmem, e_col, idesc_d, idesc_s);
+                    const uint32_t d0n = b + 1 < KB ? t0[b + 1] : 0u;
+                    const uint32_t d1n = b + 1 < KB ? t1[b + 1] : 0u;
+                    ready = mbar_test_wait(&full[(g + 1) % kQ], (uint32_t)(((g + 1) / kQ) & 1));
+                    const uint32_t r0 = ring_rec(d0), r1 = ring_rec(d1);
+                    const uint32_t base = smem_u32(smem) + ring.place(r0 + r1 + kStageB);
+                    issue_slab(h ? d1 : d0, b, base + (h ? r0 : 0u), base + r0 + r1, d_tmem, e_col, idesc_d, idesc_s);
                     any_mma = true;
-                    if (g & 1) commit2_mask(&empty[(g >> 1) % (kStages / 2)], 3);
-                    stage = next;
-                    phase = next_phase;
-                    d = d_next;
+                    commit2_mask(&empty[g % kQ], 3);
+                    d0 = d0n;
+                    d1 = d1n;
                 }
                 if (!ok) break;
                 commit2_mask(&acc_full[h], 3);
@@ -270,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- epilogue (16 warps, both CTAs) ----------------
         const int h = (warp - kEpiWarp0) >> 3;   // accumulator (strip pair) this warp drains
-        const int ch = ((warp - kEpiWarp0) >> 2) & 1;  // this warp takes every other 16-token chunk
+        const int ch = ((warp - kEpiWarp0) >> 2) & 1;  // this warp takes every other 32-token chunk
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
@@ -289,20 +324,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kAcc1);
             __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + q * 32 + lane;
             if (store) {
+                // 32-column chunks, alternating between the two warps of a lane
+                // quarter (the last chunk of a 240-token tile has 16 columns).
 #pragma unroll 1
-                for (int c0 = 16 * ch; c0 < nt; c0 += 32) {
-                    uint32_t v[16];
-                    tmem_ld_32x32b_x16(taddr + c0, v);
+                for (int c0 = 32 * ch; c0 < nt; c0 += 64) {
+                    uint32_t v[32];
+                    const int cols = nt - c0 >= 32 ? 32 : 16;
+                    if (cols == 32)
+                        tmem_ld_32x32b_x32(taddr + c0, v);
+                    else
+                        tmem_ld_32x32b_x16(taddr + c0, v);
                     tc_wait_ld();
                     const int m0 = j * kBN + c0;
-                    if (m0 + 16 <= a.M) {
+                    if (m0 + cols <= a.M) {
                         // Lanes 2i and 2i+1 hold rows 2i and 2i+1 of Y's columns;
                         // one swap per two tokens lets each lane store both rows'
                         // values of one token as a 4-byte pair (half the stores).
                         __nv_bfloat16* yq = yc - lane + (lane & ~1);
                         const bool odd = lane & 1;
 #pragma unroll
-                        for (int cc = 0; cc < 16; cc += 2) {
+                        for (int cc = 0; cc < 32; cc += 2) {
+                            if (cc >= cols) break;
                             const float x0 = __uint_as_float(v[cc]), x1 = __uint_as_float(v[cc + 1]);
                             const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
                             const __nv_bfloat162 two =
@@ -311,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     } else {
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc)
-                            if (m0 + cc < a.M)
+                        for (int cc = 0; cc < 32; ++cc)
+                            if (cc < cols && m0 + cc < a.M)
                                 yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
                     }
                 }
