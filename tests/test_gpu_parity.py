@@ -206,6 +206,21 @@ def test_wide_tiles(hsg, oracle_lib, N, M, R, C, frac):
     lin.free()
 
 
+@pytest.mark.parametrize("K,C", [(64, 64), (128, 128), (192, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_wide_short_k(hsg, oracle_lib, K, C, frac):
+    """One to three slabs per tile: many tiles pass through the slab ring and
+    its per-slab barriers in one launch (both kinds of record mixed)."""
+    p = synth.make_problem(1024, K, 2000, R=128, C=C, frac=frac, seed=K, device="cuda", tag="wides")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMM_WIDE)
+    torch.cuda.synchronize()
+    lin.check()
+    assert torch.equal(Y, lin(p.X, path=hsg.PATH_GEMM_PAIR))
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(2000, 48, K), what=f"wide K={K}")
+    lin.free()
+
+
 def test_wide_long_k(hsg, oracle_lib):
     """Many slabs per tile (K = 4096) and several tiles per CTA pair."""
     p = synth.make_problem(1024, 4096, 2000, R=128, C=128, frac=0.7, seed=11, device="cuda", tag="widek")
