@@ -3,34 +3,36 @@
 // At decode sizes the layer is bound by the bytes of W it streams; 2:4 slabs
 // carry 1.125 bytes per weight instead of 2, which is where PATCH's hybrid
 // kernel earns its speed (abstract of "PATCH: Learnable Tile-level Hybrid
-// Sparsity for LLMs"). This kernel is a streaming engine: one persistent CTA
-// per SM walks a cost-balanced list of units (strip s, K-part p); warp 0 keeps
-// up to kStages packed slab records in flight with bulk copies (plus the
-// 16-token X tile by TMA), warp 1 runs them through tcgen05.mma / .mma.sp
-// with N = 16 into one of two TMEM accumulators, and two epilogue warpgroups
-// (one per accumulator, so consecutive units drain in parallel) write each
-// unit's fp32 partial (128 rows x 16 tokens) to a workspace. The CTA that
-// finishes the last part of a strip (per-strip arrival counter) sums the
-// strip's partials in part order, so the result does not depend on which CTA
-// finishes first, writes bf16 Y and re-arms the counter for the next call.
+// Sparsity for LLMs"). This kernel is a streaming engine: four persistent
+// CTAs per SM (four independent issue loops; one loop cannot issue slabs as
+// fast as HBM delivers them) walk a cost-balanced list of units (strip s,
+// K-part p); warp 0 keeps kStages slab records in flight as 2-D TMA boxes
+// over the packed bytes (plus the 16-token X box), warp 1 runs them through
+// tcgen05.mma / .mma.sp with N = 16 into one of two TMEM accumulators, and an
+// epilogue warpgroup drains them alternately, writing each unit's fp32
+// partial (128 rows x 16 tokens) to a workspace. The CTA that finishes the
+// last part of a strip (per-strip arrival counter) sums the strip's partials
+// in part order, so the result does not depend on which CTA finishes first,
+// writes bf16 Y and re-arms the counter for the next call.
 #include "kernels.cuh"
 
 namespace patch {
 
 namespace {
 
-constexpr int kThreads = 320;           // producer, MMA, two epilogue warpgroups
+constexpr int kEpiGroups = 1;           // epilogue warpgroups (units dealt round robin)
+constexpr int kThreads = 64 + 128 * kEpiGroups;  // producer warp, MMA warp, epilogue
 constexpr int kBN = kDecodeBN;           // tokens per MMA (M <= 16)
 constexpr int kStageA = 18432;           // 16 KB dense, or 8 KB values + 2 KB metadata
 constexpr int kStageX = kBN * 128;       // 2 KB, 128-byte swizzled
 constexpr int kStageBytes = kStageA + kStageX;
-constexpr int kStages = 5;                // two CTAs share an SM (kDecodeCtasPerSm)
+constexpr int kStages = 2;               // per CTA; kDecodeCtasPerSm CTAs share an SM
 constexpr int kSmemData = kStages * kStageBytes;
 constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kECol = 2 * kBN;           // metadata columns after the two accumulators
 constexpr int kTmemCols = 64;
 
-// Named barrier of one epilogue warpgroup (ids 1 and 2).
+// Named barrier of one epilogue warpgroup (id 1 + its index).
 __device__ __forceinline__ void epi_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);  // the four warps of warpgroup i
+            mbar_init(&acc_empty[i], 4);  // the four warps of the warpgroup draining it
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -220,30 +222,31 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
             }
         }
     } else {
-        // ---------------- epilogue: warpgroup g (warps 2+4g .. 5+4g) drains accumulator g ----------------
+        // ---------------- epilogue: warpgroup g (warps 2+4g .. 5+4g) drains every kEpiGroups-th unit ----------------
         const int g = (warp - 2) >> 2;
         const int q = warp & 3;          // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;
         const int leader = 64 + 128 * g;  // first thread of the warpgroup
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
-            if ((t & 1) != g) continue;  // the other warpgroup's unit
+            if (t % kEpiGroups != g) continue;  // another warpgroup's unit
+            const int acc = t & 1;
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const LinDesc& L = a.lins[l];
             const int P = L.P;
             const int s = lu / P, p = lu % P;
-            if (!mbar_wait(&acc_full[g], (t >> 1) & 1, abort_flag)) {
+            if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
                 if (lane == 0) raise();
                 break;
             }
             tc_fence_after();
             uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kBN), v);
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN), v);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[g]);
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
             __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
             if (P == 1) {
                 // whole strip in one unit: no partial sums

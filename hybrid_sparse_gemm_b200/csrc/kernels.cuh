@@ -85,6 +85,6 @@ constexpr int kGemmBN = 128;   // tokens per CTA tile (single-CTA kernel)
 constexpr int kGemm2BN = 256;  // tokens per CTA-pair tile
 constexpr int kGemm22BN = 240; // tokens per tile of the two-strips-per-CTA pair kernel
 constexpr int kDecodeBN = 16;  // tokens per decode MMA (M <= 16)
-constexpr int kDecodeCtasPerSm = 2;  // decode CTAs resident per SM (two issue loops per SM)
+constexpr int kDecodeCtasPerSm = 4;  // decode CTAs resident per SM (four issue loops per SM)
 
 }  // namespace patch
