@@ -46,6 +46,7 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 FRACS_SWEEP = [0.0, 0.5, 0.7, 0.9, 1.0]
+METRIC = "hybrid dense/2:4 GEMM dense-equiv TFLOP/s and speedup vs dense bf16, per sparsity"
 # DRAM bytes (read + write) of one launch of a kernel on the default workload
 # (one Llama-3.2-1B layer, M = 4096, 90 % 2:4 tiles), from an ncu capture, with
 # the sha256 prefix of the kernel source it was taken on: reported only while
@@ -393,10 +394,12 @@ def main():
             steps_v.append(v)
         val = statistics.median(steps_v)
         print(json.dumps({
-            "impl": "reference", "metric": "hybrid dense/2:4 GEMM dense-equiv TFLOP/s", "value": val,
+            "impl": "reference", "metric": METRIC, "value": val,
             "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
-            "data": "synthetic", "config": {"workload": workload, "sample": "token rows of one layer per step"},
+            "data": "synthetic", "config": {"workload": workload, "M": args.M, "layers": args.layers,
+                                            "tile": args.tile, "path": "cpu oracle",
+                                            "sample": "token rows of one layer per step"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
@@ -492,7 +495,7 @@ def main():
     if rank == 0:
         packed_gb = sum(m[4] for m in members(model)) / 1e9
         line = {
-            "metric": "hybrid dense/2:4 GEMM dense-equiv TFLOP/s and speedup vs dense bf16, per sparsity",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_h, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",

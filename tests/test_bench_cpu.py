@@ -39,3 +39,19 @@ def test_measured_traffic_is_pinned_to_source():
         assert (got == t["bytes_per_launch"]) if same else (got is None)
         assert b.measured_traffic(name, ("llama2-7b", 2048, "128x128")) is None
     assert b.measured_traffic("some_other_kernel") is None
+
+
+def test_reference_arm_line():
+    """--impl reference prints one JSON line on the same metric, unit and
+    direction as the GPU arm, from the CPU oracle."""
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    b = _bench()
+    assert line["impl"] == "reference" and line["metric"] == b.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
