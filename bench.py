@@ -36,6 +36,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -98,8 +99,13 @@ class ClockSampler:
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            # PATCH_CLOCKS_CSV keeps the raw samples at a chosen path; by default
+            # they go to a temporary file that is summarised into the JSON line.
+            self.path = os.environ.get("PATCH_CLOCKS_CSV") or os.path.join(
+                tempfile.gettempdir(), f"patch_clocks_{os.getpid()}.csv")
+            d = os.path.dirname(self.path)
+            if d:
+                os.makedirs(d, exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
