@@ -111,6 +111,13 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
+            # nvidia-smi needs a few hundred ms to start; hold the timed region
+            # until its first sample is on disk (at most 5 s).
+            t0 = time.time()
+            while time.time() - t0 < 5.0 and self.proc.poll() is None:
+                if os.path.getsize(self.path) > 0:
+                    break
+                time.sleep(0.02)
         except Exception:
             self.proc = None
         return self
@@ -267,42 +274,57 @@ def flops_dense(model, M):
     return sum(2.0 * M * m[2] * m[1] for m in members(model))
 
 
+class OracleSample:
+    """The oracle on a bounded sample of the workload: token rows of the 7
+    linears of one layer. Building the inputs and calibrating the cost model
+    happen once; `run(rows)` is one timed sample."""
+
+    def __init__(self, workload: str = "llama32-1b", M: int = 4096, R: int = 128, C: int = 128, seed: int = 0):
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        shape_fn, _, _, self.model_name = WORKLOADS[workload]
+        self.M = M
+        self.shapes = shape_fn()
+        self.probs = [synth.make_problem(l.N, l.K, M, R=R, C=C, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
+                      for l in self.shapes]
+        self.bits = [p.bits.numpy() for p in self.probs]
+        # calibrate: time 4 and 16 rows of every linear (after one untimed call
+        # that starts the thread pool) and fit time = fixed + rows * per_row; the
+        # fixed part (mask expansion over the whole weight) does not shrink with rows
+        oracle.linear(self.probs[0].X[:1], self.probs[0].W, self.bits[0])
+        t4, t16 = self.run(4)[1], self.run(16)[1]
+        self.per_row = max((t16 - t4) / 12.0, 1e-6)
+        self.fixed = max(t4 - 4 * self.per_row, 0.0)
+        self.threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+    def rows_for(self, budget_s: float, min_rows: int = 1) -> int:
+        return max(min_rows, min(self.M, int((budget_s - self.fixed) / self.per_row)))
+
+    def run(self, rows: int):
+        """One pass over the 7 linears on `rows` token rows; returns
+        (dense-equivalent TFLOP/s, seconds)."""
+        flops = 0.0
+        t0 = time.perf_counter()
+        for l, p, b in zip(self.shapes, self.probs, self.bits):
+            self.oracle.linear(p.X[:rows], p.W, b)
+            flops += 2.0 * rows * l.N * l.K
+        t = time.perf_counter() - t0
+        return flops / t / 1e12, t
+
+    def describe(self, rows: int, t: float) -> str:
+        return (f"oracle (expand mask, zero pruned weights, naive fp32 loop, OpenMP) on {rows} token rows "
+                f"x the 7 {self.model_name} linears of one layer, {t:.1f} s")
+
+
 def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1, workload: str = "llama32-1b",
                M: int = 4096, R: int = 128, C: int = 128):
-    """The oracle on a bounded sample of the workload: token rows of the 7
-    linears of one layer, as many rows as fit in about `budget_s` seconds.
+    """One bounded oracle sample of about `budget_s` seconds.
     Returns (dense-equivalent TFLOP/s, threads, description)."""
-    import oracle
-    oracle.build()
-    shape_fn, _, _, model_name = WORKLOADS[workload]
-    shapes = shape_fn()
-    probs = [synth.make_problem(l.N, l.K, M, R=R, C=C, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
-             for l in shapes]
-    # calibrate: time 4 and 16 rows of every linear (after one untimed call
-    # that starts the thread pool) and fit time = fixed + rows * per_row; the
-    # fixed part (mask expansion over the whole weight) does not shrink with rows
-    oracle.linear(probs[0].X[:1], probs[0].W, probs[0].bits.numpy())
-
-    def one_pass(r):
-        t0 = time.perf_counter()
-        for p in probs:
-            oracle.linear(p.X[:r], p.W, p.bits.numpy())
-        return time.perf_counter() - t0
-
-    t4, t16 = one_pass(4), one_pass(16)
-    per_row = max((t16 - t4) / 12.0, 1e-6)
-    fixed = max(t4 - 4 * per_row, 0.0)
-    rows = max(min_rows, min(M, int((budget_s - fixed) / per_row)))
-    flops = 0.0
-    t0 = time.perf_counter()
-    for l, p in zip(shapes, probs):
-        oracle.linear(p.X[:rows], p.W, p.bits.numpy())
-        flops += 2.0 * rows * l.N * l.K
-    t = time.perf_counter() - t0
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return flops / t / 1e12, threads, (f"oracle (expand mask, zero pruned weights, naive fp32 loop, OpenMP) "
-                                       f"on {rows} token rows x the 7 {model_name} linears of one layer, "
-                                       f"{t:.1f} s")
+    s = OracleSample(workload, M, R, C, seed)
+    rows = s.rows_for(budget_s, min_rows)
+    v, t = s.run(rows)
+    return v, s.threads, s.describe(rows, t)
 
 
 def decode_bench(hsg, stream, peaks, steps=20):
@@ -392,13 +414,19 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps_v = []
+        # each step is one bounded sample, sized so that all K steps take
+        # about a minute and a half of CPU time (0.25 s to 5 s per step)
+        samp = OracleSample(args.workload, args.M, R, C)
+        rows = samp.rows_for(max(0.25, min(5.0, 90.0 / max(1, args.steps))))
         for _ in range(min(args.warmup, 1)):
-            cpu_sample(budget_s=2.0, workload=args.workload, M=args.M, R=R, C=C)
+            samp.run(rows)
+        steps_v, secs = [], []
         for _ in range(args.steps):
-            v, threads, desc = cpu_sample(budget_s=5.0, workload=args.workload, M=args.M, R=R, C=C)
+            v, t = samp.run(rows)
             steps_v.append(v)
+            secs.append(t)
         val = statistics.median(steps_v)
+        threads, desc = samp.threads, samp.describe(rows, statistics.median(secs)) + " per step"
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val,
             "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
