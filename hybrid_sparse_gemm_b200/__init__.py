@@ -33,7 +33,8 @@ PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR, PATH_GEMV_SIM
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
             "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
-            "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait"]
+            "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait",
+            "patch_partition_rows"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -65,13 +66,14 @@ _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]
 _lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
 _lib.patch_check.argtypes = [_P, _P]
 _lib.patch_plan.argtypes = [_I64, _I64, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I64)]
+_lib.patch_partition_rows.argtypes = [_I64, _I64, _P, _I, _I, _I, _I64, _P]
 _lib.patch_free.argtypes = [_P]
 _lib.patch_free.restype = None
 _lib.patch_last_error.restype = ctypes.c_char_p
 _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
            "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc",
-           "patch_group_create", "patch_group_linear"]:
+           "patch_group_create", "patch_group_linear", "patch_partition_rows"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -118,6 +120,21 @@ def patch_plan(N: int, K: int, tile_flags, tile_rows: int = 128, tile_cols: int 
     _check(_lib.patch_plan(N, K, flags.ctypes.data, tile_rows, tile_cols, slab.ctypes.data,
                            meta.ctypes.data, gemm.ctypes.data, ctypes.byref(nbytes)))
     return (slab[:ns], meta[:nm], gemm[:ng]), int(nbytes.value)
+
+
+def patch_partition_rows(N: int, K: int, tile_flags, parts: int, tile_rows: int = 128, tile_cols: int = 128,
+                         align_rows: int = 256) -> list[int]:
+    """Host-only: parts + 1 row bounds of a cost-balanced contiguous split of W."""
+    import numpy as np
+    flags = np.ascontiguousarray(np.asarray(tile_flags, dtype=np.uint8).reshape(-1))
+    if tile_rows > 0 and tile_cols > 0 and N % tile_rows == 0 and K % tile_cols == 0 and N > 0 and K > 0:
+        if flags.size != (N // tile_rows) * (K // tile_cols):
+            raise ValueError(f"tile_flags has {flags.size} entries, the {N}x{K} weight has "
+                             f"{(N // tile_rows) * (K // tile_cols)} tiles")
+    bounds = np.zeros(max(parts, 0) + 1, np.int64)
+    _check(_lib.patch_partition_rows(N, K, flags.ctypes.data, tile_rows, tile_cols, parts, align_rows,
+                                     bounds.ctypes.data))
+    return [int(b) for b in bounds]
 
 
 def patch_pack(W: torch.Tensor, mask_bits: torch.Tensor, tile_flags, tile_rows: int = 128,

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -578,6 +579,70 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
     if (meta_table) memcpy(meta_table, p.meta.data(), sizeof(uint32_t) * p.meta.size());
     if (gemm_table) memcpy(gemm_table, p.gemm.data(), sizeof(uint32_t) * p.gemm.size());
     if (packed_bytes) *packed_bytes = p.bytes;
+    return PATCH_OK;
+}
+
+patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
+                                  int parts, int64_t align_rows, int64_t* bounds) {
+    g_err.clear();
+    if (!tile_flags || !bounds) return fail(PATCH_ERR_ARG, "tile_flags and bounds must be non-NULL");
+    if (parts < 1) return fail(PATCH_ERR_ARG, "parts must be at least 1");
+    if (align_rows <= 0 || align_rows % (2 * kStrip) != 0)
+        return fail(PATCH_ERR_ARG, "align_rows must be a positive multiple of 256");
+    patch_status st = check_shape(N, K, tile_rows, tile_cols);
+    if (st != PATCH_OK) return st;
+    st = check_flags(tile_flags, (N / tile_rows) * (K / tile_cols));
+    if (st != PATCH_OK) return st;
+    Plan p;
+    build_plan(p, N, K, tile_rows, tile_cols, tile_flags);
+    // Unit u = align_rows / 256 consecutive strip pairs. Its cost, in half
+    // dense slabs so that it is an integer: every slab of a pair (dense 2,
+    // paired 2:4 1) plus 2 for the pair's epilogue, as the tile scheduler counts.
+    const int64_t per_unit = align_rows / (2 * kStrip);
+    const int64_t pairs = (int64_t)p.pair_cost.size();
+    const int64_t units = (pairs + per_unit - 1) / per_unit;
+    std::vector<int64_t> cost((size_t)units, 0);
+    for (int64_t q = 0; q < pairs; ++q) cost[(size_t)(q / per_unit)] += (int64_t)llround(2.0 * p.pair_cost[q]) + 2;
+    // Smallest bottleneck T that a left-to-right greedy packing fits into
+    // `parts` contiguous parts (the greedy is optimal for a given T).
+    auto parts_needed = [&](int64_t T) {
+        int64_t n = 1, acc = 0;
+        for (int64_t c : cost) {
+            if (acc + c > T) {
+                ++n;
+                acc = c;
+            } else {
+                acc += c;
+            }
+        }
+        return n;
+    };
+    int64_t lo = 0, hi = 0;
+    for (int64_t c : cost) {
+        lo = std::max(lo, c);
+        hi += c;
+    }
+    while (lo < hi) {
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (parts_needed(mid) <= parts)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    // Lay the parts out under T = lo, stopping a part early only to leave
+    // one unit for every later part, so no rank idles while units remain.
+    int64_t u = 0;
+    bounds[0] = 0;
+    for (int r = 0; r < parts; ++r) {
+        const int64_t later = parts - 1 - r;
+        int64_t acc = 0;
+        while (u < units && acc + cost[(size_t)u] <= lo && (acc == 0 || units - u - 1 >= later)) {
+            acc += cost[(size_t)u];
+            ++u;
+        }
+        bounds[r + 1] = std::min<int64_t>(N, u * align_rows);
+    }
+    if (u != units) return fail(PATCH_ERR_ARG, "internal: partition left rows unassigned");
     return PATCH_OK;
 }
 

@@ -131,6 +131,35 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
                         int64_t* packed_bytes);
 
 /*
+ * patch_partition_rows - split W's rows into `parts` contiguous shards of
+ * balanced tensor-core cost, for a tensor-parallel (output-feature) split of
+ * one linear across ranks. Computed on the host; touches no device.
+ *
+ * Why: each tile's dense / 2:4 choice is learned on its own, and the
+ * abstract of "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs" notes
+ * that the learned sparsity is non-uniform across layers; rows of one weight
+ * differ in the same way, so equal row counts would leave the ranks with the
+ * sparsest rows idle.
+ *
+ *   N, K, tile_flags, tile_rows, tile_cols  as for patch_pack (the whole W).
+ *   parts       number of shards (ranks), >= 1.
+ *   align_rows  every bound is a multiple of this many rows, or N; a
+ *               positive multiple of 256 so that no strip pair is cut.
+ *   bounds      host, parts + 1 int64: shard r is rows [bounds[r], bounds[r+1])
+ *               of W (and columns of Y); bounds[0] = 0, bounds[parts] = N,
+ *               non-decreasing. A shard is empty only when there are fewer
+ *               aligned blocks than parts (the trailing shards then are).
+ * Cost of a strip pair (256 rows): for each 64-column slab, 1 when dense and
+ * 1/2 when 2:4 in both strips, plus 1 for its epilogue. The split minimises
+ * the largest shard's cost over all contiguous aligned splits. Each shard
+ * W[bounds[r]:bounds[r+1]] with its rows of mask bits and tile flags is a
+ * valid patch_pack input. Same shape and flag errors as patch_plan;
+ * PATCH_ERR_ARG for a NULL pointer, parts < 1 or a bad align_rows.
+ */
+patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows,
+                                  int tile_cols, int parts, int64_t align_rows, int64_t* bounds);
+
+/*
  * patch_linear - Y = X . (W (.) Mask)^T for the packed weights of h.
  *
  *   X_bf16  dev, M*K bf16 row-major, 16-byte aligned.

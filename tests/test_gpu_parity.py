@@ -471,3 +471,40 @@ def test_group_argument_errors(hsg):
     assert lib.patch_group_create(arr, 0, ctypes.byref(g)) == 1
     assert lib.patch_group_linear(None, None, 4, None, 0, None) == 1
     lin.free()
+
+
+# ------------------------------------------------ output-feature split ---
+
+def test_row_sharded_single_rank_is_the_whole_linear(hsg):
+    """One rank: the split is the whole weight, and the product is bit-equal
+    to the unsplit linear's."""
+    from hybrid_sparse_gemm_b200 import dist
+    p = synth.make_problem(1280, 512, 300, R=64, C=128, frac=0.7, seed=21, device="cuda", tag="tp1")
+    whole = pack(hsg, p)
+    tp = dist.RowShardedLinear(p.W, p.bits, p.flags, p.R, p.C, rank=0, world=1)
+    assert tp.bounds == [0, 1280]
+    for M in (300, 5):
+        X = p.X[:M].contiguous()
+        assert torch.equal(tp(X), whole(X))
+    torch.cuda.synchronize()
+    tp.free()
+    whole.free()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("M", [300, 5])
+def test_row_shards_assemble_the_product(hsg, oracle_lib, world, M):
+    """Every rank's shard packed and run on this GPU in turn; its columns put
+    side by side give the whole product within the parity bar."""
+    from hybrid_sparse_gemm_b200 import dist
+    p = synth.make_problem(1536, 512, M, R=128, C=128, frac=0.6, seed=22, device="cuda", tag=f"tp{world}")
+    Y = torch.empty((M, 1536), dtype=torch.bfloat16, device="cuda")
+    shards = [dist.RowShardedLinear(p.W, p.bits, p.flags, p.R, p.C, rank=r, world=world) for r in range(world)]
+    for r, tp in enumerate(shards):
+        n0, n1 = tp.bounds[r], tp.bounds[r + 1]
+        assert n1 > n0
+        Y[:, n0:n1] = tp.lin(p.X)
+    torch.cuda.synchronize()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"{world} shards, M={M}")
+    for tp in shards:
+        tp.free()
