@@ -34,7 +34,7 @@ EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_hos
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
             "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
             "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait",
-            "patch_partition_rows"]
+            "patch_partition_rows", "patch_classify_tiles"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -67,13 +67,14 @@ _lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
 _lib.patch_check.argtypes = [_P, _P]
 _lib.patch_plan.argtypes = [_I64, _I64, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I64)]
 _lib.patch_partition_rows.argtypes = [_I64, _I64, _P, _I, _I, _I, _I64, _P]
+_lib.patch_classify_tiles.argtypes = [_P, _I64, _I64, _I, _I, _P, ctypes.POINTER(_I64)]
 _lib.patch_free.argtypes = [_P]
 _lib.patch_free.restype = None
 _lib.patch_last_error.restype = ctypes.c_char_p
 _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
            "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc",
-           "patch_group_create", "patch_group_linear", "patch_partition_rows"]:
+           "patch_group_create", "patch_group_linear", "patch_partition_rows", "patch_classify_tiles"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -120,6 +121,22 @@ def patch_plan(N: int, K: int, tile_flags, tile_rows: int = 128, tile_cols: int 
     _check(_lib.patch_plan(N, K, flags.ctypes.data, tile_rows, tile_cols, slab.ctypes.data,
                            meta.ctypes.data, gemm.ctypes.data, ctypes.byref(nbytes)))
     return (slab[:ns], meta[:nm], gemm[:ng]), int(nbytes.value)
+
+
+def patch_classify_tiles(mask_bits, N: int, K: int, tile_rows: int = 128, tile_cols: int = 128):
+    """Host-only: (tile flags as a uint8 numpy array [N/tile_rows, K/tile_cols],
+    number of dense tiles that prune some weight) for a bit-packed mask."""
+    import numpy as np
+    bits = mask_bits.cpu().numpy() if isinstance(mask_bits, torch.Tensor) else np.asarray(mask_bits)
+    bits = np.ascontiguousarray(bits.reshape(-1), dtype=np.uint8)
+    if bits.size != (N * K + 7) // 8:
+        raise ValueError(f"mask_bits has {bits.size} bytes, a {N}x{K} mask needs {(N * K + 7) // 8}")
+    ok = tile_rows > 0 and tile_cols > 0 and N > 0 and K > 0 and N % tile_rows == 0 and K % tile_cols == 0
+    flags = np.zeros(max((N // tile_rows) * (K // tile_cols) if ok else 1, 1), np.uint8)
+    stray = _I64(0)
+    _check(_lib.patch_classify_tiles(bits.ctypes.data, N, K, tile_rows, tile_cols, flags.ctypes.data,
+                                     ctypes.byref(stray)))
+    return flags.reshape(N // tile_rows, K // tile_cols), int(stray.value)
 
 
 def patch_partition_rows(N: int, K: int, tile_flags, parts: int, tile_rows: int = 128, tile_cols: int = 128,

@@ -582,6 +582,34 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
     return PATCH_OK;
 }
 
+patch_status patch_classify_tiles(const uint8_t* mask_bits, int64_t N, int64_t K, int tile_rows, int tile_cols,
+                                  uint8_t* tile_flags, int64_t* dense_with_pruned) {
+    g_err.clear();
+    if (!mask_bits || !tile_flags) return fail(PATCH_ERR_ARG, "mask_bits and tile_flags must be non-NULL");
+    patch_status st = check_shape(N, K, tile_rows, tile_cols);
+    if (st != PATCH_OK) return st;
+    // K and the tile width are multiples of 8, so every mask byte holds two
+    // whole groups of four k (one per nibble) in either bit order.
+    auto two_of_four = [](unsigned v) { return __builtin_popcount(v) == 2; };
+    const int64_t tiles_k = K / tile_cols, row_bytes = K / 8, tile_bytes = tile_cols / 8;
+    int64_t stray = 0;
+    for (int64_t tr = 0; tr < N / tile_rows; ++tr)
+        for (int64_t tc = 0; tc < tiles_k; ++tc) {
+            bool sparse = true, full = true;
+            for (int64_t r = tr * tile_rows; r < (tr + 1) * tile_rows; ++r) {
+                const uint8_t* row = mask_bits + r * row_bytes + tc * tile_bytes;
+                for (int64_t i = 0; i < tile_bytes; ++i) {
+                    sparse = sparse && two_of_four(row[i] >> 4) && two_of_four(row[i] & 15u);
+                    full = full && row[i] == 0xFF;
+                }
+            }
+            tile_flags[tr * tiles_k + tc] = sparse ? 1 : 0;
+            stray += !sparse && !full;
+        }
+    if (dense_with_pruned) *dense_with_pruned = stray;
+    return PATCH_OK;
+}
+
 patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                                   int parts, int64_t align_rows, int64_t* bounds) {
     g_err.clear();

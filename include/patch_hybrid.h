@@ -131,6 +131,30 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
                         int64_t* packed_bytes);
 
 /*
+ * patch_classify_tiles - the tile flags a keep/prune mask implies, computed
+ * on the host, for a mask that comes without them (a released mask file
+ * holds the mask only: model card "llama_3.2_1b-PATCH-45Sparse", release
+ * paragraph and "How to use").
+ *
+ *   mask_bits  host, ceil(N*K/8) bytes, the keep bits of W[N,K] row-major,
+ *              8 per byte, in either bit order (the rule below reads whole
+ *              groups of four, which never straddle a byte).
+ *   N, K, tile_rows, tile_cols  as for patch_pack.
+ *   tile_flags  host, (N/tile_rows)*(K/tile_cols) bytes written, row-major
+ *              over the tile grid: 1 when every group of four consecutive k
+ *              in every row of the tile keeps exactly two (a 2:4 tile), else
+ *              0 (dense; the method's dense tiles keep every weight:
+ *              "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs",
+ *              abstract, and the card's method paragraph).
+ *   dense_with_pruned  receives the number of dense tiles that still prune
+ *              some weight (patch_pack stores W (.) Mask for those, so the
+ *              product stays exact, at dense cost), or NULL.
+ * Same shape errors as patch_pack; PATCH_ERR_ARG for a NULL buffer.
+ */
+patch_status patch_classify_tiles(const uint8_t* mask_bits, int64_t N, int64_t K, int tile_rows,
+                                  int tile_cols, uint8_t* tile_flags, int64_t* dense_with_pruned);
+
+/*
  * patch_partition_rows - split W's rows into `parts` contiguous shards of
  * balanced tensor-core cost, for a tensor-parallel (output-feature) split of
  * one linear across ranks. Computed on the host; touches no device.
