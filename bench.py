@@ -92,10 +92,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, cmd=None):
         self.idx = device_index
+        self.cmd = cmd or ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                           "--format=csv,noheader,nounits", "-lms", "50"]
         self.proc = None
         self.path = None
+        self.fh = None
 
     def __enter__(self):
         try:
@@ -107,10 +110,7 @@ class ClockSampler:
             if d:
                 os.makedirs(d, exist_ok=True)
             self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.fh,
-                stderr=subprocess.DEVNULL)
+            self.proc = subprocess.Popen(self.cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
             # nvidia-smi needs a few hundred ms to start; hold the timed region
             # until its first sample is on disk (at most 5 s).
             t0 = time.time()
@@ -120,6 +120,9 @@ class ClockSampler:
                 time.sleep(0.02)
         except Exception:
             self.proc = None
+            if self.fh is not None:
+                self.fh.close()
+                self.fh = None
         return self
 
     def __exit__(self, *exc):
@@ -135,7 +138,11 @@ class ClockSampler:
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
-        for line in open(self.path):
+        with open(self.path) as f:
+            lines = f.readlines()
+        if not os.environ.get("PATCH_CLOCKS_CSV"):
+            os.remove(self.path)  # the temporary file; its summary goes into the JSON line
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue

@@ -3,6 +3,7 @@ loads, and the CPU baseline (the oracle on a bounded row sample) runs and
 reports a positive rate."""
 import importlib.util
 import os
+import time
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -55,3 +56,26 @@ def test_reference_arm_line():
     assert line["impl"] == "reference" and line["metric"] == b.METRIC
     assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_sampler_summary():
+    """The clock record: median SM clock under load, the throttle reasons that
+    were active, samples below 300 W left out; the temporary file is removed."""
+    import sys
+    b = _bench()
+    script = ("import time\n"
+              "rows = ['0, 100, 1965, 80.0, 0x0, Not Active, Not Active, Not Active, Not Active',\n"
+              "        '0, 1700, 1965, 650.0, 0x4, Not Active, Not Active, Not Active, Active',\n"
+              "        '0, 1800, 1965, 700.0, 0x4, Not Active, Not Active, Not Active, Active']\n"
+              "for r in rows * 400:\n"
+              "    print(r, flush=True)\n"
+              "    time.sleep(0.01)\n")
+    with b.ClockSampler(0, cmd=[sys.executable, "-c", script]) as c:
+        time.sleep(0.5)
+    got = c.summary()
+    assert got["sm_mhz"] in (1700.0, 1750.0, 1800.0) and got["sm_max_mhz"] == 1965.0
+    assert got["reasons"] == ["sw_power_cap"] and got["power_w_max"] == 700.0
+    assert not os.path.exists(c.path)
+    with b.ClockSampler(0, cmd=["/nonexistent/nvidia-smi"]) as c:
+        pass
+    assert c.summary()["sm_mhz"] is None
