@@ -567,7 +567,6 @@ int patch_version(void) { return 4; }
 
 patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                         uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table, int64_t* packed_bytes) {
-    g_err.clear();
     if (!tile_flags) return fail(PATCH_ERR_ARG, "tile_flags is NULL");
     patch_status st = check_shape(N, K, tile_rows, tile_cols);
     if (st != PATCH_OK) return st;
@@ -584,7 +583,6 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
 
 patch_status patch_classify_tiles(const uint8_t* mask_bits, int64_t N, int64_t K, int tile_rows, int tile_cols,
                                   uint8_t* tile_flags, int64_t* dense_with_pruned) {
-    g_err.clear();
     if (!mask_bits || !tile_flags) return fail(PATCH_ERR_ARG, "mask_bits and tile_flags must be non-NULL");
     patch_status st = check_shape(N, K, tile_rows, tile_cols);
     if (st != PATCH_OK) return st;
@@ -612,7 +610,6 @@ patch_status patch_classify_tiles(const uint8_t* mask_bits, int64_t N, int64_t K
 
 patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                                   int parts, int64_t align_rows, int64_t* bounds) {
-    g_err.clear();
     if (!tile_flags || !bounds) return fail(PATCH_ERR_ARG, "tile_flags and bounds must be non-NULL");
     if (parts < 1) return fail(PATCH_ERR_ARG, "parts must be at least 1");
     if (align_rows <= 0 || align_rows % (2 * kStrip) != 0)
@@ -677,7 +674,6 @@ patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flag
 patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t* mask_bits, int bitorder,
                         const uint8_t* tile_flags, int tile_rows, int tile_cols, void* stream,
                         patch_handle* out) {
-    g_err.clear();
     if (!out) return fail(PATCH_ERR_ARG, "out is NULL");
     *out = nullptr;
     if (!W_bf16 || !mask_bits || !tile_flags)
@@ -868,7 +864,6 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
 }
 
 patch_status patch_group_create(const patch_handle* handles, int n, patch_group* out) {
-    g_err.clear();
     if (!out) return fail(PATCH_ERR_ARG, "out is NULL");
     *out = nullptr;
     if (!handles || n < 1 || n > kMaxGroup) return fail(PATCH_ERR_ARG, "a group takes 1 to %d handles", kMaxGroup);

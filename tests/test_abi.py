@@ -124,3 +124,47 @@ def test_plan_errors(hsg):
     with pytest.raises(hsg.PatchError) as e:
         hsg.patch_plan(256, 256, np.full(4, 3, np.uint8), 128, 128)
     assert e.value.status == 1
+
+
+def test_group_and_noalloc_reject_bad_arguments(hsg):
+    lib = hsg.library()
+    g = ctypes.c_void_p()
+    assert lib.patch_linear_noalloc(None, 0x1000, 4, 0x2000, None) == 1
+    assert lib.patch_group_create(None, 1, ctypes.byref(g)) == 1 and g.value is None
+    nulls = (ctypes.c_void_p * 2)()
+    assert lib.patch_group_create(nulls, 2, ctypes.byref(g)) == 1
+    assert b"handle 0 is NULL" in lib.patch_last_error()
+    assert lib.patch_group_create(nulls, 0, ctypes.byref(g)) == 1
+    assert lib.patch_group_create(nulls, 1, None) == 1
+    out = ctypes.c_int(-1)
+    assert lib.patch_group_path(None, 16, 0, ctypes.byref(out)) == 1 and out.value == -1
+    assert lib.patch_group_linear(None, None, 4, None, 0, None) == 1
+    lib.patch_group_free(None)  # ignored
+
+
+def test_last_error_is_the_last_failure_of_this_thread(hsg):
+    import threading
+    lib = hsg.library()
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(lib.patch_last_error()))
+    t.start()
+    t.join()
+    assert seen == [b""]                       # a thread with no failed call
+    assert lib.patch_linear(None, 0x1000, 4, 0x2000, None) == 1
+    msg = lib.patch_last_error()
+    assert b"NULL" in msg
+    # a successful call leaves the last failure's message in place
+    assert hsg.patch_partition_rows(256, 128, np.zeros((2, 1), np.uint8), 1) == [0, 256]
+    assert lib.patch_last_error() == msg
+    t = threading.Thread(target=lambda: seen.append(lib.patch_last_error()))
+    t.start()
+    t.join()
+    assert seen[-1] == b""                     # other threads do not see it
+
+
+def test_selftest_without_device(hsg):
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    lib = hsg.library()
+    assert lib.patch_selftest_wait(None) in (5, 8)
+    assert lib.patch_last_error()
