@@ -467,13 +467,16 @@ def main():
     exec_flops = sum(2.0 * M * m[3] for m in members(model))
     n_launch = len(model)
 
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    nvtx = torch.cuda.nvtx  # phase markers for profilers; nothing inside the timed loops
+    with ClockSampler(torch.cuda.current_device()) as clk, nvtx.range("hybrid steps"):
         ms_h, _ = time_steps(hsg, model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
     clocks = clk.summary()
-    ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
+    with nvtx.range("dense steps"):
+        ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
     # per-launch durations for the roofline (separate pass, events around each launch)
-    _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on, per_launch=True,
-                              path=gpath)
+    with nvtx.range("per-launch timing"):
+        _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on,
+                                  per_launch=True, path=gpath)
     kern_ms = statistics.mean(sum(row) for row in launch_ms)
     kernel_name = KERNEL_NAMES.get(model[0][0].path(M, gpath) if model[0][0] is not None else hsg.PATH_GEMM_PAIR,
                                    "tensor-core GEMM")
@@ -492,7 +495,8 @@ def main():
                 with torch.cuda.stream(stream):
                     mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group,
                                                shapes=shape_fn, R=R, C=C)
-                t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
+                with nvtx.range(f"sweep f={f}"):
+                    t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
                 free_model(mdl)
                 del mdl
             sweep[str(f)] = {"tflops": hdist.job_rate(F, world, t) / 1e12, "speedup_vs_dense": ms_d / t,
@@ -526,7 +530,8 @@ def main():
     dense_model = []
     decode = None
     if not args.no_decode:
-        decode = decode_bench(hsg, stream, peaks)
+        with nvtx.range("decode"):
+            decode = decode_bench(hsg, stream, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
