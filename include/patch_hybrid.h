@@ -320,7 +320,8 @@ void patch_free(patch_handle h);
  * kernel records a timeout in a status word and returns; no fault, trap or
  * hang is involved and the context stays usable. Synchronises `stream`.
  * Returns PATCH_ERR_TIMEOUT when the path behaves as designed, PATCH_OK if the
- * wait unexpectedly completed, PATCH_ERR_CUDA / NOMEM on a runtime failure.
+ * wait unexpectedly completed, PATCH_ERR_CUDA / NOMEM on a runtime failure,
+ * PATCH_ERR_UNSUPPORTED on a device that is not compute capability 10.x.
  * Not part of the product: a check for tests and deployment health probes.
  */
 patch_status patch_selftest_wait(void* stream);
