@@ -363,6 +363,30 @@ def test_config2_llama32_1b_m4096(hsg, oracle_lib):
     _layer(hsg, oracle_lib, shapes, 4096, [c / t for c, t in zip(cnt, T)], tag="cfg2", check_bytes=True)
 
 
+@pytest.mark.parametrize("model,M", [("llama32_1b", 4096), ("llama2_7b", 2048)])
+def test_grouped_layer_as_benchmarked(hsg, oracle_lib, model, M):
+    """The launch the bench times: one layer's seven linears in one grouped
+    launch on the two-strips-per-CTA kernel, sampled rows against the oracle."""
+    shapes = getattr(synth, model)()
+    T = [(l.N // 128) * (l.K // 128) for l in shapes]
+    cnt = synth.split_fraction(T, 0.9, 0.8, 1.0, f"grp-{model}")
+    X_by_k = {K: synth.normal_bf16((M, K), 1.0, "cuda", "grp", "X", 0, M, K) for K in sorted({l.K for l in shapes})}
+    probs = [synth.make_problem(l.N, l.K, 0, n_sparse=c, seed=0, device="cuda", tag=f"grp-{model}-{l.name}")
+             for l, c in zip(shapes, cnt)]
+    lins = [pack(hsg, p) for p in probs]
+    g = hsg.LinearGroup(lins)
+    assert g.path(M) == hsg.PATH_GEMM_WIDE
+    Ys = g([X_by_k[l.K] for l in shapes])
+    torch.cuda.synchronize()
+    lins[0].check()
+    rows = sample_rows(M, 64, 1)
+    for l, p, Y in zip(shapes, probs, Ys):
+        assert_close(Y, oracle_lib, X_by_k[l.K], p.W, p.bits, p.keep, rows=rows, what=f"{model} grouped {l.name}")
+    g.free()
+    for lin in lins:
+        lin.free()
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_config3_llama2_7b_decode(hsg, oracle_lib, M):
     shapes = synth.llama2_7b()
