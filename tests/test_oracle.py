@@ -325,3 +325,36 @@ def test_pack_rejects_bad_mask(oracle_lib):
     keep[3, 0:4] = 1
     with pytest.raises(ValueError):
         oracle_lib.pack(p.W, keep, p.flags.numpy().reshape(-1), 128, 128)
+
+
+# ------------------------------------------------------------ error scale ---
+
+def test_abs_scale_pinned_to_numpy(oracle_lib):
+    """The per-element bound of every parity test is 1e-2 * sum_k |x_k w'_k|,
+    with w' the weight after the mask zeroes the pruned entries ("How to use"
+    on the "llama_3.2_1b-PATCH-45Sparse" card: apply_patch_mask). The oracle's
+    scale is checked against numpy fp64 on a mask unpacked by numpy, for a
+    non-square masked weight and a row subset out of order with a repeat, and
+    exactly on small integers (|x|.|w| sums are exact in fp64 there)."""
+    N, K, M = 256, 448, 37
+    p = synth.make_problem(N, K, M, R=64, C=64, frac=0.6, seed=21, tag="scale")
+    keep = np.unpackbits(p.bits.numpy())[: N * K].reshape(N, K)
+    Wm = oracle_lib.apply_mask(p.W, keep.astype(np.uint8))
+    Wm64 = np.abs(p.W.double().numpy() * keep)
+    X64 = np.abs(p.X.double().numpy())
+    rows = np.array([36, 2, 19, 19, 0, 11])
+    S = oracle_lib.abs_scale(p.X, Wm, rows=rows)
+    ref = X64[rows] @ Wm64.T
+    assert S.shape == (rows.size, N)
+    assert np.allclose(S, ref, rtol=1e-12, atol=0.0)
+    Sf = oracle_lib.abs_scale(p.X, Wm)
+    assert np.allclose(Sf, X64 @ Wm64.T, rtol=1e-12, atol=0.0)
+    # pruned weights contribute nothing: the scale of the unmasked weight differs
+    assert not np.allclose(Sf, X64 @ np.abs(p.W.double().numpy()).T, rtol=1e-6)
+    # small integers: exact
+    rng = np.random.default_rng(9)
+    Xi = rng.integers(-8, 9, size=(5, 24))
+    Wi = rng.integers(-8, 9, size=(3, 24))
+    S2 = oracle_lib.abs_scale(torch.tensor(Xi, dtype=torch.bfloat16), torch.tensor(Wi, dtype=torch.bfloat16),
+                              rows=np.array([4, 1, 4]))
+    assert np.array_equal(S2, (np.abs(Xi[[4, 1, 4]]) @ np.abs(Wi).T).astype(np.float64))
