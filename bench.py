@@ -1,24 +1,33 @@
 """Benchmark of the hybrid dense / 2:4 linear layer (PATCH) on B200.
 
-Default workload: every linear of a Llama-3.2-1B-shaped model (16 layers x
-q, k, v, o, gate, up, down) at M = 4096 tokens, bf16, 128x128 tiles, 90% of
-tiles 2:4 overall (45% sparsity), each linear's 2:4 fraction drawn in
-[0.8, 1.0] and adjusted to the exact global count. One step runs all 112
-linears once on their synthetic inputs; weights and activations are already
-resident in HBM. The step's working set (about 2 GB of packed weights) is far
-larger than L2, so no flush is needed between steps.
+Default workload: every linear of a Llama-2-7B-shaped model (32 layers x q, k,
+v, o, gate, up, down) at M = 2048 tokens, bf16, 128x128 tiles. The headline
+point is 90% of tiles 2:4 overall (45% sparsity), each linear's 2:4 fraction
+drawn in [0.8, 1.0] and adjusted to the exact global count; the sweep repeats
+the step at 2:4 fractions 0 / 0.5 / 0.7 / 0.9 / 1.0 (sparsity 0 / 25 / 35 /
+45 / 50%). One step runs all 224 linears once on their synthetic inputs, one
+grouped launch per layer; weights and activations are already resident in HBM.
+The step's working set (about 9 GB of packed weights) is far larger than L2,
+so no flush is needed between steps.
 
 Reported (one JSON line from rank 0):
   value        dense-equivalent TFLOP/s = 2*M*sum(N*K) / step time, all ranks
   speedup_vs_dense  step time of the same kernel on the all-dense packing of
                the same weights / hybrid step time
-  sweep        the same step at 2:4 fractions 0 / 0.5 / 0.7 / 0.9 / 1.0
-  roofline     tensor-pipe work (2*M*kept weights of each stored slab) per
-               second of the tensor-core kernel, against the measured
-               sustained bf16 peak
+  sweep        the same step at each 2:4 fraction of the sweep
+  roofline     the method's tensor work (2*M per kept weight: a 2:4 tile
+               counts half) per second of the step, whose only launches are
+               the large-M kernel, against the measured bf16 peak (burst for
+               a timed region under 2 s, sustained for longer ones under the
+               power cap)
+  llama2_13b   Llama-2-13B linears at M = 8192, 45% sparsity, for each of the
+               four tile shapes, with its own dense run
+  cublas_bf16  torch.matmul (cuBLAS) on the dense weights of the same shapes,
+               context only (not on the measured path)
   e2e          the same metric through patch_linear_host (host buffers, copies
                inside the timed region)
-  cpu_baseline the CPU oracle on a bounded sample of the same workload
+  cpu_baseline the CPU oracle on a bounded sample of the same workload, on all
+               host cores and on one
   decode       the decode kernel on Llama-2-7B shapes at M = 1, 4, 16 (GB/s)
 
 Multi-GPU (torchrun): every rank runs the whole workload on its own GPU with
@@ -167,13 +176,15 @@ class ClockSampler:
 
 # Model shapes the bench can run: (shape function, default tokens M, default layers).
 WORKLOADS = {
+    "llama2-7b": (synth.llama2_7b, 2048, 32, "Llama-2-7B"),
     "llama32-1b": (synth.llama32_1b, 4096, 16, "Llama-3.2-1B"),
-    "llama2-7b": (synth.llama2_7b, 2048, 8, "Llama-2-7B"),
     "llama2-13b": (synth.llama2_13b, 8192, 2, "Llama-2-13B"),
 }
+DEFAULT_WORKLOAD = "llama2-7b"
+TILES = ["128x128", "128x64", "64x128", "64x64"]
 
 
-def model_linears(n_layers: int, shapes=synth.llama32_1b):
+def model_linears(n_layers: int, shapes=synth.llama2_7b):
     out = []
     for layer in range(n_layers):
         for l in shapes():
@@ -184,14 +195,30 @@ def model_linears(n_layers: int, shapes=synth.llama32_1b):
 ROLE_INPUT = {"q": "attn", "k": "attn", "v": "attn", "o": "o", "gate": "mlp", "up": "mlp", "down": "down"}
 
 
+class Member:
+    """One packed linear of the model with its input and output buffers.
+
+    kept: weights the method multiplies (N*K minus the mask's zeros);
+    executed: weights the tensor-core kernel multiplies (a 2:4 slab whose
+    partner strip's slab is dense runs from its dense image)."""
+
+    def __init__(self, lin, K, N, info, X, Y):
+        self.lin, self.K, self.N, self.X, self.Y = lin, K, N, X, Y
+        self.kept = N * K - int(info.pruned)
+        self.executed = (int(info.slabs_total) - int(info.slabs_pair_sparse)) * 128 * 64 + \
+            int(info.slabs_pair_sparse) * 128 * 32
+        self.packed_bytes = int(info.packed_bytes)
+        self.sparse_area = int(info.tiles_sparse) * int(info.tile_rows) * int(info.tile_cols)
+        self.pair_sparse_area = int(info.slabs_pair_sparse) * 128 * 64
+
+
 def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1.0, rank=0, group=True,
-                shapes=synth.llama32_1b, R=128, C=128):
+                shapes=synth.llama2_7b, R=128, C=128):
     """Packs every linear of the model at global 2:4 fraction `frac`.
 
-    Returns (layers, X, Y, frac): layers is a list of per-layer launch lists;
-    each launch is (callable, [(PackedLinear, K, N, kept_weights, packed_bytes)]).
-    q/k/v read one input, gate/up another, o and down their own; every linear
-    writes its own output."""
+    Returns (layers, X, frac): layers is a list of per-layer launches, each
+    (LinearGroup or None, [Member]). q/k/v read one input, gate/up another,
+    o and down their own; every linear writes its own output."""
     lins = model_linears(n_layers, shapes)
     T = [(l.N // R) * (l.K // C) for _, l in lins]
     if frac in (0.0, 1.0):
@@ -209,76 +236,117 @@ def build_model(hsg, n_layers: int, frac: float, M: int, seed: int, lo=0.8, hi=1
         p = synth.make_problem(l.N, l.K, 0, R=R, C=C, n_sparse=cnt, seed=seed,
                                device="cuda", tag=f"L{layer}-{l.name}")
         lin = hsg.PackedLinear.pack(p.W, p.bits, p.flags.cpu(), R, C)
-        info = lin.info()
-        kept = (info.slabs_total - info.slabs_sparse) * 128 * 64 + info.slabs_sparse * 128 * 32
         Yt = torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda")
-        per_layer.setdefault(layer, []).append((lin, l.K, l.N, kept, info.packed_bytes, X[ROLE_INPUT[l.name]], Yt))
+        per_layer.setdefault(layer, []).append(Member(lin, l.K, l.N, lin.info(), X[ROLE_INPUT[l.name]], Yt))
         del p
     torch.cuda.synchronize()
     layers = []
     for layer in sorted(per_layer):
-        members = per_layer[layer]
+        mem = per_layer[layer]
         if group:
-            g = hsg.LinearGroup([m[0] for m in members])
-            layers.append((g, members))
+            layers.append((hsg.LinearGroup([m.lin for m in mem]), mem))
         else:
-            for m in members:
+            for m in mem:
                 layers.append((None, [m]))
-    return layers, X, None, sum(counts) / sum(T)
+    return layers, X, sum(counts) / sum(T)
 
 
 def free_model(layers):
-    for g, members in layers:
+    for g, mem in layers:
         if g is not None:
             g.free()
-        for m in members:
-            m[0].free()
+        for m in mem:
+            m.lin.free()
 
 
-def run_step(hsg, model, X, Y, stream, path=0, events=None):
-    for i, (g, members) in enumerate(model):
-        if events is not None:
-            events[i][0].record(stream)
+def run_step(hsg, model, stream, path=0):
+    for g, mem in model:
         if g is not None:
-            g([m[5] for m in members], [m[6] for m in members], path=path, stream=stream)
+            g([m.X for m in mem], [m.Y for m in mem], path=path, stream=stream)
         else:
-            m = members[0]
-            hsg.patch_linear_path(m[0].handle, m[5], m[6], path, stream)
-        if events is not None:
-            events[i][1].record(stream)
+            m = mem[0]
+            hsg.patch_linear_path(m.lin.handle, m.X, m.Y, path, stream)
 
 
-def time_steps(hsg, model, X, Y, steps, warmup, stream, dist_on, per_launch=False, path=0):
+def time_steps(hsg, model, steps, warmup, stream, dist_on, path=0):
+    """Mean device time of one step (ms) over `steps` timed steps, max over
+    ranks: CUDA events on the launching stream, a barrier and a device
+    synchronisation on both sides."""
     from hybrid_sparse_gemm_b200 import dist as hdist
     for _ in range(warmup):
-        run_step(hsg, model, X, Y, stream, path)
+        run_step(hsg, model, stream, path)
     torch.cuda.synchronize()
     hdist.barrier(dist_on)
-    ev = None
-    if per_launch:
-        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in model] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     start.record(stream)
-    for s in range(steps):
-        run_step(hsg, model, X, Y, stream, path, events=ev[s] if ev else None)
+    for _ in range(steps):
+        run_step(hsg, model, stream, path)
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
-    ms = hdist.max_over_ranks(ms, dist_on, device="cuda")
-    launch_ms = None
-    if ev:
-        launch_ms = [[a.elapsed_time(b) for a, b in row] for row in ev]
-    return ms / steps, launch_ms
+    hdist.barrier(dist_on)
+    return hdist.max_over_ranks(ms, dist_on, device="cuda") / steps
 
 
 def members(model):
-    return [m for _, ms in model for m in ms]
+    return [m for _, mem in model for m in mem]
 
 
 def flops_dense(model, M):
-    return sum(2.0 * M * m[2] * m[1] for m in members(model))
+    return sum(2.0 * M * m.N * m.K for m in members(model))
+
+
+def flops_kept(model, M):
+    return sum(2.0 * M * m.kept for m in members(model))
+
+
+def flops_executed(model, M):
+    return sum(2.0 * M * m.executed for m in members(model))
+
+
+def choose_peak(peaks, timed_s: float, clocks) -> tuple[float, str]:
+    """Burst bf16 peak for a timed region under 2 s; the sustained one (a
+    seconds-long loop under the power cap) only for longer regions that ran
+    under the power cap."""
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    if timed_s >= 2.0 and capped:
+        return peaks["bf16_tflops_sustained"], f"bf16 sustained ({peaks['source']}): {timed_s:.1f} s under the power cap"
+    return peaks["bf16_tflops"], f"bf16 burst ({peaks['source']}): timed region {timed_s:.2f} s"
+
+
+def roofline(model, M, ms_per_step, launches_per_step, peak, peak_kind, kernel_name, traffic):
+    """The step's launches are all the large-M kernel, back to back, so the
+    kernel's average launch time is the step time over its launches."""
+    algo = flops_kept(model, M)
+    achieved = algo / (ms_per_step / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel_name, "peak_kind": peak_kind,
+            "kernel_ms_per_launch": ms_per_step / launches_per_step,
+            "work": "2*M per kept weight (N*K minus the mask's zeros) of every linear, per launch",
+            "executed_frac": flops_executed(model, M) / (ms_per_step / 1e3) / 1e12 / peak}
+
+
+# ------------------------------------------------------------ CPU oracle ---
+
+def _libgomp():
+    import ctypes
+    try:
+        return ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 class OracleSample:
@@ -286,16 +354,21 @@ class OracleSample:
     linears of one layer. Building the inputs and calibrating the cost model
     happen once; `run(rows)` is one timed sample."""
 
-    def __init__(self, workload: str = "llama32-1b", M: int = 4096, R: int = 128, C: int = 128, seed: int = 0):
+    def __init__(self, workload: str = DEFAULT_WORKLOAD, M: int | None = None, R: int = 128, C: int = 128,
+                 seed: int = 0, threads: int | None = None):
         import oracle
         oracle.build()
         self.oracle = oracle
-        shape_fn, _, _, self.model_name = WORKLOADS[workload]
-        self.M = M
+        shape_fn, default_M, _, self.model_name = WORKLOADS[workload]
+        self.M = M or default_M
         self.shapes = shape_fn()
-        self.probs = [synth.make_problem(l.N, l.K, M, R=R, C=C, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
+        self.probs = [synth.make_problem(l.N, l.K, self.M, R=R, C=C, frac=0.9, seed=seed, tag=f"cpu-{l.name}")
                       for l in self.shapes]
         self.bits = [p.bits.numpy() for p in self.probs]
+        gomp = _libgomp()
+        if gomp is not None and threads:
+            gomp.omp_set_num_threads(int(threads))
+        self.threads = int(gomp.omp_get_max_threads()) if gomp is not None else (os.cpu_count() or 1)
         # calibrate: time 4 and 16 rows of every linear (after one untimed call
         # that starts the thread pool) and fit time = fixed + rows * per_row; the
         # fixed part (mask expansion over the whole weight) does not shrink with rows
@@ -303,10 +376,18 @@ class OracleSample:
         t4, t16 = self.run(4)[1], self.run(16)[1]
         self.per_row = max((t16 - t4) / 12.0, 1e-6)
         self.fixed = max(t4 - 4 * self.per_row, 0.0)
-        self.threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
-    def rows_for(self, budget_s: float, min_rows: int = 1) -> int:
-        return max(min_rows, min(self.M, int((budget_s - self.fixed) / self.per_row)))
+    def set_threads(self, n: int):
+        gomp = _libgomp()
+        if gomp is not None:
+            gomp.omp_set_num_threads(int(n))
+            self.threads = int(gomp.omp_get_max_threads())
+            return True
+        return False
+
+    def rows_for(self, budget_s: float, min_rows: int = 1, per_row: float | None = None) -> int:
+        per_row = per_row or self.per_row
+        return max(min_rows, min(self.M, int((budget_s - self.fixed) / per_row)))
 
     def run(self, rows: int):
         """One pass over the 7 linears on `rows` token rows; returns
@@ -324,14 +405,53 @@ class OracleSample:
                 f"x the 7 {self.model_name} linears of one layer, {t:.1f} s")
 
 
-def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1, workload: str = "llama32-1b",
-               M: int = 4096, R: int = 128, C: int = 128):
-    """One bounded oracle sample of about `budget_s` seconds.
-    Returns (dense-equivalent TFLOP/s, threads, description)."""
+def cpu_sample(budget_s: float = 15.0, seed: int = 0, min_rows: int = 1, workload: str = DEFAULT_WORKLOAD,
+               M: int | None = None, R: int = 128, C: int = 128, one_core_s: float = 0.0):
+    """One bounded oracle sample of about `budget_s` seconds on all host
+    threads, then (if one_core_s > 0) one of about `one_core_s` seconds on one
+    thread. Returns a cpu_baseline dict (value in dense-equivalent TFLOP/s)."""
     s = OracleSample(workload, M, R, C, seed)
     rows = s.rows_for(budget_s, min_rows)
     v, t = s.run(rows)
-    return v, s.threads, s.describe(rows, t)
+    out = {"value": v, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle", "sample": s.describe(rows, t),
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    if one_core_s > 0 and s.set_threads(1):
+        # the per-row cost grows about with the thread count
+        rows1 = s.rows_for(one_core_s, 1, per_row=s.per_row * max(1, out["cores"]))
+        v1, t1 = s.run(rows1)
+        out["value_1core"] = v1
+        out["sample_1core"] = s.describe(rows1, t1) + ", 1 thread"
+    return out
+
+
+# ----------------------------------------------------------- context runs ---
+
+def cublas_bf16(shapes, M: int, stream, layers: int = 4, steps: int = 10):
+    """torch.matmul (cuBLAS) on dense bf16 weights of the same shapes, layers
+    rotated so that the weights stream from HBM. Context only: the measured
+    path never calls it."""
+    Ws = [[synth.normal_bf16((l.N, l.K), 0.02, "cuda", "cublas", L, l.name) for l in shapes()] for L in range(layers)]
+    Xs = {l.K: synth.normal_bf16((M, l.K), 1.0, "cuda", "cublasX", l.K) for l in shapes()}
+    Ys = [torch.empty((M, l.N), dtype=torch.bfloat16, device="cuda") for l in shapes()]
+    with torch.cuda.stream(stream):
+        def step():
+            for W in Ws:
+                for w, y in zip(W, Ys):
+                    torch.matmul(Xs[w.shape[1]], w.t(), out=y)
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            step()
+        e.record(stream)
+        torch.cuda.synchronize()
+    ms_layer = s.elapsed_time(e) / (steps * layers)
+    fl = sum(2.0 * M * l.N * l.K for l in shapes())
+    del Ws, Xs, Ys
+    return {"ms_per_layer": ms_layer, "tflops": fl / (ms_layer / 1e3) / 1e12, "layers_rotated": layers,
+            "note": "context only: torch.matmul (cuBLAS) on dense bf16 weights, not on the measured path"}
 
 
 def decode_bench(hsg, stream, peaks, steps=20):
@@ -385,22 +505,58 @@ def decode_bench(hsg, stream, peaks, steps=20):
     return out
 
 
+def kernel_label(hsg, model, M, gpath):
+    g = model[0][0]
+    p = g.path(M, gpath) if g is not None else hsg.PATH_GEMM_PAIR
+    return KERNEL_NAMES.get(p, "tensor-core GEMM")
+
+
+def llama2_13b_tiles(hsg, stream, peaks, steps, warmup, dist_on, rank, gpath, tiles=TILES, layers=2):
+    """Llama-2-13B linears at M = 8192, 90% 2:4 tiles (45% sparsity), for each
+    tile shape, each against the all-dense packing of the same shapes."""
+    M = 8192
+    with torch.cuda.stream(stream):
+        dense, _, _ = build_model(hsg, layers, 0.0, M, seed=1, rank=rank, shapes=synth.llama2_13b)
+    ms_d = time_steps(hsg, dense, steps, warmup, stream, dist_on, gpath)
+    free_model(dense)
+    del dense
+    out = {"workload": f"Llama-2-13B linears ({layers} layers x q,k,v,o,gate,up,down), M={M} tokens, bf16, "
+                       "90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]",
+           "dense_ms_per_step": ms_d}
+    for tile in tiles:
+        R, C = (int(v) for v in tile.split("x"))
+        with torch.cuda.stream(stream):
+            mdl, _, frac = build_model(hsg, layers, 0.9, M, seed=1, rank=rank, shapes=synth.llama2_13b, R=R, C=C)
+        ms = time_steps(hsg, mdl, steps, warmup, stream, dist_on, gpath)
+        F = flops_dense(mdl, M)
+        algo = flops_kept(mdl, M) / (ms / 1e3) / 1e12
+        mem = members(mdl)
+        out[tile] = {"tflops": F / (ms / 1e3) / 1e12, "speedup_vs_dense": ms_d / ms, "ms_per_step": ms,
+                     "frac_2to4": frac, "roofline_frac": algo / peaks["bf16_tflops"],
+                     "sparse_area_run_sparse": sum(m.pair_sparse_area for m in mem) /
+                     max(1, sum(m.sparse_area for m in mem))}
+        free_model(mdl)
+        del mdl
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama32-1b", choices=sorted(WORKLOADS),
-                    help="model whose linears one step runs (default: Llama-3.2-1B, M = 4096)")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS),
+                    help="model whose linears one step runs (default: Llama-2-7B, 32 layers, M = 2048)")
     ap.add_argument("--layers", type=int, default=None, help="layers per step (default per workload)")
     ap.add_argument("--M", type=int, default=None, help="tokens (default per workload)")
-    ap.add_argument("--tile", default="128x128", choices=["128x128", "128x64", "64x128", "64x64"],
-                    help="mask tile shape")
+    ap.add_argument("--tile", default="128x128", choices=TILES, help="mask tile shape")
     ap.add_argument("--no-group", action="store_true", help="one launch per linear instead of per layer")
     ap.add_argument("--path", default="auto", choices=["auto", "pair", "wide"],
                     help="tensor-core kernel for the timed steps (auto: the library's choice)")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-13b", action="store_true", help="skip the Llama-2-13B tile-shape runs")
+    ap.add_argument("--no-cublas", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -416,7 +572,8 @@ def main():
         args.layers = default_layers
     R, C = (int(v) for v in args.tile.split("x"))
     workload = (f"{model_name} linears ({args.layers} layers x q,k,v,o,gate,up,down), M={args.M} tokens, "
-                f"bf16, {R}x{C} tiles, 90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]")
+                f"bf16, {R}x{C} tiles, 90% 2:4 tiles (45% sparsity), per-linear fraction in [0.8,1.0]; "
+                f"sweep over 2:4 fractions {'/'.join(str(f) for f in FRACS_SWEEP)}")
 
     if args.impl == "reference":
         if rank != 0:
@@ -442,7 +599,7 @@ def main():
                                             "tile": args.tile, "path": "cpu oracle",
                                             "sample": "token rows of one layer per step"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "cpu_model": cpu_model()},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
         return
 
@@ -456,31 +613,27 @@ def main():
     gpath = {"auto": hsg.PATH_AUTO, "pair": hsg.PATH_GEMM_PAIR, "wide": hsg.PATH_GEMM_WIDE}[args.path]
     M = args.M
     group = not args.no_group
+    nvtx = torch.cuda.nvtx  # phase markers for profilers; nothing inside the timed loops
 
     with torch.cuda.stream(stream):
-        model, X, _, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank, group=group,
-                                             shapes=shape_fn, R=R, C=C)
-        dense_model, _, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank, group=group,
-                                           shapes=shape_fn, R=R, C=C)
+        model, X, frac_real = build_model(hsg, args.layers, 0.9, M, seed=0, rank=rank, group=group,
+                                          shapes=shape_fn, R=R, C=C)
+        dense_model, _, _ = build_model(hsg, args.layers, 0.0, M, seed=0, rank=rank, group=group,
+                                        shapes=shape_fn, R=R, C=C)
     torch.cuda.synchronize()
     F = flops_dense(model, M)
-    exec_flops = sum(2.0 * M * m[3] for m in members(model))
     n_launch = len(model)
 
-    nvtx = torch.cuda.nvtx  # phase markers for profilers; nothing inside the timed loops
     with ClockSampler(torch.cuda.current_device()) as clk, nvtx.range("hybrid steps"):
-        ms_h, _ = time_steps(hsg, model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
+        ms_h = time_steps(hsg, model, args.steps, args.warmup, stream, dist_on, path=gpath)
     clocks = clk.summary()
     with nvtx.range("dense steps"):
-        ms_d, _ = time_steps(hsg, dense_model, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
-    # per-launch durations for the roofline (separate pass, events around each launch)
-    with nvtx.range("per-launch timing"):
-        _, launch_ms = time_steps(hsg, model, X, None, max(2, args.steps // 4), 1, stream, dist_on,
-                                  per_launch=True, path=gpath)
-    kern_ms = statistics.mean(sum(row) for row in launch_ms)
-    kernel_name = KERNEL_NAMES.get(model[0][0].path(M, gpath) if model[0][0] is not None else hsg.PATH_GEMM_PAIR,
-                                   "tensor-core GEMM")
-    achieved = exec_flops / (kern_ms / 1e3) / 1e12
+        ms_d = time_steps(hsg, dense_model, args.steps, args.warmup, stream, dist_on, path=gpath)
+    kernel_name = kernel_label(hsg, model, M, gpath)
+    peak, peak_kind = choose_peak(peaks, ms_h * args.steps / 1e3, clocks)
+    roof = roofline(model, M, ms_h, n_launch, peak, peak_kind, kernel_name,
+                    measured_traffic(kernel_name, (args.workload, M, args.tile)))
+    roof["sm_mhz"] = clocks.get("sm_mhz")
     value = hdist.job_rate(F, world, ms_h) / 1e12
 
     sweep = None
@@ -488,46 +641,65 @@ def main():
         sweep = {}
         for f in FRACS_SWEEP:
             if f == 0.0:
-                t = ms_d
+                t, mdl = ms_d, dense_model
             elif f == 0.9:
-                t = ms_h
+                t, mdl = ms_h, model
             else:
                 with torch.cuda.stream(stream):
-                    mdl, _, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group,
-                                               shapes=shape_fn, R=R, C=C)
+                    mdl, _, _ = build_model(hsg, args.layers, f, M, seed=0, rank=rank, group=group,
+                                            shapes=shape_fn, R=R, C=C)
                 with nvtx.range(f"sweep f={f}"):
-                    t, _ = time_steps(hsg, mdl, X, None, args.steps, args.warmup, stream, dist_on, path=gpath)
+                    t = time_steps(hsg, mdl, args.steps, args.warmup, stream, dist_on, path=gpath)
+            sweep[str(f)] = {"tflops": hdist.job_rate(F, world, t) / 1e12, "speedup_vs_dense": ms_d / t,
+                             "ms_per_step": t, "sparsity": 0.5 * f,
+                             "roofline_frac": flops_kept(mdl, M) / (t / 1e3) / 1e12 / peak}
+            if f not in (0.0, 0.9):
                 free_model(mdl)
                 del mdl
-            sweep[str(f)] = {"tflops": hdist.job_rate(F, world, t) / 1e12, "speedup_vs_dense": ms_d / t,
-                             "ms_per_step": t}
+    free_model(dense_model)
+    dense_model = []
 
     e2e = None
     if not args.no_e2e:
         mem = members(model)
-        Xh = {id(m[5]): m[5].cpu().pin_memory() for m in mem}
-        Yh = [torch.empty(m[6].shape, dtype=torch.bfloat16).pin_memory() for m in mem]
-        h2d = sum(M * m[1] * 2 for m in mem)
-        d2h = sum(M * m[2] * 2 for m in mem)
+        Xh = {id(m.X): m.X.cpu().pin_memory() for m in mem}
+        Yh = [torch.empty(m.Y.shape, dtype=torch.bfloat16).pin_memory() for m in mem]
+        h2d = sum(M * m.K * 2 for m in mem)
+        d2h = sum(M * m.N * 2 for m in mem)
         e2e_steps = max(1, min(args.steps, 3))
         for m, yh in zip(mem, Yh):  # warm-up
-            hsg.patch_linear_host(m[0].handle, Xh[id(m[5])], yh, stream)
+            hsg.patch_linear_host(m.lin.handle, Xh[id(m.X)], yh, stream)
         hdist.barrier(dist_on)
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         s.record(stream)
         for _ in range(e2e_steps):
             for m, yh in zip(mem, Yh):
-                hsg.patch_linear_host(m[0].handle, Xh[id(m[5])], yh, stream)
+                hsg.patch_linear_host(m.lin.handle, Xh[id(m.X)], yh, stream)
         e.record(stream)
         torch.cuda.synchronize()
         ms_e = s.elapsed_time(e) / e2e_steps
         ms_e = hdist.max_over_ranks(ms_e, dist_on, device="cuda")
         e2e = {"value": hdist.job_rate(F, world, ms_e) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
+        del Xh, Yh
 
-    free_model(dense_model)
-    dense_model = []
+    packed_gb = sum(m.packed_bytes for m in members(model)) / 1e9
+    linears = len(members(model))
+    free_model(model)
+    model = []
+
+    big = None
+    if args.workload == DEFAULT_WORKLOAD and not args.no_13b:
+        with nvtx.range("llama2-13b tiles"):
+            big = llama2_13b_tiles(hsg, stream, peaks, args.steps, args.warmup, dist_on, rank, gpath)
+
+    cublas = None
+    if rank == 0 and not args.no_cublas:
+        with nvtx.range("cublas context"):
+            cublas = cublas_bf16(shape_fn, M, stream)
+            cublas["same_step_ms"] = cublas["ms_per_layer"] * args.layers
+
     decode = None
     if not args.no_decode:
         with nvtx.range("decode"):
@@ -535,34 +707,27 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, threads, desc = cpu_sample(workload=args.workload, M=args.M, R=R, C=C)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = cpu_sample(workload=args.workload, M=args.M, R=R, C=C, one_core_s=8.0)
 
     if rank == 0:
-        packed_gb = sum(m[4] for m in members(model)) / 1e9
         line = {
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_h, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload, "M": M, "layers": args.layers, "linears": len(members(model)),
+            "config": {"workload": workload, "M": M, "layers": args.layers, "linears": linears,
                        "launches_per_step": n_launch, "grouped": group,
                        "frac_2to4": frac_real, "tile": args.tile,
                        "l2": "inputs larger than L2 (%.2f GB of packed weights per step)" % packed_gb,
                        "parallelism": f"dp{world} (M split, replicated weights)", "path": args.path},
             "speedup_vs_dense": ms_d / ms_h, "dense_ms_per_step": ms_d,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
-                         "traffic": measured_traffic(kernel_name, (args.workload, M, args.tile)),
-                         "kernel": kernel_name,
-                         "work": "2*M per kept weight of every loaded slab (a 2:4 slab counts half)",
-                         "peak_kind": f"bf16 sustained ({peaks['source']})"},
+            "roofline": roof,
             "gpu_launches": n_launch * args.steps,
             "clocks": clocks,
-            "sweep": sweep, "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
+            "sweep": sweep, "llama2_13b": big, "cublas_bf16": cublas,
+            "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
         }
         print(json.dumps(line))
-    free_model(model)
     hdist.shutdown(dist_on)
 
 

@@ -34,7 +34,7 @@ EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_hos
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
             "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
             "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait",
-            "patch_partition_rows", "patch_classify_tiles"]
+            "patch_partition_rows", "patch_classify_tiles", "patch_group_linear_host"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -57,6 +57,7 @@ _lib.patch_linear_host.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_linear_noalloc.argtypes = [_P, _P, _I64, _P, _P]
 _lib.patch_group_create.argtypes = [_P, _I, ctypes.POINTER(_P)]
 _lib.patch_group_linear.argtypes = [_P, _P, _I64, _P, _I, _P]
+_lib.patch_group_linear_host.argtypes = [_P, _P, _I64, _P, _I, _P]
 _lib.patch_group_path.argtypes = [_P, _I64, _I, ctypes.POINTER(_I)]
 _lib.patch_group_free.argtypes = [_P]
 _lib.patch_selftest_wait.argtypes = [_P]
@@ -74,7 +75,8 @@ _lib.patch_last_error.restype = ctypes.c_char_p
 _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
            "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc",
-           "patch_group_create", "patch_group_linear", "patch_partition_rows", "patch_classify_tiles"]:
+           "patch_group_create", "patch_group_linear", "patch_partition_rows", "patch_classify_tiles",
+           "patch_group_linear_host"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -236,6 +238,22 @@ class LinearGroup:
         xs = (_P * n)(*[x.data_ptr() for x in Xs])
         ys = (_P * n)(*[y.data_ptr() for y in outs])
         _check(_lib.patch_group_linear(self.handle, xs, M, ys, path, _stream(stream)))
+        return outs
+
+    def host(self, Xs, outs=None, path: int = PATH_AUTO, stream=None, sync: bool = True):
+        """Host tensors in and out (pinned for overlapped copies). With
+        sync=False the call only enqueues: the outputs are complete once
+        `stream` is."""
+        n = len(self.linears)
+        assert len(Xs) == n and all(not x.is_cuda for x in Xs)
+        M = Xs[0].shape[0]
+        if outs is None:
+            outs = [torch.empty((M, l.N), dtype=torch.bfloat16, pin_memory=True) for l in self.linears]
+        xs = (_P * n)(*[x.data_ptr() for x in Xs])
+        ys = (_P * n)(*[y.data_ptr() for y in outs])
+        _check(_lib.patch_group_linear_host(self.handle, xs, M, ys, path, _stream(stream)))
+        if sync:
+            torch.cuda.synchronize()
         return outs
 
     def path(self, M: int, path: int = PATH_AUTO) -> int:

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -14,6 +15,7 @@
 #include <mutex>
 #include <queue>
 #include <string>
+#include <thread>
 #include <vector>
 
 #include "kernels.cuh"
@@ -139,6 +141,19 @@ struct WorkList {
     int grid = 0;         // CTAs (single, decode) or CTA pairs (pair kernel)
     int* off = nullptr;   // device, grid + 1
     int* work = nullptr;  // device, units
+    int* host = nullptr;  // pinned host copy the upload reads from (kept until the group is freed)
+    cudaEvent_t ready = nullptr;      // recorded after the upload on the stream that built it
+    cudaStream_t made_on = nullptr;
+    std::atomic<bool> done{false};    // the upload is known to have completed
+};
+
+// Split-K workspace of the decode kernel for one group and one stream: per
+// member, partial sums [S][P][128][16] fp32 (NULL when P == 1) and per-strip
+// arrival counters that the kernel re-arms to zero.
+struct DecodeWs {
+    float* partial[kMaxGroup] = {};
+    unsigned* counters[kMaxGroup] = {};
+    int S[kMaxGroup] = {};
 };
 
 // Host copy of the three tables and the derived per-strip costs.
@@ -251,10 +266,10 @@ struct patch_handle_s {
     uint32_t* gemm_dev = nullptr;
     int* status_dev = nullptr;
     int decode_parts = 1;                 // K-parts per strip for the decode kernel
-    float* decode_partial = nullptr;      // [S][parts][128][16] fp32 workspace
-    unsigned* decode_counters = nullptr;  // [S], zero between calls
     LinDesc desc{};                       // host copy of the device descriptor
-    CUtensorMap tm_a16, tm_a8, tm_e;
+    std::mutex groups_mu;
+    std::vector<patch_group_s*> groups;   // groups this handle belongs to (its own one-member group too)
+    CUtensorMap tm_a32, tm_a16, tm_a8, tm_e;
     patch_info_t info{};
     patch_group_s* self = nullptr;        // one-member group used by patch_linear
     std::mutex mu;
@@ -273,20 +288,82 @@ struct patch_group_s {
     LinDesc* lins_dev = nullptr;  // n descriptors
     int* status_dev = nullptr;    // the first member's status word
     std::mutex mu;
+    std::mutex host_mu;           // serialises patch_group_linear_host calls on the host
     std::map<std::pair<int, int>, WorkList> work;  // (kernel, m_blocks or 0) -> schedule
+    // decode workspaces: one per stream that issued an uncaptured decode call
+    // (per thread for the per-thread default stream), and one that every
+    // captured call bakes into its graph
+    std::map<std::pair<cudaStream_t, size_t>, DecodeWs> decode_ws;
+    DecodeWs capture_ws;
+    // patch_group_linear_host: device staging (one X buffer per distinct
+    // host input, one Y buffer per member), two copy streams, chunk events
+    void* stage_x[kMaxGroup] = {};
+    size_t stage_x_bytes[kMaxGroup] = {};
+    void* stage_y[kMaxGroup] = {};
+    size_t stage_y_bytes[kMaxGroup] = {};
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t last_done = nullptr;      // the previous host call's last copy back
+    std::vector<cudaEvent_t> chunk_ev;    // 2 per chunk: inputs landed, outputs computed
 };
 
 namespace {
 
+void free_ws(DecodeWs& w) {
+    for (int i = 0; i < kMaxGroup; ++i) {
+        cudaFree(w.partial[i]);
+        cudaFree(w.counters[i]);
+        w.partial[i] = nullptr;
+        w.counters[i] = nullptr;
+    }
+}
+
 void free_group(patch_group g) {
     if (!g) return;
     cudaDeviceSynchronize();
+    for (int i = 0; i < g->n; ++i) {
+        if (!g->h[i]) continue;
+        std::lock_guard<std::mutex> lk(g->h[i]->groups_mu);
+        auto& v = g->h[i]->groups;
+        v.erase(std::remove(v.begin(), v.end(), g), v.end());
+    }
     cudaFree(g->lins_dev);
     for (auto& kv : g->work) {
         cudaFree(kv.second.off);
         cudaFree(kv.second.work);
+        cudaFreeHost(kv.second.host);
+        if (kv.second.ready) cudaEventDestroy(kv.second.ready);
     }
+    for (auto& kv : g->decode_ws) free_ws(kv.second);
+    free_ws(g->capture_ws);
+    for (int i = 0; i < kMaxGroup; ++i) {
+        cudaFree(g->stage_x[i]);
+        cudaFree(g->stage_y[i]);
+    }
+    if (g->h2d) cudaStreamDestroy(g->h2d);
+    if (g->d2h) cudaStreamDestroy(g->d2h);
+    if (g->last_done) cudaEventDestroy(g->last_done);
+    for (cudaEvent_t e : g->chunk_ev) cudaEventDestroy(e);
     delete g;
+}
+
+// Allocates a decode workspace for every member of g; counters zeroed on st.
+patch_status alloc_ws(patch_group g, DecodeWs* w, cudaStream_t st) {
+    for (int i = 0; i < g->n; ++i) {
+        const int S = g->h[i]->plan.S, P = g->parts[i];
+        w->S[i] = S;
+        if ((P > 1 && cudaMalloc(&w->partial[i], sizeof(float) * (size_t)S * P * 128 * kDecodeBN) != cudaSuccess) ||
+            cudaMalloc(&w->counters[i], sizeof(unsigned) * S) != cudaSuccess) {
+            cudaGetLastError();
+            free_ws(*w);
+            return fail(PATCH_ERR_NOMEM, "decode workspace allocation failed");
+        }
+        cudaError_t e = cudaMemsetAsync(w->counters[i], 0, sizeof(unsigned) * S, st);
+        if (e != cudaSuccess) {
+            free_ws(*w);
+            return cuda_fail(e, "decode workspace set-up");
+        }
+    }
+    return PATCH_OK;
 }
 
 void free_handle(patch_handle h) {
@@ -298,8 +375,6 @@ void free_handle(patch_handle h) {
     cudaFree(h->meta_dev);
     cudaFree(h->gemm_dev);
     cudaFree(h->status_dev);
-    cudaFree(h->decode_partial);
-    cudaFree(h->decode_counters);
     cudaFree(h->stage_x);
     cudaFree(h->stage_y);
     delete h;
@@ -344,7 +419,43 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
         delete g;
         return fail(PATCH_ERR_CUDA, "group descriptor upload failed");
     }
+    patch_status st = alloc_ws(g, &g->capture_ws, nullptr);
+    if (st == PATCH_OK && cudaDeviceSynchronize() != cudaSuccess) st = fail(PATCH_ERR_CUDA, "decode workspace set-up");
+    if (st != PATCH_OK) {
+        cudaFree(g->lins_dev);
+        delete g;
+        return st;
+    }
+    for (int i = 0; i < n; ++i) {
+        std::lock_guard<std::mutex> lk(hs[i]->groups_mu);
+        hs[i]->groups.push_back(g);
+    }
     *out = g;
+    return PATCH_OK;
+}
+
+// The decode workspace a call on `st` uses: the capture workspace when the
+// stream is capturing a graph, else the stream's own (allocated on its first
+// decode call; for the per-thread default stream, one per thread).
+patch_status get_decode_ws(patch_group g, cudaStream_t st, const DecodeWs** out) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cs != cudaStreamCaptureStatusNone) {
+        *out = &g->capture_ws;
+        return PATCH_OK;
+    }
+    const size_t tid = st == cudaStreamPerThread ? std::hash<std::thread::id>()(std::this_thread::get_id()) : 0;
+    const auto key = std::make_pair(st, tid);
+    std::lock_guard<std::mutex> lk(g->mu);
+    auto it = g->decode_ws.find(key);
+    if (it == g->decode_ws.end()) {
+        DecodeWs w;
+        patch_status s = alloc_ws(g, &w, st);
+        if (s != PATCH_OK) return s;
+        it = g->decode_ws.emplace(key, w).first;
+    }
+    *out = &it->second;
     return PATCH_OK;
 }
 
@@ -418,28 +529,79 @@ void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std:
     off[grid] = (int)work.size();
 }
 
-patch_status get_worklist(patch_group g, int kernel, int mb, WorkList** out) {
-    std::lock_guard<std::mutex> lk(g->mu);
-    auto key = std::make_pair(kernel, mb);
-    auto it = g->work.find(key);
-    if (it != g->work.end()) {
-        *out = &it->second;
-        return PATCH_OK;
+// The cached schedule of (kernel, mb). The first call for a key builds it and
+// uploads it asynchronously on `st` from a pinned host copy; a call on another
+// stream waits for that upload through an event until it is known complete.
+patch_status get_worklist(patch_group g, int kernel, int mb, cudaStream_t st, WorkList** out) {
+    WorkList* wl = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g->mu);
+        auto key = std::make_pair(kernel, mb);
+        auto it = g->work.find(key);
+        if (it == g->work.end()) {
+            std::vector<int> off, work;
+            lpt_schedule(g, kernel, mb, off, work);
+            const size_t n_off = off.size(), n_work = std::max<size_t>(work.size(), 1);
+            int *d_off = nullptr, *d_work = nullptr, *host = nullptr;
+            cudaEvent_t ev = nullptr;
+            if (cudaMalloc(&d_off, sizeof(int) * n_off) != cudaSuccess ||
+                cudaMalloc(&d_work, sizeof(int) * n_work) != cudaSuccess ||
+                cudaHostAlloc(&host, sizeof(int) * (n_off + n_work), cudaHostAllocDefault) != cudaSuccess ||
+                cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+                cudaGetLastError();
+                cudaFree(d_off);
+                cudaFree(d_work);
+                cudaFreeHost(host);
+                return fail(PATCH_ERR_NOMEM, "schedule allocation failed");
+            }
+            std::copy(off.begin(), off.end(), host);
+            std::copy(work.begin(), work.end(), host + n_off);
+            cudaError_t e = cudaMemcpyAsync(d_off, host, sizeof(int) * n_off, cudaMemcpyHostToDevice, st);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(d_work, host + n_off, sizeof(int) * work.size(), cudaMemcpyHostToDevice, st);
+            if (e == cudaSuccess) e = cudaEventRecord(ev, st);
+            it = g->work.emplace(std::piecewise_construct, std::forward_as_tuple(key), std::forward_as_tuple()).first;
+            WorkList& w = it->second;
+            w.grid = (int)n_off - 1;
+            w.off = d_off;
+            w.work = d_work;
+            w.host = host;
+            w.ready = ev;
+            w.made_on = st;
+            if (e != cudaSuccess) {
+                // keep nothing half-built: later calls must rebuild it
+                cudaStreamSynchronize(st);
+                cudaFree(d_off);
+                cudaFree(d_work);
+                cudaFreeHost(host);
+                cudaEventDestroy(ev);
+                g->work.erase(it);
+                return cuda_fail(e, "schedule upload");
+            }
+            *out = &w;
+            return PATCH_OK;
+        }
+        wl = &it->second;
     }
-    std::vector<int> off, work;
-    lpt_schedule(g, kernel, mb, off, work);
-    WorkList wl;
-    wl.grid = (int)off.size() - 1;
-    if (cudaMalloc(&wl.off, sizeof(int) * off.size()) != cudaSuccess ||
-        cudaMalloc(&wl.work, sizeof(int) * std::max<size_t>(work.size(), 1)) != cudaSuccess) {
-        cudaFree(wl.off);
-        cudaGetLastError();
-        return fail(PATCH_ERR_NOMEM, "schedule allocation failed");
+    if (!wl->done.load(std::memory_order_acquire) && st != wl->made_on) {
+        // a stream that is capturing a graph makes no event call: the first
+        // call for this M has completed before capture (documented rule)
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        PATCH_CUDA(cudaStreamIsCapturing(st, &cs));
+        if (cs != cudaStreamCaptureStatusNone) {
+            *out = wl;
+            return PATCH_OK;
+        }
+        const cudaError_t q = cudaEventQuery(wl->ready);
+        if (q == cudaSuccess) {
+            wl->done.store(true, std::memory_order_release);
+        } else if (q == cudaErrorNotReady) {
+            PATCH_CUDA(cudaStreamWaitEvent(st, wl->ready, 0));
+        } else {
+            return cuda_fail(q, "schedule upload");
+        }
     }
-    PATCH_CUDA(cudaMemcpy(wl.off, off.data(), sizeof(int) * off.size(), cudaMemcpyHostToDevice));
-    PATCH_CUDA(cudaMemcpy(wl.work, work.data(), sizeof(int) * work.size(), cudaMemcpyHostToDevice));
-    auto res = g->work.emplace(key, wl);
-    *out = &res.first->second;
+    *out = wl;
     return PATCH_OK;
 }
 
@@ -523,6 +685,7 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
         patch_handle h = g->h[l];
         patch_status s = encode_2d(&maps.x[l], X[l], h->K, M, kSlabK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
         if (s != PATCH_OK) return s;
+        maps.a32[l] = h->tm_a32;
         maps.a16[l] = h->tm_a16;
         maps.a8[l] = h->tm_a8;
         maps.e[l] = h->tm_e;
@@ -531,11 +694,20 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
     int grid = sched_grid;
     if (!sched_off) {
         WorkList* wl = nullptr;
-        patch_status s = get_worklist(g, kernel, mb, &wl);
+        patch_status s = get_worklist(g, kernel, mb, st, &wl);
         if (s != PATCH_OK) return s;
         sched_off = wl->off;
         sched_work = wl->work;
         grid = wl->grid;
+    }
+    if (kernel == 2) {
+        const DecodeWs* ws = nullptr;
+        patch_status s = get_decode_ws(g, st, &ws);
+        if (s != PATCH_OK) return s;
+        for (int l = 0; l < g->n; ++l) {
+            a.partial[l] = ws->partial[l];
+            a.counters[l] = ws->counters[l];
+        }
     }
     a.lins = g->lins_dev;
     a.work_off = sched_off;
@@ -722,18 +894,17 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
         cudaMalloc(&h->meta_dev, sizeof(uint32_t) * p.meta.size()) != cudaSuccess ||
         cudaMalloc(&h->gemm_dev, sizeof(uint32_t) * p.gemm.size()) != cudaSuccess ||
         cudaMalloc(&h->status_dev, sizeof(int)) != cudaSuccess ||
-        cudaMalloc(&h->decode_partial, sizeof(float) * (size_t)p.S * h->decode_parts * 128 * kDecodeBN) !=
-            cudaSuccess ||
-        cudaMalloc(&h->decode_counters, sizeof(unsigned) * p.S) != cudaSuccess ||
         cudaMalloc(&flags_dev, ntiles) != cudaSuccess ||
         cudaMalloc(&counters, 3 * sizeof(unsigned long long)) != cudaSuccess) {
         cudaGetLastError();
         return cleanup(fail(PATCH_ERR_NOMEM, "device allocation of %lld packed bytes failed", (long long)p.bytes));
     }
     // tensor maps of the packed bytes viewed as rows of 64 bf16 (128 bytes):
-    // dense slab / dense image (128 rows), 2:4 values (64 rows), metadata (16 rows)
+    // two adjacent dense records (256 rows), a dense slab / dense image or two
+    // adjacent 2:4 records (128 rows), 2:4 values (64 rows), metadata (16 rows)
     const int64_t rows = std::max<int64_t>(p.bytes, 2048) / 128;
-    if ((st = encode_2d(&h->tm_a16, h->packed, 64, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
+    if ((st = encode_2d(&h->tm_a32, h->packed, 64, rows, 64, 256, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
+        (st = encode_2d(&h->tm_a16, h->packed, 64, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
         (st = encode_2d(&h->tm_a8, h->packed, 64, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK ||
         (st = encode_2d(&h->tm_e, h->packed, 64, rows, 64, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != PATCH_OK)
         return cleanup(st);
@@ -746,8 +917,7 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(flags_dev, tile_flags, ntiles, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
         (e = cudaMemsetAsync(counters, 0, 3 * sizeof(unsigned long long), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(h->decode_counters, 0, sizeof(unsigned) * p.S, s)) != cudaSuccess)
+        (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess)
         return cleanup(cuda_fail(e, "pack set-up copies"));
     PackArgs a;
     a.W = static_cast<const uint16_t*>(W_bf16);
@@ -776,8 +946,6 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     h->desc.slab = h->slab_dev;
     h->desc.meta = h->meta_dev;
     h->desc.gemm = h->gemm_dev;
-    h->desc.partial = h->decode_partial;
-    h->desc.counters = h->decode_counters;
     h->desc.N = (int)N;
     h->desc.S = p.S;
     h->desc.KB = p.KB;
@@ -902,6 +1070,117 @@ patch_status patch_group_path(patch_group g, int64_t M, int path, int* out) {
 
 void patch_group_free(patch_group g) { free_group(g); }
 
+patch_status patch_group_linear_host(patch_group g, const void* const* X_host, int64_t M, void* const* Y_host,
+                                     int path, void* stream) {
+    if (!g) return fail(PATCH_ERR_ARG, "group is NULL");
+    if (!X_host || !Y_host) return fail(PATCH_ERR_ARG, "X and Y arrays must be non-NULL");
+    if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    for (int l = 0; l < g->n; ++l)
+        if (!X_host[l] || !Y_host[l]) return fail(PATCH_ERR_ARG, "member %d: X and Y must be non-NULL", l);
+    if (M == 0) return PATCH_OK;
+    if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
+    patch_status st = check_device_is(g->device);
+    if (st != PATCH_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lk(g->host_mu);
+
+    // distinct inputs (q, k, v read one X): slot of each member
+    int slot[kMaxGroup], nslots = 0;
+    const void* src[kMaxGroup];
+    int64_t slotK[kMaxGroup];
+    for (int l = 0; l < g->n; ++l) {
+        int f = -1;
+        for (int i = 0; i < nslots; ++i)
+            if (src[i] == X_host[l] && slotK[i] == g->h[l]->K) f = i;
+        if (f < 0) {
+            f = nslots++;
+            src[f] = X_host[l];
+            slotK[f] = g->h[l]->K;
+        }
+        slot[l] = f;
+    }
+    auto grow = [&](void** buf, size_t* have, size_t need) {
+        if (need <= *have) return true;
+        cudaFree(*buf);
+        *buf = nullptr;
+        *have = 0;
+        if (cudaMalloc(buf, need) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        *have = need;
+        return true;
+    };
+    if (!g->h2d) {
+        if (cudaStreamCreateWithFlags(&g->h2d, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&g->d2h, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&g->last_done, cudaEventDisableTiming) != cudaSuccess)
+            return fail(PATCH_ERR_CUDA, "copy stream set-up failed");
+        PATCH_CUDA(cudaEventRecord(g->last_done, g->d2h));
+    }
+    // The previous host call on this group must be done with the staging
+    // buffers before they are regrown or overwritten.
+    bool regrow = false;
+    for (int i = 0; i < nslots; ++i) regrow = regrow || (size_t)M * slotK[i] * 2 > g->stage_x_bytes[i];
+    for (int l = 0; l < g->n; ++l) regrow = regrow || (size_t)M * g->h[l]->N * 2 > g->stage_y_bytes[l];
+    if (regrow) PATCH_CUDA(cudaEventSynchronize(g->last_done));
+    for (int i = 0; i < nslots; ++i)
+        if (!grow(&g->stage_x[i], &g->stage_x_bytes[i], (size_t)M * slotK[i] * 2))
+            return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+    for (int l = 0; l < g->n; ++l)
+        if (!grow(&g->stage_y[l], &g->stage_y_bytes[l], (size_t)M * g->h[l]->N * 2))
+            return fail(PATCH_ERR_NOMEM, "staging allocation failed");
+
+    // Token chunks: chunk c's inputs land while chunk c-1 computes and chunk
+    // c-2's outputs go back (the two copy directions use separate engines).
+    // Every chunk runs the kernel a device call with this M would run, and
+    // chunks are whole multiples of its token tile, so each output element
+    // comes from the same MMA sequence: the bits equal patch_group_linear's.
+    const int rpath = resolve_path(g, path, M);
+    const int64_t bn = rpath == PATCH_PATH_GEMM_WIDE   ? kGemm22BN
+                       : rpath == PATCH_PATH_GEMM_PAIR ? kGemm2BN
+                       : rpath == PATCH_PATH_GEMM_SINGLE ? kGemmBN
+                                                         : M;
+    int64_t chunk = M;
+    if (M >= 4 * bn) chunk = ((M + 3) / 4 + bn - 1) / bn * bn;
+    const int nchunks = (int)((M + chunk - 1) / chunk);
+    while ((int)g->chunk_ev.size() < 2 * nchunks) {
+        cudaEvent_t e = nullptr;
+        PATCH_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        g->chunk_ev.push_back(e);
+    }
+    PATCH_CUDA(cudaStreamWaitEvent(g->h2d, g->last_done, 0));
+    PATCH_CUDA(cudaStreamWaitEvent(s, g->last_done, 0));
+    for (int c = 0; c < nchunks; ++c) {
+        const int64_t m0 = c * chunk, rows = std::min<int64_t>(chunk, M - m0);
+        cudaEvent_t x_ready = g->chunk_ev[2 * c], y_ready = g->chunk_ev[2 * c + 1];
+        for (int i = 0; i < nslots; ++i)
+            PATCH_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(g->stage_x[i]) + m0 * slotK[i] * 2,
+                                       static_cast<const uint8_t*>(src[i]) + m0 * slotK[i] * 2,
+                                       (size_t)rows * slotK[i] * 2, cudaMemcpyHostToDevice, g->h2d));
+        PATCH_CUDA(cudaEventRecord(x_ready, g->h2d));
+        PATCH_CUDA(cudaStreamWaitEvent(s, x_ready, 0));
+        const void* xs[kMaxGroup];
+        void* ys[kMaxGroup];
+        for (int l = 0; l < g->n; ++l) {
+            xs[l] = static_cast<const uint8_t*>(g->stage_x[slot[l]]) + m0 * g->h[l]->K * 2;
+            ys[l] = static_cast<uint8_t*>(g->stage_y[l]) + m0 * g->h[l]->N * 2;
+        }
+        st = run_group(g, xs, rows, ys, rpath, s);
+        if (st != PATCH_OK) return st;
+        PATCH_CUDA(cudaEventRecord(y_ready, s));
+        PATCH_CUDA(cudaStreamWaitEvent(g->d2h, y_ready, 0));
+        for (int l = 0; l < g->n; ++l)
+            PATCH_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(Y_host[l]) + m0 * g->h[l]->N * 2,
+                                       static_cast<const uint8_t*>(g->stage_y[l]) + m0 * g->h[l]->N * 2,
+                                       (size_t)rows * g->h[l]->N * 2, cudaMemcpyDeviceToHost, g->d2h));
+    }
+    PATCH_CUDA(cudaEventRecord(g->last_done, g->d2h));
+    PATCH_CUDA(cudaStreamWaitEvent(s, g->last_done, 0));  // Y_host is complete once `stream` is
+    return PATCH_OK;
+}
+
 patch_status patch_selftest_wait(void* stream) {
     int dev = 0;
     PATCH_CUDA(cudaGetDevice(&dev));
@@ -960,9 +1239,23 @@ patch_status patch_check(patch_handle h, void* stream) {
     PATCH_CUDA(cudaStreamSynchronize(s));
     PATCH_CUDA(cudaMemcpy(&word, h->status_dev, sizeof(int), cudaMemcpyDeviceToHost));
     if (word != 0) {
+        PATCH_CUDA(cudaDeviceSynchronize());
         PATCH_CUDA(cudaMemset(h->status_dev, 0, sizeof(int)));
-        // an abandoned decode call may leave strip counters part-way: re-arm them
-        PATCH_CUDA(cudaMemset(h->decode_counters, 0, sizeof(unsigned) * h->plan.S));
+        // an abandoned decode call may leave strip counters part-way: re-arm
+        // those of every workspace of every group this handle belongs to
+        std::vector<patch_group_s*> gs;
+        {
+            std::lock_guard<std::mutex> lk(h->groups_mu);
+            gs = h->groups;
+        }
+        for (patch_group g : gs) {
+            std::lock_guard<std::mutex> lk(g->mu);
+            std::vector<DecodeWs*> all{&g->capture_ws};
+            for (auto& kv : g->decode_ws) all.push_back(&kv.second);
+            for (DecodeWs* w : all)
+                for (int i = 0; i < g->n; ++i)
+                    if (w->counters[i]) PATCH_CUDA(cudaMemset(w->counters[i], 0, sizeof(unsigned) * w->S[i]));
+        }
         if (word == kStatusTimeout) return fail(PATCH_ERR_TIMEOUT, "a device-side wait ran past its limit");
         return fail(PATCH_ERR_CUDA, "device status word %d", word);
     }
@@ -1031,7 +1324,12 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     const int64_t mb = (M + bn - 1) / bn;
     const int64_t rows = kernel_rows(h->plan, kernel);
     const int slots = kernel_slots(h->dev, kernel);
-    if (rows * mb > kNoAllocMaxUnits || slots > kNoAllocMaxSlots)
+    if (slots > kNoAllocMaxSlots)
+        return fail(PATCH_ERR_UNSUPPORTED,
+                    "patch_linear_noalloc holds schedules for at most %d persistent CTAs or CTA pairs "
+                    "(this device runs %d); use patch_linear",
+                    kNoAllocMaxSlots, slots);
+    if (rows * mb > kNoAllocMaxUnits)
         return fail(PATCH_ERR_SHAPE,
                     "patch_linear_noalloc handles at most %d output tiles per call (this call needs %lld); "
                     "use patch_linear",

@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 continue;
             }
             // this unit's partial: workspace[s][p][row][0..15]
-            float4* dst = reinterpret_cast<float4*>(L.partial + (((size_t)s * P + p) * 128 + row) * kBN);
+            float4* dst = reinterpret_cast<float4*>(a.partial[l] + (((size_t)s * P + p) * 128 + row) * kBN);
 #pragma unroll
             for (int c = 0; c < kBN / 4; ++c)
                 dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 // the barrier orders the warpgroup's stores before this fence,
                 // which releases them with the arrival
                 __threadfence();
-                const unsigned old = atomicAdd(&L.counters[s], 1u);
+                const unsigned old = atomicAdd(&a.counters[l][s], 1u);
                 last_flag[g] = (old == (unsigned)(P - 1));
             }
             epi_bar(g);
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 for (int c = 0; c < kBN; ++c) sum[c] = 0.f;
                 for (int pp = 0; pp < P; ++pp) {
                     const float4* src =
-                        reinterpret_cast<const float4*>(L.partial + (((size_t)s * P + pp) * 128 + row) * kBN);
+                        reinterpret_cast<const float4*>(a.partial[l] + (((size_t)s * P + pp) * 128 + row) * kBN);
 #pragma unroll
                     for (int c = 0; c < kBN / 4; ++c) {
                         const float4 f = __ldcg(src + c);
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
                     if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(sum[c]);
-                if ((int)threadIdx.x == leader) L.counters[s] = 0u;  // re-armed for the next call
+                if ((int)threadIdx.x == leader) a.counters[l][s] = 0u;  // re-armed for the next call
             }
         }
     }

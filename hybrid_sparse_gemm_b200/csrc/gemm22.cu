@@ -30,7 +30,7 @@ namespace patch {
 
 namespace {
 
-constexpr int kProducers = 2;                   // TMA-issuing warps (slabs dealt round robin)
+constexpr int kProducers = 2;                   // TMA-issuing warps (stages dealt round robin)
 constexpr int kMmaWarp = kProducers;            // MMA issuers (leader CTA), one per strip pair;
 constexpr int kMmaWarps = 2;                    // the first also owns TMEM
 constexpr int kEpiWarp0 = kMmaWarp + kMmaWarps;
@@ -38,14 +38,14 @@ constexpr int kEpiWarps = 16;                   // per accumulator, two warps pe
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBN = kGemm22BN;                  // tokens per tile (both CTAs)
 constexpr int kHalfN = kBN / 2;                 // token rows of operand B per CTA
-constexpr int kStageB = kHalfN * 128;           // 15 KB of activations per slab
-constexpr int kRecDense = 16384;                // dense slab image
-constexpr int kRecSparse = 10240;               // 2:4 values (8 KB) + room for the chunk's metadata (2 KB)
-constexpr int kRing = 208896;                   // shared-memory ring the slabs are placed in, in order
-constexpr int kQ = 8;                           // per-slab barriers: more than the slabs that fit in the ring
-static_assert(kRing % 1024 == 0 && kRecSparse % 1024 == 0 && kStageB % 1024 == 0,
+constexpr int kStageX = kHalfN * 128;           // 15 KB of activations per slab
+constexpr int kRing = 208896;                   // shared-memory ring the stages are placed in, in order
+constexpr int kQ = 8;                           // per-stage barriers: more than the stages that fit in the ring
+// smallest stage: two 2:4 slabs of each strip (16 KB + 2 KB metadata) and two activation tiles
+constexpr int kMinStage = 2 * (2 * kSparseValBytes + kMetaBytes) + 2 * kStageX;
+static_assert(kRing % 1024 == 0 && kStageX % 1024 == 0 && kMetaBytes % 1024 == 0,
               "every record starts 1024-byte aligned (128-byte swizzle atoms)");
-static_assert(kRing / (2 * kRecSparse + kStageB) + 2 <= kQ, "slabs in flight stay within the barrier window");
+static_assert(kRing / kMinStage + 2 <= kQ, "stages in flight stay within the barrier window");
 constexpr int kSmemData = kRing;
 constexpr int kSmemBytes = kSmemData + 1024 + 256;
 constexpr int kAcc1 = 256;                      // first column of accumulator 1
@@ -60,17 +60,35 @@ __device__ __forceinline__ int tile_tokens(int j, int M) {
     return rem >= kBN ? kBN : ((rem + 15) & ~15);
 }
 
-// Record bytes of one slab (values or dense image, plus metadata at the first
-// 2:4 slab of a chunk).
-__device__ __forceinline__ uint32_t record_bytes(uint32_t d) {
-    return ((d & kSlabSparse) ? kSparseValBytes : kDenseSlabBytes) + ((d & kSlabFirst) ? kMetaBytes : 0);
+__device__ __forceinline__ uint32_t rec_bytes(uint32_t d) {
+    return (d & kSlabSparse) ? kSparseValBytes : kDenseSlabBytes;
 }
 
-__device__ __forceinline__ uint32_t ring_rec(uint32_t d) { return (d & kSlabSparse) ? kRecSparse : kRecDense; }
+// One stage is one chunk (two 64-column slabs, one for an odd last chunk) of
+// both strips this CTA holds, plus the activation tiles of those slabs. A
+// strip's part of the stage: its slab records back to back, then the chunk's
+// 2 KB metadata block when either slab runs on the sparse MMA.
+struct Chunk {
+    uint32_t d[2];  // gemm-table records of the chunk's slabs
+    int n;          // slabs in the chunk (1 or 2)
+    __device__ __forceinline__ bool sparse() const {
+        return ((d[0] | (n > 1 ? d[1] : 0u)) & kSlabSparse) != 0;
+    }
+    __device__ __forceinline__ uint32_t recs() const { return rec_bytes(d[0]) + (n > 1 ? rec_bytes(d[1]) : 0u); }
+    __device__ __forceinline__ uint32_t bytes() const { return recs() + (sparse() ? (uint32_t)kMetaBytes : 0u); }
+};
 
-// Slabs are placed one after another in a ring of kRing bytes; a slab that
+__device__ __forceinline__ Chunk load_chunk(const uint32_t* t, int c, int KB) {
+    Chunk k;
+    k.n = (2 * c + 1 < KB) ? 2 : 1;
+    k.d[0] = t[2 * c];
+    k.d[1] = k.n > 1 ? t[2 * c + 1] : 0u;
+    return k;
+}
+
+// Stages are placed one after another in a ring of kRing bytes; a stage that
 // does not fit before the end starts again at 0. `pos` counts bytes placed so
-// far (including skipped ends); returns the ring offset of this slab.
+// far (including skipped ends); returns the ring offset of this stage.
 struct Ring {
     uint32_t pos = 0, off = 0;
     __device__ __forceinline__ uint32_t place(uint32_t size) {
@@ -85,25 +103,24 @@ struct Ring {
     }
 };
 
-// One strip pair's MMAs for one slab: 4 dense K=16 MMAs, or the metadata copy
-// (first 2:4 slab of a chunk) and 2 sparse K=32 MMAs.
-__device__ __forceinline__ void issue_slab(uint32_t d, int b, uint32_t a_addr, uint32_t b_addr, uint32_t d_tmem,
-                                           uint32_t e_col, uint32_t idesc_d, uint32_t idesc_s) {
+// One strip pair's MMAs for one slab: 4 dense K=16 MMAs, or 2 sparse K=32
+// MMAs reading the metadata columns of this slab's half of the chunk.
+__device__ __forceinline__ void issue_slab(uint32_t d, int half, bool first, uint32_t a_addr, uint32_t b_addr,
+                                           uint32_t d_tmem, uint32_t e_col, uint32_t idesc_d, uint32_t idesc_s) {
     if (d & kSlabSparse) {
-        if (d & kSlabFirst) cp2_128x128b(e_col, smem_desc(a_addr + kSparseValBytes, 16, 128, kLayoutNone));
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const uint64_t ad = smem_desc(a_addr + i * 32, 16, 512, kLayoutSw64);
             const uint64_t bd = smem_desc(b_addr + i * 64, 16, 1024, kLayoutSw128);
-            const uint32_t ecol = e_col + (uint32_t)((b & 1) * 2 + i);
-            mma2_sp_bf16(d_tmem, ad, bd, idesc_s | (ecol & 1u), ecol & ~1u, (b | i) != 0);
+            const uint32_t ecol = e_col + (uint32_t)(half * 2 + i);
+            mma2_sp_bf16(d_tmem, ad, bd, idesc_s | (ecol & 1u), ecol & ~1u, !(first && i == 0));
         }
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint64_t ad = smem_desc(a_addr + i * 32, 16, 1024, kLayoutSw128);
             const uint64_t bd = smem_desc(b_addr + i * 32, 16, 1024, kLayoutSw128);
-            mma2_bf16(d_tmem, ad, bd, idesc_d, (b | i) != 0);
+            mma2_bf16(d_tmem, ad, bd, idesc_d, !(first && i == 0));
         }
     }
 }
@@ -114,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
-    uint64_t* full = bars;                       // [kQ] leader: both CTAs' bytes of slab g (at g % kQ)
-    uint64_t* empty = full + kQ;                 // [kQ] every CTA: slab g consumed by both issuers
+    uint64_t* full = bars;                       // [kQ] leader: both CTAs' bytes of stage g (at g % kQ)
+    uint64_t* empty = full + kQ;                 // [kQ] every CTA: stage g consumed by both issuers
     uint64_t* acc_full = empty + kQ;             // [2] both CTAs: accumulator h ready
     uint64_t* acc_empty = acc_full + 2;          // [2] leader: the 16 epilogue warps of accumulator h drained it
     uint64_t* drain = acc_empty + 2;             // [2]
@@ -170,37 +187,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kProducers) {
         if (lane == 0) {
             // ---------------- producers (both CTAs) ----------------
-            // Every producer walks the whole slab sequence to place each slab in
-            // the ring; it loads the slabs g with g % kProducers == me. Before
-            // loading, the slabs that last used those ring bytes must have been
-            // consumed (in-order, so waiting for the latest of them suffices).
+            // Every producer walks the whole stage sequence to place each stage
+            // in the ring; it loads the stages g with g % kProducers == me.
+            // Before loading, the stages that last used those ring bytes must
+            // have been consumed (in order, so waiting for the latest suffices).
             const int me = warp;
             Ring ring;
-            uint32_t hist[kQ];   // ring positions where the last kQ slabs started
+            uint32_t hist[kQ];   // ring positions where the last kQ stages started
             int g = 0;
-            int my_last = -1;    // sequence index of the last slab this producer loaded
+            int my_last = -1;    // sequence index of the last stage this producer loaded
             bool ok = true;
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
                 const int c = lu / a.MB, j = lu % a.MB;
-                const int KB = L.KB;
+                const int KB = L.KB, KC = L.KC;
                 const int s0 = strip_of(c, 0, L.S), s1 = strip_of(c, 1, L.S);
                 const uint32_t* t0 = L.gemm + (size_t)s0 * KB;
                 const uint32_t* t1 = L.gemm + (size_t)s1 * KB;
-                const uint32_t* m0 = L.meta + (size_t)s0 * L.KC;
-                const uint32_t* m1 = L.meta + (size_t)s1 * L.KC;
+                const uint32_t* m0 = L.meta + (size_t)s0 * KC;
+                const uint32_t* m1 = L.meta + (size_t)s1 * KC;
                 const CUtensorMap* tm_x = &maps.x[l];
-                const CUtensorMap* tm_a16 = &maps.a16[l];
-                const CUtensorMap* tm_a8 = &maps.a8[l];
-                const CUtensorMap* tm_e = &maps.e[l];
                 const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
-                for (int b = 0; b < KB; ++b, ++g) {
-                    const uint32_t d0 = t0[b], d1 = t1[b];
-                    const uint32_t r0 = ring_rec(d0), r1 = ring_rec(d1);
-                    const uint32_t off = ring.place(r0 + r1 + kStageB);
-                    hist[g % kQ] = ring.pos - (r0 + r1 + kStageB);
+                for (int kc = 0; kc < KC; ++kc, ++g) {
+                    const Chunk k0 = load_chunk(t0, kc, KB), k1 = load_chunk(t1, kc, KB);
+                    const uint32_t size = k0.bytes() + k1.bytes() + (uint32_t)k0.n * kStageX;
+                    const uint32_t off = ring.place(size);
+                    hist[g % kQ] = ring.pos - size;
                     if (g % kProducers != me) continue;
                     if (ring.pos > (uint32_t)kRing) {
                         const uint32_t need = ring.pos - (uint32_t)kRing;
@@ -217,22 +231,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     const uint32_t bar = map_to_rank(smem_u32(&full[g % kQ]), 0);
-                    if (pr == 0)
-                        mbar_arrive_expect_tx(&full[g % kQ], 2u * (record_bytes(d0) + record_bytes(d1) + kStageB));
-                    const uint32_t base = smem_u32(smem) + off;
-                    tma_load_2d_pair(base, (d0 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0, (int)(slab_offset_bytes(d0) >> 7));
-                    if (d0 & kSlabFirst)
-                        tma_load_2d_pair(base + kSparseValBytes, tm_e, bar, 0, (int)(m0[b >> 1] >> 3));
-                    tma_load_2d_pair(base + r0, (d1 & kSlabSparse) ? tm_a8 : tm_a16, bar, 0,
-                                     (int)(slab_offset_bytes(d1) >> 7));
-                    if (d1 & kSlabFirst)
-                        tma_load_2d_pair(base + r0 + kSparseValBytes, tm_e, bar, 0, (int)(m1[b >> 1] >> 3));
-                    tma_load_2d_pair(base + r0 + r1, tm_x, bar, b * kSlabK, tok);
+                    if (pr == 0) mbar_arrive_expect_tx(&full[g % kQ], 2u * size);
+                    uint32_t dst = smem_u32(smem) + off;
+                    for (int h = 0; h < 2; ++h) {
+                        const Chunk& k = h ? k1 : k0;
+                        const uint32_t mrow = (h ? m1 : m0)[kc];
+                        // both slabs in one copy when their records are adjacent
+                        // and of one kind (a 2:4 pair is one 128-row box, a dense
+                        // pair one 256-row box)
+                        const bool joint = k.n == 2 && ((k.d[0] ^ k.d[1]) & kSlabSparse) == 0 &&
+                                           slab_offset_bytes(k.d[1]) == slab_offset_bytes(k.d[0]) + rec_bytes(k.d[0]);
+                        if (joint) {
+                            tma_load_2d_pair(dst, (k.d[0] & kSlabSparse) ? &maps.a16[l] : &maps.a32[l], bar, 0,
+                                             (int)(slab_offset_bytes(k.d[0]) >> 7));
+                        } else {
+                            for (int i = 0; i < k.n; ++i)
+                                tma_load_2d_pair(dst + (i ? rec_bytes(k.d[0]) : 0u),
+                                                 (k.d[i] & kSlabSparse) ? &maps.a8[l] : &maps.a16[l], bar, 0,
+                                                 (int)(slab_offset_bytes(k.d[i]) >> 7));
+                        }
+                        if (k.sparse()) tma_load_2d_pair(dst + k.recs(), &maps.e[l], bar, 0, (int)(mrow >> 3));
+                        dst += k.bytes();
+                    }
+                    for (int i = 0; i < k0.n; ++i) tma_load_2d_pair(dst + i * kStageX, tm_x, bar, (2 * kc + i) * kSlabK, tok);
                     my_last = g;
                 }
             }
             if (pr == 0) {
-                // Bounded wait for the loads of my last slabs, whatever the
+                // Bounded wait for the loads of my last stages, whatever the
                 // abort flag says, so none lands after the cluster exits.
                 for (int gg = my_last - kQ + 1; gg <= my_last; ++gg) {
                     if (gg < 0 || gg % kProducers != me) continue;
@@ -246,51 +272,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kMmaWarp + kMmaWarps) {
         if (lane == 0 && pr == 0) {
             // ---------------- MMA issuers (leader CTA), one per strip pair ----------------
-            // Both read every slab; a slab's ring bytes are free once both have
-            // committed it. Two issuing threads keep the tensor pipe fed while
-            // either one waits on a barrier or computes descriptors.
+            // Both read every stage; a stage's ring bytes are free once both
+            // have committed it. Two issuing threads keep the tensor pipe fed
+            // while either one waits on a barrier or computes descriptors.
             const int h = warp - kMmaWarp;
             const uint32_t d_tmem = tmem_base + (uint32_t)(h * kAcc1);
             const uint32_t e_col = tmem_base + (uint32_t)(h ? kECol1 : kECol0);
             Ring ring;
             int g = 0;
             bool ok = true, any_mma = false;
-            bool ready = false;  // full[g % kQ] already seen complete by the look-ahead
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int u = a.work[it];
                 const LinDesc& L = a.lins[u >> kUnitShift];
                 const int lu = u & kUnitMask;
                 const int c = lu / a.MB, j = lu % a.MB;
-                const int KB = L.KB;
-                // both strip pairs' records place the slab in the ring
+                const int KB = L.KB, KC = L.KC;
+                // both strip pairs' records place the stage in the ring
                 const uint32_t* t0 = L.gemm + (size_t)strip_of(c, 0, L.S) * KB;
                 const uint32_t* t1 = L.gemm + (size_t)strip_of(c, 1, L.S) * KB;
                 const int nt = tile_tokens(j, a.M);
                 const uint32_t idesc_d = idesc_bf16(256, nt, false);
                 const uint32_t idesc_s = idesc_bf16(256, nt, true);
-                uint32_t d0 = t0[0], d1 = t1[0];
+                Chunk k0 = load_chunk(t0, 0, KB), k1 = load_chunk(t1, 0, KB);
                 if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
                     raise();
                     break;
                 }
                 tc_fence_after();
-                for (int b = 0; b < KB; ++b, ++g) {
-                    if (!ready && !mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
+                for (int kc = 0; kc < KC; ++kc, ++g) {
+                    if (!mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
                         raise();
                         ok = false;
                         break;
                     }
-                    const uint32_t d0n = b + 1 < KB ? t0[b + 1] : 0u;
-                    const uint32_t d1n = b + 1 < KB ? t1[b + 1] : 0u;
-                    ready = mbar_test_wait(&full[(g + 1) % kQ], (uint32_t)(((g + 1) / kQ) & 1));
-                    const uint32_t r0 = ring_rec(d0), r1 = ring_rec(d1);
-                    const uint32_t base = smem_u32(smem) + ring.place(r0 + r1 + kStageB);
-                    issue_slab(h ? d1 : d0, b, base + (h ? r0 : 0u), base + r0 + r1, d_tmem, e_col, idesc_d, idesc_s);
+                    // next chunk's records, read while this one's MMAs issue
+                    Chunk n0, n1;
+                    if (kc + 1 < KC) {
+                        n0 = load_chunk(t0, kc + 1, KB);
+                        n1 = load_chunk(t1, kc + 1, KB);
+                    }
+                    const uint32_t base = smem_u32(smem) + ring.place(k0.bytes() + k1.bytes() + (uint32_t)k0.n * kStageX);
+                    const Chunk& k = h ? k1 : k0;
+                    const uint32_t a_addr = base + (h ? k0.bytes() : 0u);
+                    const uint32_t b_addr = base + k0.bytes() + k1.bytes();
+                    if (k.sparse()) cp2_128x128b(e_col, smem_desc(a_addr + k.recs(), 16, 128, kLayoutNone));
+                    issue_slab(k.d[0], 0, kc == 0, a_addr, b_addr, d_tmem, e_col, idesc_d, idesc_s);
+                    if (k.n > 1)
+                        issue_slab(k.d[1], 1, false, a_addr + rec_bytes(k.d[0]), b_addr + kStageX, d_tmem, e_col,
+                                   idesc_d, idesc_s);
                     any_mma = true;
                     commit2_mask(&empty[g % kQ], 3);
-                    d0 = d0n;
-                    d1 = d1n;
+                    if (kc + 1 < KC) {
+                        k0 = n0;
+                        k1 = n1;
+                    }
                 }
                 if (!ok) break;
                 commit2_mask(&acc_full[h], 3);

@@ -34,16 +34,14 @@ struct LinDesc {
     const uint32_t* slab;      // per-strip slab table
     const uint32_t* meta;      // metadata block table
     const uint32_t* gemm;      // CTA-pair slab table
-    float* partial;            // decode workspace [S][P][128][16] fp32
-    unsigned* counters;        // decode arrivals per strip, zero between calls
     int N, S, KB, KC, P;       // P: decode K-parts per strip
 };
 
 // Tensor maps: X of every member (per call) and the packed bytes of every
-// member viewed as 128-byte rows with 128-, 64- and 16-row boxes.
+// member viewed as 128-byte rows with 256-, 128-, 64- and 16-row boxes.
 struct GroupMaps {
     CUtensorMap x[kMaxGroup];
-    CUtensorMap a16[kMaxGroup], a8[kMaxGroup], e[kMaxGroup];
+    CUtensorMap a32[kMaxGroup], a16[kMaxGroup], a8[kMaxGroup], e[kMaxGroup];
 };
 
 // Per-call arguments. A work unit is (member << 24) | local index, the local
@@ -52,6 +50,11 @@ struct GroupMaps {
 struct GroupArgs {
     const LinDesc* lins;
     __nv_bfloat16* Y[kMaxGroup];
+    // decode only: split-K workspace [S][P][128][16] fp32 and per-strip
+    // arrival counters (zero between calls) of each member, owned by the
+    // calling stream so that calls on different streams never share them
+    float* partial[kMaxGroup];
+    unsigned* counters[kMaxGroup];
     const int* work_off;       // per CTA (or per CTA pair): [work_off[c], work_off[c+1])
     const int* work;
     int M, MB;

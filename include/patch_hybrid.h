@@ -23,10 +23,20 @@
  *     stream. Calls are stream-ordered and asynchronous unless stated.
  *   - No call throws, aborts or traps. Each returns a patch_status; the
  *     message of the last failure on the calling thread is patch_last_error().
- *   - The caller owns every buffer it passes. A handle owns only the packed
- *     copy of the weights and its own tables.
- *   - A handle is immutable after patch_pack: concurrent patch_linear calls on
- *     one handle from several streams or threads are safe.
+ *   - The caller owns every buffer it passes. A handle owns the packed copy
+ *     of the weights, its tables, its cached schedules and the decode
+ *     kernel's split-K workspaces.
+ *   - Concurrency: patch_linear, patch_linear_path and patch_group_linear
+ *     calls on one handle or group may overlap on the GPU when they are
+ *     issued on different streams or threads. The decode kernel (M <= 16)
+ *     keeps its split-K partial sums in a workspace per stream (per thread
+ *     for the per-thread default stream); the other kernels keep no per-call
+ *     state. Three exceptions: patch_linear_host calls on one handle share a
+ *     staging buffer; all patch_linear_noalloc calls share one array; and
+ *     every CUDA graph that captured decode calls of one handle or group uses
+ *     that handle's or group's one capture workspace. Calls in each of these
+ *     three classes must not overlap on the GPU (order them on one stream, or
+ *     synchronise between them).
  */
 #ifndef PATCH_HYBRID_H
 #define PATCH_HYBRID_H
@@ -50,7 +60,8 @@ typedef enum {
     PATCH_ERR_CUDA = 5,        /* a CUDA runtime call failed */
     PATCH_ERR_TIMEOUT = 6,     /* a device-side wait ran past its limit */
     PATCH_ERR_NOMEM = 7,       /* device or host allocation failed */
-    PATCH_ERR_UNSUPPORTED = 8  /* current device is not compute capability 10.x */
+    PATCH_ERR_UNSUPPORTED = 8  /* the current device is not compute capability 10.x, or is
+                                  larger than a fixed limit of patch_linear_noalloc */
 } patch_status;
 
 /* Which kernel patch_linear_path runs. AUTO picks by M: GEMV for M <= 16,
@@ -191,8 +202,12 @@ patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flag
  *   Y_bf16  dev, M*N bf16 row-major, 16-byte aligned. Every element is
  *           written: fp32 accumulation, one round-to-nearest-even to bf16.
  * Picks the tensor-core kernel or the decode kernel by M. The first call for
- * a new value of M builds and uploads that M's work schedule (allocates); do
- * one such call before capturing later ones in a CUDA graph.
+ * a new value of M builds that M's work schedule and uploads it
+ * asynchronously on `stream` (it allocates device and pinned host memory);
+ * a call on another stream waits for that upload on the device. The first
+ * uncaptured decode call (M <= 16) on a stream allocates that stream's
+ * workspace. Before capturing later calls in a CUDA graph, make one call
+ * with the same M and let it complete.
  */
 patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                           void* stream);
@@ -222,18 +237,28 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
  * allocates on first use. Callers whose device memory is owned by someone
  * else (a frozen allocator, another framework's memory pool, a thread that
  * may not call cudaMalloc) use this call instead: it allocates nothing and
- * keeps the schedule in one fixed array inside this library's device image,
- * sized for at most 65536 output tiles per call (256-token tiles for
- * M >= 256, 128-token tiles below; PATCH_ERR_SHAPE beyond that). Every GPU
- * that loads the library holds that array (about 257 KiB) until the process
- * exits.
+ * keeps the schedule in one fixed array inside this library's device image.
+ * Every GPU that loads the library holds that array (about 257 KiB) until
+ * the process exits.
  *
- *   Arguments, layouts and results as for patch_linear (AUTO path).
- * The first call on a device looks up the array's device address; make that
- * first call before capturing later calls in a CUDA graph. All calls share
- * the one array and each overwrites it, so calls that overlap on the GPU
- * (different streams, or several handles at once) race: order them on one
- * stream or synchronise between them.
+ *   Arguments and layouts as for patch_linear. Kernel per M:
+ *     M <= 8         CUDA-core decode kernel (GEMV_SIMT), no schedule;
+ *     9 <= M < 256   single-CTA tensor-core kernel, 128-row x 128-token tiles;
+ *     M >= 256       the CTA-pair kernel patch_linear would run for this M:
+ *                    GEMM_WIDE (512-row x 240-token tiles) or GEMM_PAIR
+ *                    (256-row x 256-token tiles).
+ *   For M >= 17 the result is bit-identical to patch_linear's (same kernel,
+ *   same schedule); for M <= 16 patch_linear runs the tensor-core decode
+ *   kernel instead, which sums in another order (both within the tolerance
+ *   of the fp32 product).
+ * Limits: at most 65536 output tiles per call (tiles as above;
+ * PATCH_ERR_SHAPE beyond that) and at most 256 persistent CTAs or CTA pairs
+ * on the device (PATCH_ERR_UNSUPPORTED beyond that).
+ * The first call on each device looks up the array's device address
+ * (set-up); make that first call before any stream capture begins. All calls
+ * share the one array and each overwrites it, so calls that overlap on the
+ * GPU (different streams, or several handles at once) race: order them on
+ * one stream or synchronise between them.
  */
 patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                                   void* stream);
@@ -263,6 +288,31 @@ patch_status patch_group_create(const patch_handle* handles, int n, patch_group*
  */
 patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, void* const* Y, int path,
                                 void* stream);
+
+/*
+ * patch_group_linear_host - patch_group_linear from and to HOST memory, with
+ * the copies overlapped with the product.
+ *
+ *   X  host array of n host pointers, X_i: M x K_i bf16 row-major. Members
+ *      that pass the same pointer (q, k, v) share one upload.
+ *   Y  host array of n host pointers, Y_i: M x N_i bf16 row-major.
+ *   M, path as for patch_group_linear; stream is where the product runs.
+ * The tokens are cut into up to four chunks, each a whole number of token
+ * tiles of the kernel patch_group_linear would run for this M (so Y is bit
+ * for bit the device call's): the inputs of chunk c go up on one copy stream
+ * while chunk c-1 is computed on `stream` and the outputs of chunk c-2 come
+ * back on another, so both copy directions and the tensor cores work at
+ * once. Pinned host memory gives
+ * asynchronous copies; pageable memory works, with copies that block the
+ * host. Asynchronous: the call returns once everything is enqueued; the Y
+ * buffers are complete when `stream` is (it waits for the last copy back),
+ * and X and Y must stay valid until then. The group owns the device staging
+ * buffers (grown on demand: the first call for a larger M allocates and
+ * waits for the group's previous host call). Calls on one group are ordered
+ * among themselves on the device; issue them from one host thread at a time.
+ */
+patch_status patch_group_linear_host(patch_group g, const void* const* X, int64_t M, void* const* Y,
+                                     int path, void* stream);
 
 /*
  * patch_group_path - the explicit path (GEMV, GEMV_SIMT, GEMM_SINGLE,

@@ -24,10 +24,36 @@ def test_bench_imports_and_peaks():
 
 
 def test_cpu_baseline_sample():
+    """All host threads, then one thread: both rates positive, the thread
+    counts and the CPU model reported."""
     b = _bench()
-    rate, threads, desc = b.cpu_sample(budget_s=0.2, min_rows=1)
-    assert rate > 0 and threads >= 1
-    assert "oracle" in desc and "token rows" in desc
+    got = b.cpu_sample(budget_s=0.2, min_rows=1, workload="llama32-1b", one_core_s=0.5)
+    assert got["value"] > 0 and got["cores"] >= 1 and got["kind"] == "oracle"
+    assert "oracle" in got["sample"] and "token rows" in got["sample"]
+    assert got["cpu_model"] and got["nproc"] >= 1
+    assert got["value_1core"] > 0 and "1 thread" in got["sample_1core"]
+
+
+def test_peak_choice_and_roofline():
+    """Burst peak for a short timed region, sustained only for a long one
+    under the power cap; the roofline's achieved rate is the kept-weight work
+    of the step over the step time."""
+    b = _bench()
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured", "hbm_gbs": 1.0}
+    assert b.choose_peak(peaks, 0.3, {"reasons": ["sw_power_cap"]})[0] == 1600.0
+    assert b.choose_peak(peaks, 5.0, {"reasons": []})[0] == 1600.0
+    assert b.choose_peak(peaks, 5.0, {"reasons": ["sw_power_cap"]})[0] == 1400.0
+
+    class Info:
+        pruned, slabs_total, slabs_pair_sparse, packed_bytes = 64 * 128, 4, 1, 0
+        tiles_sparse, tile_rows, tile_cols = 1, 128, 128
+
+    m = b.Member(None, 256, 128, Info(), None, None)
+    assert m.kept == 128 * 256 - 64 * 128 and m.executed == 3 * 8192 + 4096
+    model = [(None, [m, m])]
+    r = b.roofline(model, 10, 2.0, 4, 1600.0, "burst", "k", None)
+    assert abs(r["achieved"] - 2 * 2.0 * 10 * m.kept / 2e-3 / 1e12) < 1e-12
+    assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-15 and r["kernel_ms_per_launch"] == 0.5
 
 
 def test_measured_traffic_is_pinned_to_source():

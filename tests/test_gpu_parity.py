@@ -298,6 +298,121 @@ def test_empty_and_misaligned(hsg):
     lin.free()
 
 
+def test_decode_concurrent_streams(hsg, oracle_lib):
+    """Decode calls on one handle and on one group from two streams, with no
+    synchronisation between the streams: each stream has its own split-K
+    workspace, so both streams' results equal the sequential ones bit for bit
+    (and the oracle)."""
+    p = synth.make_problem(1152, 4096, 16, R=128, C=128, frac=0.7, seed=19, device="cuda")
+    q = synth.make_problem(640, 4096, 16, R=128, C=128, frac=0.5, seed=20, device="cuda")
+    lp, lq = pack(hsg, p), pack(hsg, q)
+    g = hsg.LinearGroup([lp, lq])
+    Xa, Xb = p.X[:16].contiguous(), p.X[:3].contiguous()
+    ref_a, ref_b = lp(Xa, path=hsg.PATH_GEMV), lp(Xb, path=hsg.PATH_GEMV)
+    gref = g([Xa, q.X[:16].contiguous()], path=hsg.PATH_GEMV)
+    torch.cuda.synchronize()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    outs_a, outs_b, gouts = [], [], []
+    for _ in range(20):
+        outs_a.append(lp(Xa, path=hsg.PATH_GEMV, stream=sa))
+        outs_b.append(lp(Xb, path=hsg.PATH_GEMV, stream=sb))
+        gouts.append(g([Xa, q.X[:16].contiguous()], path=hsg.PATH_GEMV, stream=sb))
+    torch.cuda.synchronize()
+    lp.check()
+    for Ya, Yb, Yg in zip(outs_a, outs_b, gouts):
+        assert torch.equal(Ya, ref_a) and torch.equal(Yb, ref_b)
+        assert torch.equal(Yg[0], gref[0]) and torch.equal(Yg[1], gref[1])
+    assert_close(outs_a[-1], oracle_lib, Xa, p.W, p.bits, p.keep, what="decode stream a")
+    assert_close(outs_b[-1], oracle_lib, Xb, p.W, p.bits, p.keep, what="decode stream b")
+    g.free()
+    lp.free()
+    lq.free()
+
+
+def test_first_call_schedule_used_from_another_stream(hsg, oracle_lib):
+    """The first call for an M uploads its schedule asynchronously; a call on
+    another stream right after it (no host synchronisation) waits for the
+    upload on the device and gives the same bits."""
+    p = synth.make_problem(1024, 2048, 777, R=128, C=128, frac=0.9, seed=23, device="cuda")
+    lin = pack(hsg, p)
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    Ya = lin(p.X, stream=sa)
+    Yb = lin(p.X, stream=sb)
+    torch.cuda.synchronize()
+    assert torch.equal(Ya, Yb)
+    rows = sample_rows(777)
+    assert_close(Yb, oracle_lib, p.X, p.W, p.bits, p.keep, rows=rows, what="schedule from another stream")
+    lin.free()
+
+
+@pytest.mark.parametrize("M", [5, 300, 1000, 2048])
+def test_group_host_matches_device(hsg, M):
+    """patch_group_linear_host (token chunks whose copies overlap the product)
+    gives the device call's bits; members sharing a host input (q, k, v) and
+    two calls in a row without a host synchronisation between them."""
+    shapes = [(512, 1024), (256, 1024), (384, 768)]
+    probs = [synth.make_problem(N, K, M, R=128, C=128, frac=0.7, seed=40 + i, device="cuda", tag="gh")
+             for i, (N, K) in enumerate(shapes)]
+    lins = [pack(hsg, p) for p in probs]
+    g = hsg.LinearGroup(lins)
+    X1 = probs[0].X
+    Xs_dev = [X1, X1, probs[2].X]
+    ref = g(Xs_dev)
+    torch.cuda.synchronize()
+    xa = X1.cpu().pin_memory()
+    Xh = [xa, xa, probs[2].X.cpu().pin_memory()]
+    out1 = g.host(Xh, sync=False)
+    Xh2 = [x.clone().pin_memory() for x in Xh]
+    out2 = g.host(Xh2, sync=False)
+    torch.cuda.synchronize()
+    for o1, o2, r in zip(out1, out2, ref):
+        assert torch.equal(o1, r.cpu()) and torch.equal(o2, r.cpu())
+    # pageable host memory works too (copies block the host)
+    out3 = g.host([x.clone() for x in Xh], outs=[torch.empty_like(r, device="cpu") for r in ref])
+    for o, r in zip(out3, ref):
+        assert torch.equal(o, r.cpu())
+    g.free()
+    for l in lins:
+        l.free()
+
+
+def test_cuda_graph_capture_and_replay(hsg):
+    """After one call with the same M has completed, patch_linear and
+    patch_group_linear calls (tensor-core GEMM and decode) can be captured in
+    a CUDA graph; replays give the eager bits."""
+    p = synth.make_problem(1024, 2048, 600, R=128, C=128, frac=0.7, seed=29, device="cuda")
+    q = synth.make_problem(512, 2048, 600, R=128, C=128, frac=0.9, seed=30, device="cuda")
+    lp, lq = pack(hsg, p), pack(hsg, q)
+    g = hsg.LinearGroup([lp, lq])
+    X16 = p.X[:16].contiguous()
+    Y1 = torch.empty((600, 1024), dtype=torch.bfloat16, device="cuda")
+    Y2 = torch.empty((16, 1024), dtype=torch.bfloat16, device="cuda")
+    G = [torch.empty((600, 1024), dtype=torch.bfloat16, device="cuda"),
+         torch.empty((600, 512), dtype=torch.bfloat16, device="cuda")]
+    eager1, eager2 = lp(p.X), lp(X16)
+    eg = g([p.X, q.X])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        lp(p.X, out=Y1)
+        lp(X16, out=Y2)
+        g([p.X, q.X], G)
+    for _ in range(3):
+        Y1.zero_()
+        Y2.zero_()
+        G[0].zero_()
+        G[1].zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y1, eager1) and torch.equal(Y2, eager2)
+        assert torch.equal(G[0], eg[0]) and torch.equal(G[1], eg[1])
+    lp.check()
+    del graph
+    g.free()
+    lp.free()
+    lq.free()
+
+
 def test_deterministic_and_host_path(hsg):
     p = synth.make_problem(512, 1024, 300, R=128, C=64, frac=0.7, seed=8, device="cuda")
     lin = pack(hsg, p)
