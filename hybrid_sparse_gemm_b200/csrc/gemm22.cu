@@ -30,7 +30,10 @@ namespace patch {
 
 namespace {
 
-constexpr int kProducers = 2;                   // TMA-issuing warps (stages dealt round robin)
+#ifndef PATCH_GEMM22_PRODUCERS
+#define PATCH_GEMM22_PRODUCERS 2
+#endif
+constexpr int kProducers = PATCH_GEMM22_PRODUCERS;  // TMA-issuing warps (stages dealt round robin)
 constexpr int kMmaWarp = kProducers;            // MMA issuers (leader CTA), one per strip pair;
 constexpr int kMmaWarps = 2;                    // the first also owns TMEM
 constexpr int kEpiWarp0 = kMmaWarp + kMmaWarps;
@@ -41,13 +44,26 @@ constexpr int kHalfN = kBN / 2;                 // token rows of operand B per C
 constexpr int kStageX = kHalfN * 128;           // 15 KB of activations per slab
 constexpr int kRing = 208896;                   // shared-memory ring the stages are placed in, in order
 constexpr int kQ = 8;                           // per-stage barriers: more than the stages that fit in the ring
-// smallest stage: two 2:4 slabs of each strip (16 KB + 2 KB metadata) and two activation tiles
-constexpr int kMinStage = 2 * (2 * kSparseValBytes + kMetaBytes) + 2 * kStageX;
+#ifndef PATCH_GEMM22_MAX_STAGE
+#define PATCH_GEMM22_MAX_STAGE 70 * 1024
+#endif
+constexpr uint32_t kMaxStage = PATCH_GEMM22_MAX_STAGE;  // larger two-slab stages are cut into one-slab stages
+// smallest stage: one 2:4 slab of each strip and its activation tile
+constexpr int kMinStage = 2 * kSparseValBytes + kStageX;
 static_assert(kRing % 1024 == 0 && kStageX % 1024 == 0 && kMetaBytes % 1024 == 0,
               "every record starts 1024-byte aligned (128-byte swizzle atoms)");
 static_assert(kRing / kMinStage + 2 <= kQ, "stages in flight stay within the barrier window");
+static_assert(kMaxStage >= 2 * (2 * kSparseValBytes + kMetaBytes) + 2 * kStageX, "two 2:4 slabs form one stage");
+// Each producer and issuer warp copies the slab records (and, for producers,
+// the metadata block offsets) of its current tile's two strips into shared
+// memory, so that no stage waits on a table read from L2. Weights with more
+// than kTabKB slabs per strip read the tables from global memory instead.
+constexpr int kTabKB = 256;                     // K up to 16384
+constexpr int kTabWords = 2 * kTabKB + 2 * (kTabKB / 2);
 constexpr int kSmemData = kRing;
-constexpr int kSmemBytes = kSmemData + 1024 + 256;
+constexpr int kSmemTab = (kProducers + kMmaWarps) * kTabWords * 4;
+constexpr int kSmemBytes = kSmemData + kSmemTab + 1024 + 256;
+static_assert(kSmemBytes <= 232448, "fits the 227 KB of shared memory a CTA may use");
 constexpr int kAcc1 = 256;                      // first column of accumulator 1
 constexpr int kECol0 = kBN;                     // metadata columns of strip pair 0
 constexpr int kECol1 = kBN + 8;                 // ... and of strip pair 1
@@ -64,18 +80,29 @@ __device__ __forceinline__ uint32_t rec_bytes(uint32_t d) {
     return (d & kSlabSparse) ? kSparseValBytes : kDenseSlabBytes;
 }
 
-// One stage is one chunk (two 64-column slabs, one for an odd last chunk) of
-// both strips this CTA holds, plus the activation tiles of those slabs. A
-// strip's part of the stage: its slab records back to back, then the chunk's
-// 2 KB metadata block when either slab runs on the sparse MMA.
+// A chunk is two 64-column slabs (one for an odd last chunk) of a strip. A
+// stage holds both strips' records of one chunk, or of one slab of it when
+// the two-slab stage would exceed kMaxStage (a chunk with dense records is
+// cut in two, so that enough stages fit in the ring to cover the load
+// latency), plus the activation tiles of those slabs. A strip's part of a
+// stage: its slab records back to back, then, in the stage that holds the
+// chunk's first slab, the chunk's 2 KB metadata block when either slab runs
+// on the sparse MMA (the metadata columns it fills in TMEM serve both slabs).
 struct Chunk {
     uint32_t d[2];  // gemm-table records of the chunk's slabs
     int n;          // slabs in the chunk (1 or 2)
     __device__ __forceinline__ bool sparse() const {
         return ((d[0] | (n > 1 ? d[1] : 0u)) & kSlabSparse) != 0;
     }
-    __device__ __forceinline__ uint32_t recs() const { return rec_bytes(d[0]) + (n > 1 ? rec_bytes(d[1]) : 0u); }
-    __device__ __forceinline__ uint32_t bytes() const { return recs() + (sparse() ? (uint32_t)kMetaBytes : 0u); }
+    // record bytes of slabs [f, f + m)
+    __device__ __forceinline__ uint32_t recs(int f, int m) const {
+        return rec_bytes(d[f]) + (m > 1 ? rec_bytes(d[f + 1]) : 0u);
+    }
+    __device__ __forceinline__ bool meta_in(int f) const { return f == 0 && sparse(); }
+    // this strip's bytes in the stage of slabs [f, f + m)
+    __device__ __forceinline__ uint32_t bytes(int f, int m) const {
+        return recs(f, m) + (meta_in(f) ? (uint32_t)kMetaBytes : 0u);
+    }
 };
 
 __device__ __forceinline__ Chunk load_chunk(const uint32_t* t, int c, int KB) {
@@ -130,7 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData);
+    uint32_t* tabs = reinterpret_cast<uint32_t*>(smem + kSmemData);  // [warp][kTabWords]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemData + kSmemTab);
     uint64_t* full = bars;                       // [kQ] leader: both CTAs' bytes of stage g (at g % kQ)
     uint64_t* empty = full + kQ;                 // [kQ] every CTA: stage g consumed by both issuers
     uint64_t* acc_full = empty + kQ;             // [2] both CTAs: accumulator h ready
@@ -183,9 +211,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int w_begin = a.work_off[cl];
     const int w_end = a.work_off[cl + 1];
+    // Warp-cooperative copy of n table entries into shared memory; returns the
+    // shared copy, or the global table itself when it does not fit.
+    auto stage_table = [&](uint32_t* dst, const uint32_t* src, int n) -> const uint32_t* {
+        if (n > kTabKB) return src;
+        for (int i = lane; i < n; i += 32) dst[i] = src[i];
+        return dst;
+    };
 
     if (warp < kProducers) {
-        if (lane == 0) {
+        {
             // ---------------- producers (both CTAs) ----------------
             // Every producer walks the whole stage sequence to place each stage
             // in the ring; it loads the stages g with g % kProducers == me.
@@ -204,15 +239,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = lu / a.MB, j = lu % a.MB;
                 const int KB = L.KB, KC = L.KC;
                 const int s0 = strip_of(c, 0, L.S), s1 = strip_of(c, 1, L.S);
-                const uint32_t* t0 = L.gemm + (size_t)s0 * KB;
-                const uint32_t* t1 = L.gemm + (size_t)s1 * KB;
-                const uint32_t* m0 = L.meta + (size_t)s0 * KC;
-                const uint32_t* m1 = L.meta + (size_t)s1 * KC;
+                uint32_t* tab = tabs + warp * kTabWords;
+                const uint32_t* t0 = stage_table(tab, L.gemm + (size_t)s0 * KB, KB);
+                const uint32_t* t1 = stage_table(tab + kTabKB, L.gemm + (size_t)s1 * KB, KB);
+                const uint32_t* m0 = stage_table(tab + 2 * kTabKB, L.meta + (size_t)s0 * KC, KB > kTabKB ? kTabKB + 1 : KC);
+                const uint32_t* m1 =
+                    stage_table(tab + 2 * kTabKB + kTabKB / 2, L.meta + (size_t)s1 * KC, KB > kTabKB ? kTabKB + 1 : KC);
+                __syncwarp();
                 const CUtensorMap* tm_x = &maps.x[l];
                 const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
-                for (int kc = 0; kc < KC; ++kc, ++g) {
+                for (int kc = 0, part = 0; lane == 0 && kc < KC; ++g) {
                     const Chunk k0 = load_chunk(t0, kc, KB), k1 = load_chunk(t1, kc, KB);
-                    const uint32_t size = k0.bytes() + k1.bytes() + (uint32_t)k0.n * kStageX;
+                    const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > kMaxStage;
+                    const int f = split ? part : 0, m = split ? 1 : k0.n;
+                    const int kc_now = kc;
+                    if (!split || part == 1) {
+                        ++kc;
+                        part = 0;
+                    } else {
+                        part = 1;
+                    }
+                    const uint32_t size = k0.bytes(f, m) + k1.bytes(f, m) + (uint32_t)m * kStageX;
                     const uint32_t off = ring.place(size);
                     hist[g % kQ] = ring.pos - size;
                     if (g % kProducers != me) continue;
@@ -235,32 +282,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t dst = smem_u32(smem) + off;
                     for (int h = 0; h < 2; ++h) {
                         const Chunk& k = h ? k1 : k0;
-                        const uint32_t mrow = (h ? m1 : m0)[kc];
                         // both slabs in one copy when their records are adjacent
                         // and of one kind (a 2:4 pair is one 128-row box, a dense
                         // pair one 256-row box)
-                        const bool joint = k.n == 2 && ((k.d[0] ^ k.d[1]) & kSlabSparse) == 0 &&
+                        const bool joint = m == 2 && ((k.d[0] ^ k.d[1]) & kSlabSparse) == 0 &&
                                            slab_offset_bytes(k.d[1]) == slab_offset_bytes(k.d[0]) + rec_bytes(k.d[0]);
                         if (joint) {
                             tma_load_2d_pair(dst, (k.d[0] & kSlabSparse) ? &maps.a16[l] : &maps.a32[l], bar, 0,
                                              (int)(slab_offset_bytes(k.d[0]) >> 7));
                         } else {
-                            for (int i = 0; i < k.n; ++i)
-                                tma_load_2d_pair(dst + (i ? rec_bytes(k.d[0]) : 0u),
-                                                 (k.d[i] & kSlabSparse) ? &maps.a8[l] : &maps.a16[l], bar, 0,
-                                                 (int)(slab_offset_bytes(k.d[i]) >> 7));
+                            for (int i = 0; i < m; ++i)
+                                tma_load_2d_pair(dst + (i ? rec_bytes(k.d[f]) : 0u),
+                                                 (k.d[f + i] & kSlabSparse) ? &maps.a8[l] : &maps.a16[l], bar, 0,
+                                                 (int)(slab_offset_bytes(k.d[f + i]) >> 7));
                         }
-                        if (k.sparse()) tma_load_2d_pair(dst + k.recs(), &maps.e[l], bar, 0, (int)(mrow >> 3));
-                        dst += k.bytes();
+                        if (k.meta_in(f))
+                            tma_load_2d_pair(dst + k.recs(f, m), &maps.e[l], bar, 0, (int)((h ? m1 : m0)[kc_now] >> 3));
+                        dst += k.bytes(f, m);
                     }
-                    for (int i = 0; i < k0.n; ++i) tma_load_2d_pair(dst + i * kStageX, tm_x, bar, (2 * kc + i) * kSlabK, tok);
+                    for (int i = 0; i < m; ++i)
+                        tma_load_2d_pair(dst + i * kStageX, tm_x, bar, (2 * kc_now + f + i) * kSlabK, tok);
                     my_last = g;
                 }
+                // the whole warp moves on to the next tile (or stops) with lane 0
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                __syncwarp();
             }
-            if (pr == 0) {
-                // Bounded wait for the loads of my last stages, whatever the
-                // abort flag says, so none lands after the cluster exits.
-                for (int gg = my_last - kQ + 1; gg <= my_last; ++gg) {
+            if (pr == 0 && lane == 0) {
+                // Bounded wait for the loads of my stages among the last kQ of
+                // the sequence, whatever the abort flag says, so none lands
+                // after the cluster exits. (Earlier stages were consumed before
+                // the ring bytes were reused, and no stage gg + kQ exists to
+                // have moved the barrier past the phase waited for.)
+                for (int gg = g - kQ; gg <= my_last; ++gg) {
                     if (gg < 0 || gg % kProducers != me) continue;
                     const uint64_t t0 = globaltimer();
                     while (!mbar_try_wait(&full[gg % kQ], (uint32_t)((gg / kQ) & 1)) &&
@@ -270,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp < kMmaWarp + kMmaWarps) {
-        if (lane == 0 && pr == 0) {
+        if (pr == 0) {
             // ---------------- MMA issuers (leader CTA), one per strip pair ----------------
             // Both read every stage; a stage's ring bytes are free once both
             // have committed it. Two issuing threads keep the tensor pipe fed
@@ -289,49 +343,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = lu / a.MB, j = lu % a.MB;
                 const int KB = L.KB, KC = L.KC;
                 // both strip pairs' records place the stage in the ring
-                const uint32_t* t0 = L.gemm + (size_t)strip_of(c, 0, L.S) * KB;
-                const uint32_t* t1 = L.gemm + (size_t)strip_of(c, 1, L.S) * KB;
-                const int nt = tile_tokens(j, a.M);
-                const uint32_t idesc_d = idesc_bf16(256, nt, false);
-                const uint32_t idesc_s = idesc_bf16(256, nt, true);
-                Chunk k0 = load_chunk(t0, 0, KB), k1 = load_chunk(t1, 0, KB);
-                if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
-                    raise();
-                    break;
-                }
-                tc_fence_after();
-                for (int kc = 0; kc < KC; ++kc, ++g) {
-                    if (!mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
+                uint32_t* tab = tabs + warp * kTabWords;
+                const uint32_t* t0 = stage_table(tab, L.gemm + (size_t)strip_of(c, 0, L.S) * KB, KB);
+                const uint32_t* t1 = stage_table(tab + kTabKB, L.gemm + (size_t)strip_of(c, 1, L.S) * KB, KB);
+                __syncwarp();
+                if (lane == 0) {
+                    const int nt = tile_tokens(j, a.M);
+                    const uint32_t idesc_d = idesc_bf16(256, nt, false);
+                    const uint32_t idesc_s = idesc_bf16(256, nt, true);
+                    Chunk k0 = load_chunk(t0, 0, KB), k1 = load_chunk(t1, 0, KB);
+                    if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
                         raise();
                         ok = false;
-                        break;
                     }
-                    // next chunk's records, read while this one's MMAs issue
-                    Chunk n0, n1;
-                    if (kc + 1 < KC) {
-                        n0 = load_chunk(t0, kc + 1, KB);
-                        n1 = load_chunk(t1, kc + 1, KB);
+                    tc_fence_after();
+                    for (int kc = 0, part = 0; ok && kc < KC; ++g) {
+                        if (!mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
+                            raise();
+                            ok = false;
+                            break;
+                        }
+                        const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > kMaxStage;
+                        const int f = split ? part : 0, m = split ? 1 : k0.n;
+                        const bool last_of_chunk = !split || part == 1;
+                        // next chunk's records, read while this stage's MMAs issue
+                        Chunk n0 = k0, n1 = k1;
+                        if (last_of_chunk && kc + 1 < KC) {
+                            n0 = load_chunk(t0, kc + 1, KB);
+                            n1 = load_chunk(t1, kc + 1, KB);
+                        }
+                        const uint32_t b0 = k0.bytes(f, m), b1 = k1.bytes(f, m);
+                        const uint32_t base = smem_u32(smem) + ring.place(b0 + b1 + (uint32_t)m * kStageX);
+                        const Chunk& k = h ? k1 : k0;
+                        const uint32_t a_addr = base + (h ? b0 : 0u);
+                        const uint32_t b_addr = base + b0 + b1;
+                        if (k.meta_in(f)) cp2_128x128b(e_col, smem_desc(a_addr + k.recs(f, m), 16, 128, kLayoutNone));
+                        issue_slab(k.d[f], f, kc == 0 && f == 0, a_addr, b_addr, d_tmem, e_col, idesc_d, idesc_s);
+                        if (m > 1)
+                            issue_slab(k.d[1], 1, false, a_addr + rec_bytes(k.d[0]), b_addr + kStageX, d_tmem, e_col,
+                                       idesc_d, idesc_s);
+                        any_mma = true;
+                        commit2_mask(&empty[g % kQ], 3);
+                        if (last_of_chunk) {
+                            ++kc;
+                            part = 0;
+                            k0 = n0;
+                            k1 = n1;
+                        } else {
+                            part = 1;
+                        }
                     }
-                    const uint32_t base = smem_u32(smem) + ring.place(k0.bytes() + k1.bytes() + (uint32_t)k0.n * kStageX);
-                    const Chunk& k = h ? k1 : k0;
-                    const uint32_t a_addr = base + (h ? k0.bytes() : 0u);
-                    const uint32_t b_addr = base + k0.bytes() + k1.bytes();
-                    if (k.sparse()) cp2_128x128b(e_col, smem_desc(a_addr + k.recs(), 16, 128, kLayoutNone));
-                    issue_slab(k.d[0], 0, kc == 0, a_addr, b_addr, d_tmem, e_col, idesc_d, idesc_s);
-                    if (k.n > 1)
-                        issue_slab(k.d[1], 1, false, a_addr + rec_bytes(k.d[0]), b_addr + kStageX, d_tmem, e_col,
-                                   idesc_d, idesc_s);
-                    any_mma = true;
-                    commit2_mask(&empty[g % kQ], 3);
-                    if (kc + 1 < KC) {
-                        k0 = n0;
-                        k1 = n1;
-                    }
+                    if (ok) commit2_mask(&acc_full[h], 3);
                 }
-                if (!ok) break;
-                commit2_mask(&acc_full[h], 3);
+                // the whole warp moves on to the next tile (or stops) with lane 0
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                __syncwarp();
             }
-            if (*abort_flag && any_mma) {
+            if (lane == 0 && *abort_flag && any_mma) {
                 commit2_local(&drain[h]);
                 const uint64_t t0 = globaltimer();
                 while (!mbar_try_wait(&drain[h], 0) && globaltimer() - t0 < kWaitLimitNs) {
