@@ -67,6 +67,7 @@ MEASURED_TRAFFIC = {
 }
 KERNEL_NAMES = {4: "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
                 6: "hybrid_gemm22_kernel (CTA pair, two strips per CTA, 512x240 tiles)",
+                7: "hybrid_gemm22_kernel (CTA pair, two strips per CTA, 512x240 tiles; pure 2:4 instance)",
                 3: "hybrid_gemm_kernel (single CTA, 128x128 tiles)"}
 
 

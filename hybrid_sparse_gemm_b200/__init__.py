@@ -29,6 +29,7 @@ STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_ARG", 2: "PATCH_ERR_SHAPE", 3: "PAT
                 4: "PATCH_ERR_MASK", 5: "PATCH_ERR_CUDA", 6: "PATCH_ERR_TIMEOUT",
                 7: "PATCH_ERR_NOMEM", 8: "PATCH_ERR_UNSUPPORTED"}
 PATH_AUTO, PATH_GEMM, PATH_GEMV, PATH_GEMM_SINGLE, PATH_GEMM_PAIR, PATH_GEMV_SIMT, PATH_GEMM_WIDE = 0, 1, 2, 3, 4, 5, 6
+PATH_GEMM_WIDE_24 = 7
 
 EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",

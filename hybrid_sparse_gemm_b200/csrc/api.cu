@@ -287,6 +287,7 @@ struct patch_group_s {
     int parts[kMaxGroup] = {};    // decode K-parts per strip of each member in this group
     LinDesc* lins_dev = nullptr;  // n descriptors
     int* status_dev = nullptr;    // the first member's status word
+    bool pure24 = false;          // every slab of every member runs on the sparse MMA
     std::mutex mu;
     std::mutex host_mu;           // serialises patch_group_linear_host calls on the host
     std::map<std::pair<int, int>, WorkList> work;  // (kernel, m_blocks or 0) -> schedule
@@ -387,6 +388,9 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     g->dev = hs[0]->dev;
     g->n = n;
     g->status_dev = hs[0]->status_dev;
+    g->pure24 = true;
+    for (int i = 0; i < n; ++i)
+        g->pure24 = g->pure24 && hs[i]->plan.pair_sparse == (int64_t)hs[i]->plan.S * hs[i]->plan.KB;
     LinDesc d[kMaxGroup];
     // Decode units: a lone linear keeps its own split (enough units for every
     // SM); in a group the members' units already fill the GPU, so parts are
@@ -617,14 +621,19 @@ patch_status check_device_is(int device) {
 // when the launch has enough strip quads to keep every CTA pair busy (it
 // feeds each activation tile to twice the weight rows, but a small weight
 // gives it half as many work units as the one-strip pair kernel).
+// The wide kernel runs its pure 2:4 instance (GEMM_WIDE_24) when every slab
+// of every member runs on the sparse MMA.
 int resolve_path(patch_group g, int path, int64_t M) {
     if (path == PATCH_PATH_AUTO) path = (M <= kDecodeBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
-    if (path != PATCH_PATH_GEMM) return path;
-    if (M < kPairMinM) return PATCH_PATH_GEMM_SINGLE;
-    int64_t quads = 0;
-    for (int l = 0; l < g->n; ++l) quads += (g->h[l]->plan.S + 3) / 4;
-    const int64_t units = quads * ((M + kGemm22BN - 1) / kGemm22BN);
-    return units >= 2 * (int64_t)g->dev.wide_clusters ? PATCH_PATH_GEMM_WIDE : PATCH_PATH_GEMM_PAIR;
+    if (path == PATCH_PATH_GEMM) {
+        if (M < kPairMinM) return PATCH_PATH_GEMM_SINGLE;
+        int64_t quads = 0;
+        for (int l = 0; l < g->n; ++l) quads += (g->h[l]->plan.S + 3) / 4;
+        const int64_t units = quads * ((M + kGemm22BN - 1) / kGemm22BN);
+        path = units >= 2 * (int64_t)g->dev.wide_clusters ? PATCH_PATH_GEMM_WIDE : PATCH_PATH_GEMM_PAIR;
+    }
+    if (path == PATCH_PATH_GEMM_WIDE && g->pure24) return PATCH_PATH_GEMM_WIDE_24;
+    return path;
 }
 
 patch_status run_simt(patch_handle h, const void* X, int64_t M, void* Y, cudaStream_t st) {
@@ -651,7 +660,7 @@ int choose_kernel(patch_group g, int path) {
     (void)g;
     if (path == PATCH_PATH_GEMM_SINGLE) return 0;
     if (path == PATCH_PATH_GEMV) return 2;
-    if (path == PATCH_PATH_GEMM_WIDE) return 4;
+    if (path == PATCH_PATH_GEMM_WIDE || path == PATCH_PATH_GEMM_WIDE_24) return 4;
     return 1;
 }
 
@@ -668,8 +677,10 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
         return PATCH_OK;
     }
     if (path != PATCH_PATH_GEMV && path != PATCH_PATH_GEMM_SINGLE && path != PATCH_PATH_GEMM_PAIR &&
-        path != PATCH_PATH_GEMM_WIDE)
+        path != PATCH_PATH_GEMM_WIDE && path != PATCH_PATH_GEMM_WIDE_24)
         return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path == PATCH_PATH_GEMM_WIDE_24 && !g->pure24)
+        return fail(PATCH_ERR_ARG, "GEMM_WIDE_24 needs every slab of every member to be 2:4 in both strips of its pair");
     if (path == PATCH_PATH_GEMV && M > kDecodeBN)
         return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
@@ -717,7 +728,7 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
     a.status = g->status_dev;
     cudaError_t e = kernel == 0   ? launch_gemm(maps, a, grid, st)
                     : kernel == 1 ? launch_gemm2(maps, a, grid, st)
-                    : kernel == 4 ? launch_gemm22(maps, a, grid, st)
+                    : kernel == 4 ? launch_gemm22(maps, a, grid, path == PATCH_PATH_GEMM_WIDE_24, st)
                                   : launch_decode(maps, a, grid, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return PATCH_OK;
@@ -977,7 +988,7 @@ patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, vo
                                void* stream) {
     if (!h) return fail(PATCH_ERR_ARG, "handle is NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE_24) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     patch_status st = check_xy(X_bf16, Y_bf16);
     if (st != PATCH_OK) return st;
@@ -1049,7 +1060,7 @@ patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, 
     if (!g) return fail(PATCH_ERR_ARG, "group is NULL");
     if (!X || !Y) return fail(PATCH_ERR_ARG, "X and Y arrays must be non-NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE_24) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (M == 0) return PATCH_OK;
     for (int l = 0; l < g->n; ++l) {
         patch_status st = check_xy(X[l], Y[l]);
@@ -1063,7 +1074,7 @@ patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, 
 patch_status patch_group_path(patch_group g, int64_t M, int path, int* out) {
     if (!g || !out) return fail(PATCH_ERR_ARG, "group and out must be non-NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE_24) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     *out = resolve_path(g, path, M);
     return PATCH_OK;
 }
@@ -1075,7 +1086,7 @@ patch_status patch_group_linear_host(patch_group g, const void* const* X_host, i
     if (!g) return fail(PATCH_ERR_ARG, "group is NULL");
     if (!X_host || !Y_host) return fail(PATCH_ERR_ARG, "X and Y arrays must be non-NULL");
     if (M < 0) return fail(PATCH_ERR_ARG, "M must be >= 0");
-    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE) return fail(PATCH_ERR_ARG, "unknown path %d", path);
+    if (path < PATCH_PATH_AUTO || path > PATCH_PATH_GEMM_WIDE_24) return fail(PATCH_ERR_ARG, "unknown path %d", path);
     for (int l = 0; l < g->n; ++l)
         if (!X_host[l] || !Y_host[l]) return fail(PATCH_ERR_ARG, "member %d: X and Y must be non-NULL", l);
     if (M == 0) return PATCH_OK;
@@ -1138,7 +1149,7 @@ patch_status patch_group_linear_host(patch_group g, const void* const* X_host, i
     // chunks are whole multiples of its token tile, so each output element
     // comes from the same MMA sequence: the bits equal patch_group_linear's.
     const int rpath = resolve_path(g, path, M);
-    const int64_t bn = rpath == PATCH_PATH_GEMM_WIDE   ? kGemm22BN
+    const int64_t bn = (rpath == PATCH_PATH_GEMM_WIDE || rpath == PATCH_PATH_GEMM_WIDE_24) ? kGemm22BN
                        : rpath == PATCH_PATH_GEMM_PAIR ? kGemm2BN
                        : rpath == PATCH_PATH_GEMM_SINGLE ? kGemmBN
                                                          : M;

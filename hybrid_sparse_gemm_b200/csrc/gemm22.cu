@@ -54,15 +54,15 @@ static_assert(kRing % 1024 == 0 && kStageX % 1024 == 0 && kMetaBytes % 1024 == 0
               "every record starts 1024-byte aligned (128-byte swizzle atoms)");
 static_assert(kRing / kMinStage + 2 <= kQ, "stages in flight stay within the barrier window");
 static_assert(kMaxStage >= 2 * (2 * kSparseValBytes + kMetaBytes) + 2 * kStageX, "two 2:4 slabs form one stage");
-// Each producer and issuer warp copies the slab records (and, for producers,
-// the metadata block offsets) of its current tile's two strips into shared
-// memory, so that no stage waits on a table read from L2. Weights with more
-// than kTabKB slabs per strip read the tables from global memory instead.
+// Each producer warp copies the slab records and metadata block offsets of
+// its current tile's two strips into shared memory, so that no stage waits
+// on a table read from L2. Weights with more than kTabKB slabs per strip read
+// the tables from global memory instead.
 constexpr int kTabKB = 256;                     // K up to 16384
 constexpr int kTabWords = 2 * kTabKB + 2 * (kTabKB / 2);
 constexpr int kSmemData = kRing;
-constexpr int kSmemTab = (kProducers + kMmaWarps) * kTabWords * 4;
-constexpr int kSmemBytes = kSmemData + kSmemTab + 1024 + 256;
+constexpr int kSmemTab = kProducers * kTabWords * 4;
+constexpr int kSmemBytes = kSmemData + kSmemTab + 1024 + 512;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB of shared memory a CTA may use");
 constexpr int kAcc1 = 256;                      // first column of accumulator 1
 constexpr int kECol0 = kBN;                     // metadata columns of strip pair 0
@@ -89,29 +89,63 @@ __device__ __forceinline__ uint32_t rec_bytes(uint32_t d) {
 // chunk's first slab, the chunk's 2 KB metadata block when either slab runs
 // on the sparse MMA (the metadata columns it fills in TMEM serve both slabs).
 struct Chunk {
-    uint32_t d[2];  // gemm-table records of the chunk's slabs
-    int n;          // slabs in the chunk (1 or 2)
+    uint32_t d0, d1;  // gemm-table records of the chunk's slabs
+    int n;            // slabs in the chunk (1 or 2)
+    __device__ __forceinline__ uint32_t rec(int i) const { return i ? d1 : d0; }
     __device__ __forceinline__ bool sparse() const {
-        return ((d[0] | (n > 1 ? d[1] : 0u)) & kSlabSparse) != 0;
+        return ((d0 | (n > 1 ? d1 : 0u)) & kSlabSparse) != 0;
     }
     // record bytes of slabs [f, f + m)
     __device__ __forceinline__ uint32_t recs(int f, int m) const {
-        return rec_bytes(d[f]) + (m > 1 ? rec_bytes(d[f + 1]) : 0u);
+        return m > 1 ? rec_bytes(d0) + rec_bytes(d1) : rec_bytes(rec(f));
     }
     __device__ __forceinline__ bool meta_in(int f) const { return f == 0 && sparse(); }
     // this strip's bytes in the stage of slabs [f, f + m)
     __device__ __forceinline__ uint32_t bytes(int f, int m) const {
         return recs(f, m) + (meta_in(f) ? (uint32_t)kMetaBytes : 0u);
     }
+    // kinds of this strip's slabs in the stage: bit 0 first slab 2:4, bit 1
+    // second slab 2:4, bit 2 the chunk's metadata block is in the stage
+    __device__ __forceinline__ uint32_t kinds(int f, int m) const {
+        return (rec(f) & kSlabSparse) | (m > 1 ? (d1 & kSlabSparse) << 1 : 0u) | (meta_in(f) ? 4u : 0u);
+    }
 };
 
 __device__ __forceinline__ Chunk load_chunk(const uint32_t* t, int c, int KB) {
     Chunk k;
     k.n = (2 * c + 1 < KB) ? 2 : 1;
-    k.d[0] = t[2 * c];
-    k.d[1] = k.n > 1 ? t[2 * c + 1] : 0u;
+    k.d0 = t[2 * c];
+    k.d1 = k.n > 1 ? t[2 * c + 1] : 0u;
     return k;
 }
+
+// A weight whose every slab runs on the sparse MMA (a pure 2:4 weight, the
+// MaskLLM end of the hybrid range) has a packed layout with no dense records
+// and no dense images: strip s's compressed slab b sits at (s*KB + b) * 8 KB,
+// and the metadata block of its chunk c right after all values, at
+// S*KB*8 KB + (s*KC + c) * 2 KB. The kernel instance for such weights
+// computes the records instead of reading the tables.
+__device__ __forceinline__ Chunk pure_chunk(int s, int c, int KB) {
+    Chunk k;
+    k.n = (2 * c + 1 < KB) ? 2 : 1;
+    const uint32_t v = (uint32_t)(((size_t)s * KB + 2 * c) * (kSparseValBytes / 16));
+    k.d0 = (v << 2) | kSlabSparse;
+    k.d1 = k.n > 1 ? ((v + kSparseValBytes / 16) << 2) | kSlabSparse : 0u;
+    return k;
+}
+__device__ __forceinline__ uint32_t pure_meta(int S, int KB, int KC, int s, int c) {
+    return (uint32_t)(((size_t)S * KB * kSparseValBytes + ((size_t)s * KC + c) * kMetaBytes) / 16);
+}
+
+// What the MMA issuers need of a stage, written by the leader CTA's producer
+// that loads it, before the stage's loads are counted on its full barrier
+// (so the issuers' wait on that barrier also orders this read):
+//   x ring offset, y bytes of strip pair 0's part | strip pair 1's << 16,
+//   z kinds of strip pair 0 | strip pair 1's << 8, w slabs (1 or 2) | first
+//   slab's half of the chunk << 2 | first stage of the tile << 3 | last << 4.
+struct StageDesc {
+    uint32_t off, bytes, kinds, flags;
+};
 
 // Stages are placed one after another in a ring of kRing bytes; a stage that
 // does not fit before the end starts again at 0. `pos` counts bytes placed so
@@ -152,6 +186,7 @@ __device__ __forceinline__ void issue_slab(uint32_t d, int half, bool first, uin
     }
 }
 
+template <bool kPure24>
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_gemm22_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -164,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* acc_full = empty + kQ;             // [2] both CTAs: accumulator h ready
     uint64_t* acc_empty = acc_full + 2;          // [2] leader: the 16 epilogue warps of accumulator h drained it
     uint64_t* drain = acc_empty + 2;             // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+    StageDesc* sdesc = reinterpret_cast<StageDesc*>(drain + 2);  // [kQ] leader: stage g at g % kQ
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sdesc + kQ);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -240,16 +276,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int KB = L.KB, KC = L.KC;
                 const int s0 = strip_of(c, 0, L.S), s1 = strip_of(c, 1, L.S);
                 uint32_t* tab = tabs + warp * kTabWords;
-                const uint32_t* t0 = stage_table(tab, L.gemm + (size_t)s0 * KB, KB);
-                const uint32_t* t1 = stage_table(tab + kTabKB, L.gemm + (size_t)s1 * KB, KB);
-                const uint32_t* m0 = stage_table(tab + 2 * kTabKB, L.meta + (size_t)s0 * KC, KB > kTabKB ? kTabKB + 1 : KC);
-                const uint32_t* m1 =
-                    stage_table(tab + 2 * kTabKB + kTabKB / 2, L.meta + (size_t)s1 * KC, KB > kTabKB ? kTabKB + 1 : KC);
-                __syncwarp();
+                const uint32_t *t0 = nullptr, *t1 = nullptr, *m0 = nullptr, *m1 = nullptr;
+                if (!kPure24) {
+                    t0 = stage_table(tab, L.gemm + (size_t)s0 * KB, KB);
+                    t1 = stage_table(tab + kTabKB, L.gemm + (size_t)s1 * KB, KB);
+                    m0 = stage_table(tab + 2 * kTabKB, L.meta + (size_t)s0 * KC, KB > kTabKB ? kTabKB + 1 : KC);
+                    m1 = stage_table(tab + 2 * kTabKB + kTabKB / 2, L.meta + (size_t)s1 * KC,
+                                     KB > kTabKB ? kTabKB + 1 : KC);
+                    __syncwarp();
+                }
                 const CUtensorMap* tm_x = &maps.x[l];
                 const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
                 for (int kc = 0, part = 0; lane == 0 && kc < KC; ++g) {
-                    const Chunk k0 = load_chunk(t0, kc, KB), k1 = load_chunk(t1, kc, KB);
+                    const Chunk k0 = kPure24 ? pure_chunk(s0, kc, KB) : load_chunk(t0, kc, KB);
+                    const Chunk k1 = kPure24 ? pure_chunk(s1, kc, KB) : load_chunk(t1, kc, KB);
                     const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > kMaxStage;
                     const int f = split ? part : 0, m = split ? 1 : k0.n;
                     const int kc_now = kc;
@@ -278,26 +318,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     const uint32_t bar = map_to_rank(smem_u32(&full[g % kQ]), 0);
-                    if (pr == 0) mbar_arrive_expect_tx(&full[g % kQ], 2u * size);
+                    if (pr == 0) {
+                        StageDesc sd;
+                        sd.off = off;
+                        sd.bytes = k0.bytes(f, m) | (k1.bytes(f, m) << 16);
+                        sd.kinds = k0.kinds(f, m) | (k1.kinds(f, m) << 8);
+                        sd.flags = (uint32_t)m | ((uint32_t)f << 2) | ((kc_now == 0 && f == 0) ? 8u : 0u) |
+                                   (kc >= KC ? 16u : 0u);
+                        sdesc[g % kQ] = sd;
+                        mbar_arrive_expect_tx(&full[g % kQ], 2u * size);
+                    }
                     uint32_t dst = smem_u32(smem) + off;
+#pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const Chunk& k = h ? k1 : k0;
+                        const Chunk k = h ? k1 : k0;
+                        const uint32_t da = k.rec(f), db = k.d1;
                         // both slabs in one copy when their records are adjacent
                         // and of one kind (a 2:4 pair is one 128-row box, a dense
                         // pair one 256-row box)
-                        const bool joint = m == 2 && ((k.d[0] ^ k.d[1]) & kSlabSparse) == 0 &&
-                                           slab_offset_bytes(k.d[1]) == slab_offset_bytes(k.d[0]) + rec_bytes(k.d[0]);
+                        const bool joint = m == 2 && ((da ^ db) & kSlabSparse) == 0 &&
+                                           slab_offset_bytes(db) == slab_offset_bytes(da) + rec_bytes(da);
                         if (joint) {
-                            tma_load_2d_pair(dst, (k.d[0] & kSlabSparse) ? &maps.a16[l] : &maps.a32[l], bar, 0,
-                                             (int)(slab_offset_bytes(k.d[0]) >> 7));
+                            tma_load_2d_pair(dst, (da & kSlabSparse) ? &maps.a16[l] : &maps.a32[l], bar, 0,
+                                             (int)(slab_offset_bytes(da) >> 7));
                         } else {
-                            for (int i = 0; i < m; ++i)
-                                tma_load_2d_pair(dst + (i ? rec_bytes(k.d[f]) : 0u),
-                                                 (k.d[f + i] & kSlabSparse) ? &maps.a8[l] : &maps.a16[l], bar, 0,
-                                                 (int)(slab_offset_bytes(k.d[f + i]) >> 7));
+                            tma_load_2d_pair(dst, (da & kSlabSparse) ? &maps.a8[l] : &maps.a16[l], bar, 0,
+                                             (int)(slab_offset_bytes(da) >> 7));
+                            if (m > 1)
+                                tma_load_2d_pair(dst + rec_bytes(da), (db & kSlabSparse) ? &maps.a8[l] : &maps.a16[l],
+                                                 bar, 0, (int)(slab_offset_bytes(db) >> 7));
                         }
-                        if (k.meta_in(f))
-                            tma_load_2d_pair(dst + k.recs(f, m), &maps.e[l], bar, 0, (int)((h ? m1 : m0)[kc_now] >> 3));
+                        if (k.meta_in(f)) {
+                            const uint32_t mrow =
+                                kPure24 ? pure_meta(L.S, KB, KC, h ? s1 : s0, kc_now) : (h ? m1 : m0)[kc_now];
+                            tma_load_2d_pair(dst + k.recs(f, m), &maps.e[l], bar, 0, (int)(mrow >> 3));
+                        }
                         dst += k.bytes(f, m);
                     }
                     for (int i = 0; i < m; ++i)
@@ -324,82 +379,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp < kMmaWarp + kMmaWarps) {
-        if (pr == 0) {
+        if (lane == 0 && pr == 0) {
             // ---------------- MMA issuers (leader CTA), one per strip pair ----------------
             // Both read every stage; a stage's ring bytes are free once both
             // have committed it. Two issuing threads keep the tensor pipe fed
-            // while either one waits on a barrier or computes descriptors.
+            // while either one waits on a barrier or computes descriptors. The
+            // stage layout comes from the descriptor its producer wrote.
             const int h = warp - kMmaWarp;
             const uint32_t d_tmem = tmem_base + (uint32_t)(h * kAcc1);
             const uint32_t e_col = tmem_base + (uint32_t)(h ? kECol1 : kECol0);
-            Ring ring;
+            const uint32_t ring0 = smem_u32(smem);
             int g = 0;
             bool ok = true, any_mma = false;
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
-                const int u = a.work[it];
-                const LinDesc& L = a.lins[u >> kUnitShift];
-                const int lu = u & kUnitMask;
-                const int c = lu / a.MB, j = lu % a.MB;
-                const int KB = L.KB, KC = L.KC;
-                // both strip pairs' records place the stage in the ring
-                uint32_t* tab = tabs + warp * kTabWords;
-                const uint32_t* t0 = stage_table(tab, L.gemm + (size_t)strip_of(c, 0, L.S) * KB, KB);
-                const uint32_t* t1 = stage_table(tab + kTabKB, L.gemm + (size_t)strip_of(c, 1, L.S) * KB, KB);
-                __syncwarp();
-                if (lane == 0) {
-                    const int nt = tile_tokens(j, a.M);
-                    const uint32_t idesc_d = idesc_bf16(256, nt, false);
-                    const uint32_t idesc_s = idesc_bf16(256, nt, true);
-                    Chunk k0 = load_chunk(t0, 0, KB), k1 = load_chunk(t1, 0, KB);
-                    if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
+                const int j = (a.work[it] & kUnitMask) % a.MB;
+                const int nt = tile_tokens(j, a.M);
+                const uint32_t idesc_d = idesc_bf16(256, nt, false);
+                const uint32_t idesc_s = idesc_bf16(256, nt, true);
+                if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
+                    raise();
+                    break;
+                }
+                tc_fence_after();
+                for (bool last = false; !last; ++g) {
+                    if (!mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
                         raise();
                         ok = false;
+                        break;
                     }
-                    tc_fence_after();
-                    for (int kc = 0, part = 0; ok && kc < KC; ++g) {
-                        if (!mbar_wait(&full[g % kQ], (uint32_t)((g / kQ) & 1), abort_flag)) {
-                            raise();
-                            ok = false;
-                            break;
-                        }
-                        const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > kMaxStage;
-                        const int f = split ? part : 0, m = split ? 1 : k0.n;
-                        const bool last_of_chunk = !split || part == 1;
-                        // next chunk's records, read while this stage's MMAs issue
-                        Chunk n0 = k0, n1 = k1;
-                        if (last_of_chunk && kc + 1 < KC) {
-                            n0 = load_chunk(t0, kc + 1, KB);
-                            n1 = load_chunk(t1, kc + 1, KB);
-                        }
-                        const uint32_t b0 = k0.bytes(f, m), b1 = k1.bytes(f, m);
-                        const uint32_t base = smem_u32(smem) + ring.place(b0 + b1 + (uint32_t)m * kStageX);
-                        const Chunk& k = h ? k1 : k0;
-                        const uint32_t a_addr = base + (h ? b0 : 0u);
-                        const uint32_t b_addr = base + b0 + b1;
-                        if (k.meta_in(f)) cp2_128x128b(e_col, smem_desc(a_addr + k.recs(f, m), 16, 128, kLayoutNone));
-                        issue_slab(k.d[f], f, kc == 0 && f == 0, a_addr, b_addr, d_tmem, e_col, idesc_d, idesc_s);
-                        if (m > 1)
-                            issue_slab(k.d[1], 1, false, a_addr + rec_bytes(k.d[0]), b_addr + kStageX, d_tmem, e_col,
-                                       idesc_d, idesc_s);
-                        any_mma = true;
-                        commit2_mask(&empty[g % kQ], 3);
-                        if (last_of_chunk) {
-                            ++kc;
-                            part = 0;
-                            k0 = n0;
-                            k1 = n1;
-                        } else {
-                            part = 1;
-                        }
-                    }
-                    if (ok) commit2_mask(&acc_full[h], 3);
+                    const StageDesc sd = sdesc[g % kQ];
+                    const uint32_t b0 = sd.bytes & 0xFFFFu, b1 = sd.bytes >> 16;
+                    const uint32_t kd = h ? (sd.kinds >> 8) & 0xFFu : sd.kinds & 0xFFu;
+                    const int m = (int)(sd.flags & 3u), f = (int)((sd.flags >> 2) & 1u);
+                    const bool first = (sd.flags & 8u) != 0;
+                    last = (sd.flags & 16u) != 0;
+                    const uint32_t a_addr = ring0 + sd.off + (h ? b0 : 0u);
+                    const uint32_t b_addr = ring0 + sd.off + b0 + b1;
+                    const uint32_t r0 = (kd & 1u) ? (uint32_t)kSparseValBytes : (uint32_t)kDenseSlabBytes;
+                    const uint32_t r1 = m > 1 ? ((kd & 2u) ? (uint32_t)kSparseValBytes : (uint32_t)kDenseSlabBytes) : 0u;
+                    if (kd & 4u) cp2_128x128b(e_col, smem_desc(a_addr + r0 + r1, 16, 128, kLayoutNone));
+                    issue_slab(kd & 1u, f, first, a_addr, b_addr, d_tmem, e_col, idesc_d, idesc_s);
+                    if (m > 1)
+                        issue_slab((kd >> 1) & 1u, 1, false, a_addr + r0, b_addr + kStageX, d_tmem, e_col, idesc_d,
+                                   idesc_s);
+                    any_mma = true;
+                    commit2_mask(&empty[g % kQ], 3);
                 }
-                // the whole warp moves on to the next tile (or stops) with lane 0
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                __syncwarp();
+                if (!ok) break;
+                commit2_mask(&acc_full[h], 3);
             }
-            if (lane == 0 && *abort_flag && any_mma) {
+            if (*abort_flag && any_mma) {
                 commit2_local(&drain[h]);
                 const uint64_t t0 = globaltimer();
                 while (!mbar_try_wait(&drain[h], 0) && globaltimer() - t0 < kWaitLimitNs) {
@@ -497,21 +527,24 @@ cudaLaunchConfig_t config(int clusters, cudaLaunchAttribute* attr, cudaStream_t 
 
 cudaError_t gemm_prepare_wide(int* max_clusters) {
     cudaError_t e =
-        cudaFuncSetAttribute(hybrid_gemm22_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(hybrid_gemm22_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(hybrid_gemm22_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr;
     cudaLaunchConfig_t cfg = config(1, &attr, nullptr);
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm22_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, hybrid_gemm22_kernel<false>, &cfg);
     if (e != cudaSuccess) return e;
     *max_clusters = n;
     return cudaSuccess;
 }
 
-cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st) {
+cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, bool pure24, cudaStream_t st) {
     cudaLaunchAttribute attr;
     cudaLaunchConfig_t cfg = config(clusters, &attr, st);
-    return cudaLaunchKernelEx(&cfg, hybrid_gemm22_kernel, maps, a);
+    return pure24 ? cudaLaunchKernelEx(&cfg, hybrid_gemm22_kernel<true>, maps, a)
+                  : cudaLaunchKernelEx(&cfg, hybrid_gemm22_kernel<false>, maps, a);
 }
 
 }  // namespace patch

@@ -75,7 +75,8 @@ struct GemvArgs {
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_gemm(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
-cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
+// pure24: every member's slabs all run on the sparse MMA (no tables read)
+cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, bool pure24, cudaStream_t st);
 cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 cudaError_t launch_selftest_wait(int* status, cudaStream_t st);

@@ -65,9 +65,10 @@ typedef enum {
 } patch_status;
 
 /* Which kernel patch_linear_path runs. AUTO picks by M: GEMV for M <= 16,
- * GEMM_SINGLE below M = 256, and above it GEMM_WIDE when the call (or group)
- * has at least two 512-row x 240-token tiles per co-resident CTA pair,
- * otherwise GEMM_PAIR. GEMM is AUTO restricted to the tensor-core GEMMs. */
+ * GEMM_SINGLE below M = 256, and above it GEMM_WIDE (GEMM_WIDE_24 for pure
+ * 2:4 weights) when the call (or group) has at least two 512-row x 240-token
+ * tiles per co-resident CTA pair, otherwise GEMM_PAIR. GEMM is AUTO
+ * restricted to the tensor-core GEMMs. */
 typedef enum {
     PATCH_PATH_AUTO = 0,
     PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core GEMM, variant chosen as for AUTO */
@@ -75,9 +76,15 @@ typedef enum {
     PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
     PATCH_PATH_GEMM_PAIR = 4,    /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
     PATCH_PATH_GEMV_SIMT = 5,    /* decode on CUDA cores (M <= 16), no workspace */
-    PATCH_PATH_GEMM_WIDE = 6     /* tcgen05 cta_group::2, two strips per CTA: one CTA pair
+    PATCH_PATH_GEMM_WIDE = 6,    /* tcgen05 cta_group::2, two strips per CTA: one CTA pair
                                     per 512-row x 240-token tile (each activation tile feeds
                                     both strip pairs); strips padded to a multiple of four */
+    PATCH_PATH_GEMM_WIDE_24 = 7  /* the GEMM_WIDE kernel's instance for pure 2:4 weights
+                                    (every slab of every member runs on the sparse MMA, the
+                                    MaskLLM end of the range): it computes each record's
+                                    place instead of reading the tables. GEMM_WIDE, GEMM and
+                                    AUTO run it whenever the weights allow; requesting it for
+                                    other weights gives PATCH_ERR_ARG */
 } patch_path;
 
 typedef struct {
@@ -316,7 +323,7 @@ patch_status patch_group_linear_host(patch_group g, const void* const* X, int64_
 
 /*
  * patch_group_path - the explicit path (GEMV, GEMV_SIMT, GEMM_SINGLE,
- * GEMM_PAIR or GEMM_WIDE) that patch_group_linear would run for this M and
+ * GEMM_PAIR, GEMM_WIDE or GEMM_WIDE_24) that patch_group_linear would run for this M and
  * requested path; nothing is launched. *out receives the value.
  * Errors: PATCH_ERR_ARG for a NULL group or out, M < 0 or an unknown path.
  */

@@ -502,6 +502,38 @@ def test_grouped_layer_as_benchmarked(hsg, oracle_lib, model, M):
         lin.free()
 
 
+@pytest.mark.parametrize("model,M,members", [("llama2_7b", 2048, None), ("llama2_13b", 8192, ["q", "up", "down"])])
+def test_pure_24_instance(hsg, oracle_lib, model, M, members):
+    """Pure 2:4 weights (every tile 2:4, the MaskLLM end of the range) run the
+    wide kernel's pure instance, which computes each record's place instead
+    of reading the tables: a Llama-2-7B layer at M = 2048 and Llama-2-13B
+    linears at M = 8192. AUTO picks it, an explicit request gives the same
+    bits, and sampled rows match the oracle."""
+    shapes = [l for l in getattr(synth, model)() if members is None or l.name in members]
+    X_by_k = {K: synth.normal_bf16((M, K), 1.0, "cuda", "pure", "X", 0, M, K) for K in sorted({l.K for l in shapes})}
+    probs = [synth.make_problem(l.N, l.K, 0, frac=1.0, seed=0, device="cuda", tag=f"pure-{model}-{l.name}")
+             for l in shapes]
+    lins = [pack(hsg, p) for p in probs]
+    for lin in lins:
+        info = lin.info()
+        assert info.slabs_pair_sparse == info.slabs_total and info.dense_images == 0
+        assert abs(info.sparsity - 0.5) < 1e-12
+    g = hsg.LinearGroup(lins)
+    assert g.path(M) == hsg.PATH_GEMM_WIDE_24
+    xs = [X_by_k[l.K] for l in shapes]
+    Ys = g(xs)
+    Ys2 = g(xs, path=hsg.PATH_GEMM_WIDE_24)
+    torch.cuda.synchronize()
+    lins[0].check()
+    assert all(torch.equal(a, b) for a, b in zip(Ys, Ys2))
+    rows = sample_rows(M, 48, 2)
+    for l, p, Y in zip(shapes, probs, Ys):
+        assert_close(Y, oracle_lib, X_by_k[l.K], p.W, p.bits, p.keep, rows=rows, what=f"{model} pure 2:4 {l.name}")
+    g.free()
+    for lin in lins:
+        lin.free()
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_config3_llama2_7b_decode(hsg, oracle_lib, M):
     shapes = synth.llama2_7b()
@@ -576,8 +608,16 @@ def test_group_path_choice(hsg):
     assert gb.path(4096) == hsg.PATH_GEMM_WIDE         # 16 quads x 18 token blocks
     assert gb.path(4096, hsg.PATH_GEMM_PAIR) == hsg.PATH_GEMM_PAIR
     assert gs.path(4, hsg.PATH_GEMV_SIMT) == hsg.PATH_GEMV_SIMT
-    for g in (gs, gb):
+    pure = pack(hsg, synth.make_problem(8192, 256, 0, frac=1.0, seed=3, device="cuda", tag="gp3"))
+    gp = hsg.LinearGroup([pure])
+    assert gp.path(4096) == hsg.PATH_GEMM_WIDE_24      # every slab 2:4: the pure instance
+    assert gp.path(4096, hsg.PATH_GEMM_WIDE) == hsg.PATH_GEMM_WIDE_24
+    assert gp.path(300, hsg.PATH_GEMM_PAIR) == hsg.PATH_GEMM_PAIR
+    with pytest.raises(hsg.PatchError):
+        gb([torch.empty((300, 256), dtype=torch.bfloat16, device="cuda")], path=hsg.PATH_GEMM_WIDE_24)
+    for g in (gs, gb, gp):
         g.free()
+    pure.free()
     small.free()
     big.free()
 
