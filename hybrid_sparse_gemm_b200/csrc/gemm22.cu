@@ -31,7 +31,7 @@ namespace patch {
 namespace {
 
 #ifndef PATCH_GEMM22_PRODUCERS
-#define PATCH_GEMM22_PRODUCERS 2
+#define PATCH_GEMM22_PRODUCERS 4
 #endif
 constexpr int kProducers = PATCH_GEMM22_PRODUCERS;  // TMA-issuing warps (stages dealt round robin)
 constexpr int kMmaWarp = kProducers;            // MMA issuers (leader CTA), one per strip pair;
@@ -42,18 +42,24 @@ constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBN = kGemm22BN;                  // tokens per tile (both CTAs)
 constexpr int kHalfN = kBN / 2;                 // token rows of operand B per CTA
 constexpr int kStageX = kHalfN * 128;           // 15 KB of activations per slab
-constexpr int kRing = 208896;                   // shared-memory ring the stages are placed in, in order
-constexpr int kQ = 8;                           // per-stage barriers: more than the stages that fit in the ring
-#ifndef PATCH_GEMM22_MAX_STAGE
-#define PATCH_GEMM22_MAX_STAGE 70 * 1024
+#ifndef PATCH_GEMM22_RING
+#define PATCH_GEMM22_RING 218112
 #endif
-constexpr uint32_t kMaxStage = PATCH_GEMM22_MAX_STAGE;  // larger two-slab stages are cut into one-slab stages
+constexpr int kRing = PATCH_GEMM22_RING;        // shared-memory ring the stages are placed in, in order
+constexpr int kQ = 8;                           // per-stage barriers: more than the stages that fit in the ring
+// Largest two-slab stage; larger ones are cut into one-slab stages. The pure
+// 2:4 instance keeps two-slab stages (66 KB); the general instance cuts every
+// chunk, which keeps six or more stages in flight to cover the load latency.
+constexpr uint32_t kMaxStagePure = 70 * 1024;
+#ifndef PATCH_GEMM22_MAX_STAGE
+#define PATCH_GEMM22_MAX_STAGE 40 * 1024
+#endif
+constexpr uint32_t kMaxStageMixed = PATCH_GEMM22_MAX_STAGE;
 // smallest stage: one 2:4 slab of each strip and its activation tile
 constexpr int kMinStage = 2 * kSparseValBytes + kStageX;
 static_assert(kRing % 1024 == 0 && kStageX % 1024 == 0 && kMetaBytes % 1024 == 0,
               "every record starts 1024-byte aligned (128-byte swizzle atoms)");
 static_assert(kRing / kMinStage + 2 <= kQ, "stages in flight stay within the barrier window");
-static_assert(kMaxStage >= 2 * (2 * kSparseValBytes + kMetaBytes) + 2 * kStageX, "two 2:4 slabs form one stage");
 // Each producer warp copies the slab records and metadata block offsets of
 // its current tile's two strips into shared memory, so that no stage waits
 // on a table read from L2. Weights with more than kTabKB slabs per strip read
@@ -82,8 +88,8 @@ __device__ __forceinline__ uint32_t rec_bytes(uint32_t d) {
 
 // A chunk is two 64-column slabs (one for an odd last chunk) of a strip. A
 // stage holds both strips' records of one chunk, or of one slab of it when
-// the two-slab stage would exceed kMaxStage (a chunk with dense records is
-// cut in two, so that enough stages fit in the ring to cover the load
+// the two-slab stage would exceed the instance's limit (kMaxStagePure or
+// kMaxStageMixed: more, smaller stages in the ring cover more of the load
 // latency), plus the activation tiles of those slabs. A strip's part of a
 // stage: its slab records back to back, then, in the stage that holds the
 // chunk's first slab, the chunk's 2 KB metadata block when either slab runs
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kc = 0, part = 0; lane == 0 && kc < KC; ++g) {
                     const Chunk k0 = kPure24 ? pure_chunk(s0, kc, KB) : load_chunk(t0, kc, KB);
                     const Chunk k1 = kPure24 ? pure_chunk(s1, kc, KB) : load_chunk(t1, kc, KB);
-                    const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > kMaxStage;
+                    const bool split = k0.n == 2 && k0.bytes(0, 2) + k1.bytes(0, 2) + 2 * kStageX > (kPure24 ? kMaxStagePure : kMaxStageMixed);
                     const int f = split ? part : 0, m = split ? 1 : k0.n;
                     const int kc_now = kc;
                     if (!split || part == 1) {
