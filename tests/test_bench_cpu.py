@@ -40,9 +40,13 @@ def test_peak_choice_and_roofline():
     of the step over the step time."""
     b = _bench()
     peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured", "hbm_gbs": 1.0}
-    assert b.choose_peak(peaks, 0.3, {"reasons": ["sw_power_cap"]})[0] == 1600.0
-    assert b.choose_peak(peaks, 5.0, {"reasons": []})[0] == 1600.0
-    assert b.choose_peak(peaks, 5.0, {"reasons": ["sw_power_cap"]})[0] == 1400.0
+    hi = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    lo = {"sm_mhz": 1515.0, "sm_max_mhz": 1965.0}
+    assert b.choose_peak(peaks, 0.3, dict(hi, reasons=["sw_power_cap"]))[0] == 1600.0
+    assert b.choose_peak(peaks, 5.0, dict(lo, reasons=[]))[0] == 1600.0
+    assert b.choose_peak(peaks, 5.0, dict(hi, reasons=["sw_power_cap"]))[0] == 1400.0
+    assert b.choose_peak(peaks, 0.3, dict(lo, reasons=["sw_power_cap"]))[0] == 1400.0
+    assert b.choose_peak(peaks, 0.3, {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]})[0] == 1600.0
 
     class Info:
         pruned, slabs_total, slabs_pair_sparse, packed_bytes = 64 * 128, 4, 1, 0
@@ -51,9 +55,10 @@ def test_peak_choice_and_roofline():
     m = b.Member(None, 256, 128, Info(), None, None)
     assert m.kept == 128 * 256 - 64 * 128 and m.executed == 3 * 8192 + 4096
     model = [(None, [m, m])]
-    r = b.roofline(model, 10, 2.0, 4, 1600.0, "burst", "k", None)
+    r = b.roofline(model, 10, 2.0, 4, 1600.0, "burst", "k", None, peaks)
     assert abs(r["achieved"] - 2 * 2.0 * 10 * m.kept / 2e-3 / 1e12) < 1e-12
     assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-15 and r["kernel_ms_per_launch"] == 0.5
+    assert abs(r["frac_of_sustained"] - r["achieved"] / 1400.0) < 1e-15
 
 
 def test_measured_traffic_is_pinned_to_source():
