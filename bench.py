@@ -58,12 +58,12 @@ import synth  # noqa: E402
 FRACS_SWEEP = [0.0, 0.5, 0.7, 0.9, 1.0]
 METRIC = "hybrid dense/2:4 GEMM dense-equiv TFLOP/s and speedup vs dense bf16, per sparsity"
 # DRAM bytes (read + write) of one launch of a kernel on the default workload
-# (one Llama-3.2-1B layer, M = 4096, 90 % 2:4 tiles), from an ncu capture, with
+# (one Llama-2-7B layer, M = 2048, 90 % 2:4 tiles), from an ncu capture, with
 # the sha256 prefix of the kernel source it was taken on: reported only while
 # that source is unchanged.
 MEASURED_TRAFFIC = {
-    "hybrid_gemm22_kernel": {"source": "hybrid_sparse_gemm_b200/csrc/gemm22.cu", "sha256": "fab2917e4fbf7991",
-                             "workload": ("llama32-1b", 4096, "128x128"), "bytes_per_launch": 407.99e6},
+    "hybrid_gemm22_kernel": {"source": "hybrid_sparse_gemm_b200/csrc/gemm22.cu", "sha256": "f2c71c3aed83f010",
+                             "workload": ("llama2-7b", 2048, "128x128"), "bytes_per_launch": 658.78e6},
 }
 KERNEL_NAMES = {4: "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
                 6: "hybrid_gemm22_kernel (CTA pair, two strips per CTA, 512x240 tiles)",
@@ -71,7 +71,7 @@ KERNEL_NAMES = {4: "hybrid_gemm2_kernel (CTA pair, 256x256 tiles)",
                 3: "hybrid_gemm_kernel (single CTA, 128x128 tiles)"}
 
 
-def measured_traffic(kernel_name: str, workload=("llama32-1b", 4096, "128x128")):
+def measured_traffic(kernel_name: str, workload=("llama2-7b", 2048, "128x128")):
     """ncu DRAM bytes per launch for this kernel on this workload, or None if
     none was taken on the current source."""
     import hashlib

@@ -69,7 +69,7 @@ def test_measured_traffic_is_pinned_to_source():
             same = hashlib.sha256(f.read()).hexdigest()[:16] == t["sha256"]
         got = b.measured_traffic(name + " (any label)", t["workload"])
         assert (got == t["bytes_per_launch"]) if same else (got is None)
-        assert b.measured_traffic(name, ("llama2-7b", 2048, "128x128")) is None
+        assert b.measured_traffic(name, ("llama32-1b", 4096, "128x128")) is None
     assert b.measured_traffic("some_other_kernel") is None
 
 
