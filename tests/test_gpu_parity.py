@@ -232,6 +232,20 @@ def test_wide_long_k(hsg, oracle_lib):
     lin.free()
 
 
+@pytest.mark.parametrize("frac", [0.6, 1.0])
+def test_wide_tables_beyond_shared_copy(hsg, oracle_lib, frac):
+    """K = 16448 (257 slabs per strip): more records than the producers copy
+    into shared memory, so the general instance reads its tables from global
+    memory; the pure 2:4 instance computes them. A K % 128 == 64 tail too."""
+    p = synth.make_problem(512, 16448, 300, R=128, C=64, frac=frac, seed=13, device="cuda", tag="widetab")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMM_WIDE)
+    torch.cuda.synchronize()
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=sample_rows(300, 24, 6), what=f"wide K=16448 f={frac}")
+    lin.free()
+
+
 def test_single_strip_single_slab(hsg, oracle_lib):
     for frac in (0.0, 1.0):
         p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")
