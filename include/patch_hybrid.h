@@ -213,8 +213,9 @@ patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flag
  * asynchronously on `stream` (it allocates device and pinned host memory);
  * a call on another stream waits for that upload on the device. The first
  * uncaptured decode call (M <= 16) on a stream allocates that stream's
- * workspace. Before capturing later calls in a CUDA graph, make one call
- * with the same M and let it complete.
+ * workspace (a few MB, held until the handle or group is freed). Before
+ * capturing later calls in a CUDA graph, make one call with the same M and
+ * let it complete.
  */
 patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                           void* stream);
