@@ -274,6 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int g = 0;
             int my_last = -1;    // sequence index of the last stage this producer loaded
             bool ok = true;
+            // every strip quad of a member reads the same activation tiles, so
+            // they are kept in L2 over the weight records (each read by one
+            // wave of token tiles)
+            const uint64_t pol_x = policy_evict_last();
             for (int it = w_begin; it < w_end && ok; ++it) {
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         dst += k.bytes(f, m);
                     }
                     for (int i = 0; i < m; ++i)
-                        tma_load_2d_pair(dst + i * kStageX, tm_x, bar, (2 * kc_now + f + i) * kSlabK, tok);
+                        tma_load_2d_pair_hint(dst + i * kStageX, tm_x, bar, (2 * kc_now + f + i) * kSlabK, tok, pol_x);
                     my_last = g;
                 }
                 // the whole warp moves on to the next tile (or stops) with lane 0
