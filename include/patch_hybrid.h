@@ -318,6 +318,8 @@ patch_status patch_group_linear(patch_group g, const void* const* X, int64_t M, 
  * buffers (grown on demand: the first call for a larger M allocates and
  * waits for the group's previous host call). Calls on one group are ordered
  * among themselves on the device; issue them from one host thread at a time.
+ * A call that fails part-way may have enqueued some copies: synchronise
+ * `stream` before the next call on the group.
  */
 patch_status patch_group_linear_host(patch_group g, const void* const* X, int64_t M, void* const* Y,
                                      int path, void* stream);
