@@ -28,7 +28,8 @@ Reported (one JSON line from rank 0):
                inside the timed region)
   cpu_baseline the CPU oracle on a bounded sample of the same workload, on all
                host cores and on one
-  decode       the decode kernel on Llama-2-7B shapes at M = 1, 4, 16 (GB/s)
+  decode       the decode kernels on Llama-2-7B shapes at M = 1, 4, 16, and the
+               single-CTA kernel at M = 64, 128 (GB/s of the bytes they must read)
 
 Multi-GPU (torchrun): every rank runs the whole workload on its own GPU with
 its own tokens (data-parallel M split, weak scaling); no collective touches
@@ -486,11 +487,14 @@ def decode_bench(hsg, stream, peaks, steps=20):
             del p
         layers.append((hsg.LinearGroup([m[0] for m in mem]), mem))
     out = {}
-    for M in (1, 4, 16):
+    for M in (1, 4, 16, 64, 128):
         X = {K: synth.normal_bf16((M, K), 1.0, "cuda", "decX", M, K) for K in (4096, 11008)}
         Y = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _, _, N, _ in mem] for _, mem in layers]
         res = {}
-        for name, path in (("tc", 2), ("simt", 5)):
+        # M <= 16: the tensor-core decode kernel and the CUDA-core one; above,
+        # the library's choice (the single-CTA tensor-core kernel, one
+        # 128-token tile, so each weight record is still read once)
+        for name, path in ((("tc", 2), ("simt", 5)) if M <= 16 else (("auto", 0),)):
             def step():
                 for (g, mem), ys in zip(layers, Y):
                     g([X[K] for _, K, _, _ in mem], ys, path=path, stream=stream)
@@ -507,7 +511,9 @@ def decode_bench(hsg, stream, peaks, steps=20):
             nbytes = steps * sum(a + M * K * 2 + M * N * 2 for _, mem in layers for _, K, N, a in mem)
             gbs = nbytes / (ms / 1e3) / 1e9
             res[name] = {"GB_s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                         "us_per_layer": ms * 1e3 / (steps * len(layers))}
+                         "us_per_layer": ms * 1e3 / (steps * len(layers)),
+                         "tflops": steps * sum(2.0 * M * K * N for _, mem in layers for _, K, N, _ in mem)
+                         / (ms / 1e3) / 1e12}
         out[f"M{M}"] = res
     for g, mem in layers:
         g.free()
