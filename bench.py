@@ -466,7 +466,7 @@ def cublas_bf16(shapes, M: int, stream, layers: int = 4, steps: int = 10):
             "note": "context only: torch.matmul (cuBLAS) on dense bf16 weights, not on the measured path"}
 
 
-def decode_bench(hsg, stream, peaks, steps=20):
+def decode_bench(hsg, stream, peaks, steps=20, Ms=(1, 4, 16, 32, 64, 128)):
     """Decode kernel on Llama-2-7B layer shapes, 70% 2:4 tiles: each layer's 7
     linears in one grouped launch, 4 layers rotated (about 1.1 GB of weights,
     far above L2) so every launch streams its weights from HBM. Bytes counted
@@ -487,14 +487,21 @@ def decode_bench(hsg, stream, peaks, steps=20):
             del p
         layers.append((hsg.LinearGroup([m[0] for m in mem]), mem))
     out = {}
-    for M in (1, 4, 16, 64, 128):
+    for M in Ms:
         X = {K: synth.normal_bf16((M, K), 1.0, "cuda", "decX", M, K) for K in (4096, 11008)}
         Y = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _, _, N, _ in mem] for _, mem in layers]
         res = {}
-        # M <= 16: the tensor-core decode kernel and the CUDA-core one; above,
-        # the library's choice (the single-CTA tensor-core kernel, one
-        # 128-token tile, so each weight record is still read once)
-        for name, path in ((("tc", 2), ("simt", 5)) if M <= 16 else (("auto", 0),)):
+        # M <= 16: the tensor-core decode kernel (16-token MMAs) and the
+        # CUDA-core one; 16 < M <= 64: the decode kernel's 64-token instance
+        # and the single-CTA GEMM (one 128-token tile, so each weight record
+        # is still read once, but no split-K); above: the library's choice
+        if M <= 16:
+            paths = (("tc", hsg.PATH_GEMV), ("simt", hsg.PATH_GEMV_SIMT))
+        elif M <= 64:
+            paths = (("tc", hsg.PATH_GEMV), ("gemm", hsg.PATH_GEMM_SINGLE))
+        else:
+            paths = (("auto", hsg.PATH_AUTO),)
+        for name, path in paths:
             def step():
                 for (g, mem), ys in zip(layers, Y):
                     g([X[K] for _, K, _, _ in mem], ys, path=path, stream=stream)

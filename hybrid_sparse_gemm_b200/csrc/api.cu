@@ -151,7 +151,8 @@ struct WorkList {
 // member, partial sums [S][P][128][16] fp32 (NULL when P == 1) and per-strip
 // arrival counters that the kernel re-arms to zero.
 struct DecodeWs {
-    float* partial[kMaxGroup] = {};
+    float* partial[kMaxGroup] = {};       // 16-token partials (M <= 16)
+    float* partial_wide[kMaxGroup] = {};  // kDecodeWideBN-token partials, allocated on the first call with M > 16
     unsigned* counters[kMaxGroup] = {};
     int S[kMaxGroup] = {};
 };
@@ -312,8 +313,10 @@ namespace {
 void free_ws(DecodeWs& w) {
     for (int i = 0; i < kMaxGroup; ++i) {
         cudaFree(w.partial[i]);
+        cudaFree(w.partial_wide[i]);
         cudaFree(w.counters[i]);
         w.partial[i] = nullptr;
+        w.partial_wide[i] = nullptr;
         w.counters[i] = nullptr;
     }
 }
@@ -438,26 +441,53 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     return PATCH_OK;
 }
 
+// Gives w the 64-token partial buffers if it lacks them (once; they live
+// until the group is destroyed, so captured graphs may keep their address).
+patch_status ensure_wide_ws(patch_group g, DecodeWs* w) {
+    for (int i = 0; i < g->n; ++i) {
+        if (g->parts[i] <= 1 || w->partial_wide[i]) continue;
+        if (cudaMalloc(&w->partial_wide[i], sizeof(float) * (size_t)w->S[i] * g->parts[i] * 128 * kDecodeWideBN) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            w->partial_wide[i] = nullptr;
+            return fail(PATCH_ERR_NOMEM, "decode workspace allocation failed");
+        }
+    }
+    return PATCH_OK;
+}
+
 // The decode workspace a call on `st` uses: the capture workspace when the
 // stream is capturing a graph, else the stream's own (allocated on its first
-// decode call; for the per-thread default stream, one per thread).
-patch_status get_decode_ws(patch_group g, cudaStream_t st, const DecodeWs** out) {
+// decode call; for the per-thread default stream, one per thread). A call
+// with bn = kDecodeWideBN also gives the capture workspace its 64-token
+// buffers, so a graph captured after one uncaptured call of that size
+// allocates nothing.
+patch_status get_decode_ws(patch_group g, cudaStream_t st, int bn, const DecodeWs** out) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     cudaError_t e = cudaStreamIsCapturing(st, &cs);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    const bool wide = bn == kDecodeWideBN;
+    std::lock_guard<std::mutex> lk(g->mu);
+    if (wide) {
+        patch_status s = ensure_wide_ws(g, &g->capture_ws);
+        if (s != PATCH_OK) return s;
+    }
     if (cs != cudaStreamCaptureStatusNone) {
         *out = &g->capture_ws;
         return PATCH_OK;
     }
     const size_t tid = st == cudaStreamPerThread ? std::hash<std::thread::id>()(std::this_thread::get_id()) : 0;
     const auto key = std::make_pair(st, tid);
-    std::lock_guard<std::mutex> lk(g->mu);
     auto it = g->decode_ws.find(key);
     if (it == g->decode_ws.end()) {
         DecodeWs w;
         patch_status s = alloc_ws(g, &w, st);
         if (s != PATCH_OK) return s;
         it = g->decode_ws.emplace(key, w).first;
+    }
+    if (wide) {
+        patch_status s = ensure_wide_ws(g, &it->second);
+        if (s != PATCH_OK) return s;
     }
     *out = &it->second;
     return PATCH_OK;
@@ -467,12 +497,17 @@ patch_status get_decode_ws(patch_group g, cudaStream_t st, const DecodeWs** out)
 // persistent CTAs (or clusters). kernel 0: (strip, token block), cost = slab
 // work (dense 1, 2:4 1/2) + one epilogue; kernel 1: (strip pair, token block),
 // same costs; kernel 3: (four strips, token block), the slower pair's cost;
-// kernel 2: (strip, K-part), cost = streamed bytes of the part.
-// Per tensor-core kernel (0 single CTA, 1 CTA pair, 2 decode, 4 CTA pair with
-// two strips per CTA): tokens per tile,
+// kernels 2 and 5: (strip, K-part), cost = streamed bytes of the part.
+// Per tensor-core kernel (0 single CTA, 1 CTA pair, 2 decode with 16-token
+// MMAs, 4 CTA pair with two strips per CTA, 5 decode with 64-token MMAs):
+// tokens per tile,
 // activation rows per TMA box, weight rows of a work unit, persistent slots.
 int kernel_bn(int kernel) {
-    return kernel == 0 ? kGemmBN : kernel == 2 ? kDecodeBN : kernel == 4 ? kGemm22BN : kGemm2BN;
+    return kernel == 0   ? kGemmBN
+           : kernel == 2 ? kDecodeBN
+           : kernel == 5 ? kDecodeWideBN
+           : kernel == 4 ? kGemm22BN
+                         : kGemm2BN;
 }
 int kernel_box_rows(int kernel) {
     return kernel == 1 ? kGemm2BN / 2 : kernel == 4 ? kGemm22BN / 2 : kernel_bn(kernel);
@@ -482,7 +517,11 @@ int64_t kernel_rows(const Plan& p, int kernel) {
     return kernel == 0 ? (int64_t)p.strip_cost.size() : kernel == 1 ? pairs : (pairs + 1) / 2;
 }
 int kernel_slots(const DeviceInfo& d, int kernel) {
-    return kernel == 1 ? d.pair_clusters : kernel == 4 ? d.wide_clusters : kernel == 2 ? kDecodeCtasPerSm * d.sms : d.sms;
+    return kernel == 1   ? d.pair_clusters
+           : kernel == 4 ? d.wide_clusters
+           : kernel == 2 ? kDecodeCtasPerSm * d.sms
+           : kernel == 5 ? kDecodeWideCtasPerSm * d.sms
+                         : d.sms;
 }
 
 void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std::vector<int>& work) {
@@ -624,7 +663,7 @@ patch_status check_device_is(int device) {
 // The wide kernel runs its pure 2:4 instance (GEMM_WIDE_24) when every slab
 // of every member runs on the sparse MMA.
 int resolve_path(patch_group g, int path, int64_t M) {
-    if (path == PATCH_PATH_AUTO) path = (M <= kDecodeBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
+    if (path == PATCH_PATH_AUTO) path = (M <= kDecodeWideBN) ? PATCH_PATH_GEMV : PATCH_PATH_GEMM;
     if (path == PATCH_PATH_GEMM) {
         if (M < kPairMinM) return PATCH_PATH_GEMM_SINGLE;
         int64_t quads = 0;
@@ -654,12 +693,12 @@ patch_status run_simt(patch_handle h, const void* X, int64_t M, void* Y, cudaStr
     return PATCH_OK;
 }
 
-// Kernel for a resolved path: 0 single CTA, 1 CTA pair, 3 two CTA pairs
-// sharing activations, 2 decode.
-int choose_kernel(patch_group g, int path) {
+// Kernel for a resolved path: 0 single CTA, 1 CTA pair, 4 CTA pair with two
+// strips per CTA, 2 / 5 decode with 16- / 64-token MMAs.
+int choose_kernel(patch_group g, int path, int64_t M) {
     (void)g;
     if (path == PATCH_PATH_GEMM_SINGLE) return 0;
-    if (path == PATCH_PATH_GEMV) return 2;
+    if (path == PATCH_PATH_GEMV) return M <= kDecodeBN ? 2 : 5;
     if (path == PATCH_PATH_GEMM_WIDE || path == PATCH_PATH_GEMM_WIDE_24) return 4;
     return 1;
 }
@@ -681,13 +720,15 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
         return fail(PATCH_ERR_ARG, "unknown path %d", path);
     if (path == PATCH_PATH_GEMM_WIDE_24 && !g->pure24)
         return fail(PATCH_ERR_ARG, "GEMM_WIDE_24 needs every slab of every member to be 2:4 in both strips of its pair");
-    if (path == PATCH_PATH_GEMV && M > kDecodeBN)
-        return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= 16 (got %lld)", (long long)M);
+    if (path == PATCH_PATH_GEMV && M > kDecodeWideBN)
+        return fail(PATCH_ERR_SHAPE, "the decode kernel takes M <= %d (got %lld)", kDecodeWideBN, (long long)M);
     if (M > (int64_t)INT32_MAX / 2) return fail(PATCH_ERR_SHAPE, "M too large");
-    const int kernel = choose_kernel(g, path);
+    const int kernel = choose_kernel(g, path, M);
+    const bool decode = kernel == 2 || kernel == 5;
     const int bn = kernel_bn(kernel);
-    const int mb = kernel == 2 ? 0 : (int)((M + bn - 1) / bn);
-    const int box_rows = kernel_box_rows(kernel);
+    const int mb = decode ? 0 : (int)((M + bn - 1) / bn);
+    // the decode kernels load (and multiply) only M rounded up to 16 tokens
+    const int box_rows = decode ? (int)std::min<int64_t>(bn, (M + 15) & ~15) : kernel_box_rows(kernel);
     GroupMaps maps;
     GroupArgs a;
     memset(&maps, 0, sizeof(maps));
@@ -711,12 +752,12 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
         sched_work = wl->work;
         grid = wl->grid;
     }
-    if (kernel == 2) {
+    if (decode) {
         const DecodeWs* ws = nullptr;
-        patch_status s = get_decode_ws(g, st, &ws);
+        patch_status s = get_decode_ws(g, st, bn, &ws);
         if (s != PATCH_OK) return s;
         for (int l = 0; l < g->n; ++l) {
-            a.partial[l] = ws->partial[l];
+            a.partial[l] = kernel == 5 ? ws->partial_wide[l] : ws->partial[l];
             a.counters[l] = ws->counters[l];
         }
     }
@@ -729,7 +770,7 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
     cudaError_t e = kernel == 0   ? launch_gemm(maps, a, grid, st)
                     : kernel == 1 ? launch_gemm2(maps, a, grid, st)
                     : kernel == 4 ? launch_gemm22(maps, a, grid, path == PATCH_PATH_GEMM_WIDE_24, st)
-                                  : launch_decode(maps, a, grid, st);
+                                  : launch_decode(maps, a, grid, bn, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return PATCH_OK;
 }
@@ -1330,7 +1371,7 @@ extern "C" patch_status patch_linear_noalloc(patch_handle h, const void* X_bf16,
     // Decode sizes: the CUDA-core kernel needs no schedule and no scratch.
     if (M <= 8) return run_simt(h, X_bf16, M, Y_bf16, st);
     const int path = resolve_path(h->self, PATCH_PATH_GEMM, M);
-    const int kernel = choose_kernel(h->self, path);
+    const int kernel = choose_kernel(h->self, path, M);
     const int bn = kernel_bn(kernel);
     const int64_t mb = (M + bn - 1) / bn;
     const int64_t rows = kernel_rows(h->plan, kernel);

@@ -1,42 +1,65 @@
-// Decode-sized product (M <= 16 tokens) on the tensor core with split-K.
+// Decode-sized product (M <= 64 tokens) on the tensor core with split-K.
 //
 // At decode sizes the layer is bound by the bytes of W it streams; 2:4 slabs
 // carry 1.125 bytes per weight instead of 2, which is where PATCH's hybrid
 // kernel earns its speed (abstract of "PATCH: Learnable Tile-level Hybrid
 // Sparsity for LLMs"). This kernel is a streaming engine: four persistent
-// CTAs per SM (four independent issue loops; one loop cannot issue slabs as
-// fast as HBM delivers them) walk a cost-balanced list of units (strip s,
-// K-part p); warp 0 keeps kStages slab records in flight as 2-D TMA boxes
-// over the packed bytes (plus the 16-token X box), warp 1 runs them through
-// tcgen05.mma / .mma.sp with N = 16 into one of two TMEM accumulators, and an
-// epilogue warpgroup drains them alternately, writing each unit's fp32
-// partial (128 rows x 16 tokens) to a workspace. The CTA that finishes the
-// last part of a strip (per-strip arrival counter) sums the strip's partials
-// in part order, so the result does not depend on which CTA finishes first,
-// writes bf16 Y and re-arms the counter for the next call.
+// CTAs per SM (independent issue loops; one loop cannot issue slabs as fast
+// as HBM delivers them) walk a cost-balanced list of units (strip s, K-part
+// p); warp 0 keeps the stages' slab records in flight as 2-D TMA boxes over
+// the packed bytes (with an L2 evict-first hint: each is read once per call)
+// plus the X box of M rounded up to 16 tokens, warp 1 runs them through
+// tcgen05.mma / .mma.sp with N = that token count into a TMEM accumulator,
+// and an epilogue warpgroup drains it, writing each unit's fp32 partial
+// (128 rows x the tokens, token-major so a warp's accesses are coalesced) to
+// a workspace. The CTA that finishes the last part of a strip (per-strip
+// arrival counter) sums the strip's partials in part order, so the result
+// does not depend on which CTA finishes first, writes bf16 Y and re-arms the
+// counter for the next call.
+//
+// Two instances: up to 16 tokens (two stages and two 16-column accumulators
+// per CTA) and up to 64 (two stages and one 64-column accumulator: four CTAs
+// then fit the SM's 512 TMEM columns, and while one CTA's MMAs wait for its
+// epilogue the other three keep streaming).
 #include "kernels.cuh"
 
 namespace patch {
 
 namespace {
 
-constexpr int kEpiGroups = 1;           // epilogue warpgroups (units dealt round robin)
-constexpr int kThreads = 64 + 128 * kEpiGroups;  // producer warp, MMA warp, epilogue
-constexpr int kBN = kDecodeBN;           // tokens per MMA (M <= 16)
-constexpr int kStageA = 18432;           // 16 KB dense, or 8 KB values + 2 KB metadata
-constexpr int kStageX = kBN * 128;       // 2 KB, 128-byte swizzled
-constexpr int kStageBytes = kStageA + kStageX;
-constexpr int kStages = 2;               // per CTA; kDecodeCtasPerSm CTAs share an SM
-constexpr int kSmemData = kStages * kStageBytes;
-constexpr int kSmemBytes = kSmemData + 1024 + 256;
-constexpr int kECol = 2 * kBN;           // metadata columns after the two accumulators
-constexpr int kTmemCols = 64;
+constexpr int kThreads = 64 + 128;      // producer warp, MMA warp, one epilogue warpgroup
+constexpr int kStageA = 18432;          // 16 KB dense, or 8 KB values + 2 KB metadata
 
-// Named barrier of one epilogue warpgroup (id 1 + its index).
-__device__ __forceinline__ void epi_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory"); }
+constexpr int tmem_cols_for(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
-__global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
+// BN tokens per MMA, CTAS resident CTAs per SM, STAGES slab stages and ACCS
+// TMEM accumulators per CTA (with one, the MMAs of the next unit wait for the
+// epilogue to read the last one; the other CTAs on the SM keep streaming).
+template <int BN, int CTAS, int STAGES, int ACCS>
+struct DecodeCfg {
+    static constexpr int kStageX = BN * 128;  // up to BN rows of 128 bytes, 128-byte swizzled
+    static constexpr int kStageBytes = kStageA + kStageX;
+    static constexpr int kSmemData = STAGES * kStageBytes;
+    static constexpr int kSmemBytes = kSmemData + 1024 + 256;
+    static constexpr int kECol = ACCS * BN;   // metadata columns after the accumulators
+    static constexpr int kTmemCols = tmem_cols_for(kECol + 4);
+    // tokens the split-K sum holds in registers at once
+    static constexpr int kRed = CTAS > 2 && BN > 32 ? 32 : BN;
+    static_assert(ACCS == 1 || ACCS == 2, "one or two accumulators");
+    static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+    static_assert(kECol + 4 <= kTmemCols && kTmemCols * CTAS <= 512, "TMEM columns of the resident CTAs");
+    static_assert(CTAS * (kSmemBytes + 1024) <= 228 * 1024, "shared memory of the resident CTAs");
+};
+
+// Named barrier of the epilogue warpgroup.
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN, int CTAS, int STAGES, int ACCS>
+__global__ void __launch_bounds__(kThreads, CTAS)
     hybrid_decode_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupArgs a) {
+    using Cfg = DecodeCfg<BN, CTAS, STAGES, ACCS>;
+    constexpr int kBN = BN, kStages = STAGES, kStageBytes = Cfg::kStageBytes;
+    constexpr int kSmemData = Cfg::kSmemData, kECol = Cfg::kECol, kTmemCols = Cfg::kTmemCols;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -48,10 +71,13 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
     uint64_t* drain = acc_full + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;  // one per epilogue warpgroup
+    volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // token columns in use: M rounded up to the MMA's N granule of 16; the X
+    // box (encoded by the host) and every MMA cover just these
+    const int n_tok = min(kBN, (a.M + 15) & ~15);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -102,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 part_range(L, p, b0, b1);
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
                 const uint32_t* mrow = L.meta + (size_t)s * L.KC;
+                const uint64_t pol_w = policy_evict_first();  // weights are read once per call
                 const CUtensorMap* tmap_x = &maps.x[l];
                 uint32_t d_next = b0 < b1 ? trow[b0] : 0u;
                 for (int b = b0; b < b1; ++b) {
@@ -115,11 +142,13 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                     const bool sp = d & kSlabSparse, first = d & kSlabFirst;
                     const uint32_t bytes_a = sp ? kSparseValBytes : kDenseSlabBytes;
                     uint8_t* st = smem + stage * kStageBytes;
-                    mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + kStageX);
+                    mbar_arrive_expect_tx(&full[stage], bytes_a + (first ? kMetaBytes : 0) + (uint32_t)n_tok * 128u);
                     // the packed bytes viewed as 128-byte rows: one 2-D box per record
-                    tma_load_2d(st, sp ? &maps.a8[l] : &maps.a16[l], &full[stage], 0, (int)(slab_offset_bytes(d) >> 7));
+                    tma_load_2d_hint(st, sp ? &maps.a8[l] : &maps.a16[l], &full[stage], 0,
+                                     (int)(slab_offset_bytes(d) >> 7), pol_w);
                     if (first)
-                        tma_load_2d(st + kSparseValBytes, &maps.e[l], &full[stage], 0, (int)(mrow[b >> 1] >> 3));
+                        tma_load_2d_hint(st + kSparseValBytes, &maps.e[l], &full[stage], 0, (int)(mrow[b >> 1] >> 3),
+                                         pol_w);
                     tma_load_2d(st + kStageA, tmap_x, &full[stage], b * kSlabK, 0);
                     ++issued;
                     if (++stage == kStages) {
@@ -143,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            const uint32_t idesc_d = idesc_bf16(128, kBN, false);
-            const uint32_t idesc_s = idesc_bf16(128, kBN, true);
+            const uint32_t idesc_d = idesc_bf16(128, n_tok, false);
+            const uint32_t idesc_s = idesc_bf16(128, n_tok, true);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, any_mma = false;
@@ -158,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 int b0, b1;
                 part_range(L, p, b0, b1);
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
-                const int acc = t & 1;
-                if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
+                const int acc = t % ACCS;
+                if (!mbar_wait(&acc_empty[acc], ((t / ACCS) & 1) ^ 1u, abort_flag)) {
                     raise();
                     break;
                 }
@@ -222,76 +251,85 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
             }
         }
     } else {
-        // ---------------- epilogue: warpgroup g (warps 2+4g .. 5+4g) drains every kEpiGroups-th unit ----------------
-        const int g = (warp - 2) >> 2;
-        const int q = warp & 3;          // TMEM lane quadrant this warp may access
+        // ---------------- epilogue: warps 2..5, one TMEM lane quadrant each ----------------
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;
-        const int leader = 64 + 128 * g;  // first thread of the warpgroup
+        constexpr int kLeader = 64;  // first thread of the warpgroup
         int t = 0;
         for (int it = w_begin; it < w_end; ++it, ++t) {
-            if (t % kEpiGroups != g) continue;  // another warpgroup's unit
-            const int acc = t & 1;
+            const int acc = t % ACCS;
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const LinDesc& L = a.lins[l];
             const int P = L.P;
             const int s = lu / P, p = lu % P;
-            if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
+            if (!mbar_wait(&acc_full[acc], (t / ACCS) & 1, abort_flag)) {
                 if (lane == 0) raise();
                 break;
             }
             tc_fence_after();
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN), v);
-            tc_wait_ld();
+            __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
+            // this unit's partial, workspace[s][p][token][row]: a warp's
+            // stores and loads of one token cover 128 contiguous bytes
+            float* dst = P > 1 ? a.partial[l] + ((size_t)s * P + p) * kBN * 128 + row : nullptr;
+            const int cols = n_tok;
+            // 16 columns at a time: Y directly when the strip is one unit,
+            // else the partial
+#pragma unroll
+            for (int c0 = 0; c0 < kBN; c0 += 16) {
+                if (c0 >= cols) break;
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN + c0), v);
+                tc_wait_ld();
+                if (P == 1) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c0 + c < a.M) yc[(size_t)(c0 + c) * L.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) __stcg(dst + (c0 + c) * 128, __uint_as_float(v[c]));
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
-            __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
-            if (P == 1) {
-                // whole strip in one unit: no partial sums
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
-                continue;
-            }
-            // this unit's partial: workspace[s][p][row][0..15]
-            float4* dst = reinterpret_cast<float4*>(a.partial[l] + (((size_t)s * P + p) * 128 + row) * kBN);
-#pragma unroll
-            for (int c = 0; c < kBN / 4; ++c)
-                dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
-                                     __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
-            epi_bar(g);
-            if ((int)threadIdx.x == leader) {
+            if (P == 1) continue;
+            epi_bar();
+            if ((int)threadIdx.x == kLeader) {
                 // the barrier orders the warpgroup's stores before this fence,
                 // which releases them with the arrival
                 __threadfence();
                 const unsigned old = atomicAdd(&a.counters[l][s], 1u);
-                last_flag[g] = (old == (unsigned)(P - 1));
+                *last_flag = (old == (unsigned)(P - 1));
             }
-            epi_bar(g);
-            if (last_flag[g]) {
+            epi_bar();
+            if (*last_flag) {
                 __threadfence();
-                float sum[kBN];
+                // sum the parts in part order; all of one part's loads of a
+                // chunk of kRed tokens are in flight together
+                constexpr int kRed = Cfg::kRed;
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) sum[c] = 0.f;
-                for (int pp = 0; pp < P; ++pp) {
-                    const float4* src =
-                        reinterpret_cast<const float4*>(a.partial[l] + (((size_t)s * P + pp) * 128 + row) * kBN);
+                for (int c0 = 0; c0 < kBN; c0 += kRed) {
+                    if (c0 >= cols) break;
+                    float sum[kRed];
 #pragma unroll
-                    for (int c = 0; c < kBN / 4; ++c) {
-                        const float4 f = __ldcg(src + c);
-                        sum[4 * c] += f.x;
-                        sum[4 * c + 1] += f.y;
-                        sum[4 * c + 2] += f.z;
-                        sum[4 * c + 3] += f.w;
+                    for (int c = 0; c < kRed; ++c) sum[c] = 0.f;
+                    const float* src = a.partial[l] + (size_t)s * P * kBN * 128 + c0 * 128 + row;
+                    for (int pp = 0; pp < P; ++pp, src += kBN * 128) {
+                        float v[kRed];
+#pragma unroll
+                        for (int c = 0; c < kRed; ++c) v[c] = c0 + c < cols ? __ldcg(src + c * 128) : 0.f;
+#pragma unroll
+                        for (int c = 0; c < kRed; ++c) sum[c] += v[c];
                     }
-                }
 #pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (c < a.M) yc[(size_t)c * L.N] = __float2bfloat16_rn(sum[c]);
-                if ((int)threadIdx.x == leader) a.counters[l][s] = 0u;  // re-armed for the next call
+                    for (int c = 0; c < kRed; ++c)
+                        if (c0 + c < a.M) yc[(size_t)(c0 + c) * L.N] = __float2bfloat16_rn(sum[c]);
+                }
+                if ((int)threadIdx.x == kLeader) a.counters[l][s] = 0u;  // re-armed for the next call
             }
+            // the flag is rewritten only after the next unit's first barrier,
+            // which every thread reaches after reading it here
         }
     }
 
@@ -305,12 +343,34 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
 
 }  // namespace
 
+// BN = 16: M <= 16, four CTAs per SM, two stages and two accumulators each.
+// BN = kDecodeWideBN: 16 < M <= kDecodeWideBN, kDecodeWideCtasPerSm CTAs per SM
+// (the stage and accumulator counts are macros so that other splits of the
+// SM's shared memory and TMEM can be measured).
+#ifndef PATCH_DECODE_WIDE_STAGES
+#define PATCH_DECODE_WIDE_STAGES 2
+#endif
+#ifndef PATCH_DECODE_WIDE_ACCS
+#define PATCH_DECODE_WIDE_ACCS 1
+#endif
+using Narrow = DecodeCfg<kDecodeBN, kDecodeCtasPerSm, 2, 2>;
+using Wide = DecodeCfg<kDecodeWideBN, kDecodeWideCtasPerSm, PATCH_DECODE_WIDE_STAGES, PATCH_DECODE_WIDE_ACCS>;
+#define PATCH_DECODE16 hybrid_decode_kernel<kDecodeBN, kDecodeCtasPerSm, 2, 2>
+#define PATCH_DECODE_WIDE \
+    hybrid_decode_kernel<kDecodeWideBN, kDecodeWideCtasPerSm, PATCH_DECODE_WIDE_STAGES, PATCH_DECODE_WIDE_ACCS>
+
 cudaError_t decode_prepare() {
-    return cudaFuncSetAttribute(hybrid_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(PATCH_DECODE16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Narrow::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(PATCH_DECODE_WIDE, cudaFuncAttributeMaxDynamicSharedMemorySize, Wide::kSmemBytes);
 }
 
-cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st) {
-    hybrid_decode_kernel<<<grid, kThreads, kSmemBytes, st>>>(maps, a);
+cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, int bn, cudaStream_t st) {
+    if (bn == kDecodeWideBN)
+        PATCH_DECODE_WIDE<<<grid, kThreads, Wide::kSmemBytes, st>>>(maps, a);
+    else
+        PATCH_DECODE16<<<grid, kThreads, Narrow::kSmemBytes, st>>>(maps, a);
     return cudaGetLastError();
 }
 

@@ -77,7 +77,8 @@ cudaError_t launch_gemm(const GroupMaps& maps, const GroupArgs& a, int grid, cud
 cudaError_t launch_gemm2(const GroupMaps& maps, const GroupArgs& a, int clusters, cudaStream_t st);
 // pure24: every member's slabs all run on the sparse MMA (no tables read)
 cudaError_t launch_gemm22(const GroupMaps& maps, const GroupArgs& a, int clusters, bool pure24, cudaStream_t st);
-cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, cudaStream_t st);
+// bn: tokens per decode MMA, kDecodeBN (M <= 16) or kDecodeWideBN (M <= 64)
+cudaError_t launch_decode(const GroupMaps& maps, const GroupArgs& a, int grid, int bn, cudaStream_t st);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 cudaError_t launch_selftest_wait(int* status, cudaStream_t st);
 cudaError_t gemm_prepare_single();
@@ -90,5 +91,13 @@ constexpr int kGemm2BN = 256;  // tokens per CTA-pair tile
 constexpr int kGemm22BN = 240; // tokens per tile of the two-strips-per-CTA pair kernel
 constexpr int kDecodeBN = 16;  // tokens per decode MMA (M <= 16)
 constexpr int kDecodeCtasPerSm = 4;  // decode CTAs resident per SM (four issue loops per SM)
+#ifndef PATCH_DECODE_WIDE_BN
+#define PATCH_DECODE_WIDE_BN 64
+#endif
+#ifndef PATCH_DECODE_WIDE_CTAS
+#define PATCH_DECODE_WIDE_CTAS 4
+#endif
+constexpr int kDecodeWideBN = PATCH_DECODE_WIDE_BN;  // tokens per MMA of the decode instance for 16 < M
+constexpr int kDecodeWideCtasPerSm = PATCH_DECODE_WIDE_CTAS;  // its CTAs per SM
 
 }  // namespace patch

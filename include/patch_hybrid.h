@@ -28,7 +28,7 @@
  *     kernel's split-K workspaces.
  *   - Concurrency: patch_linear, patch_linear_path and patch_group_linear
  *     calls on one handle or group may overlap on the GPU when they are
- *     issued on different streams or threads. The decode kernel (M <= 16)
+ *     issued on different streams or threads. The decode kernel (M <= 64)
  *     keeps its split-K partial sums in a workspace per stream (per thread
  *     for the per-thread default stream); the other kernels keep no per-call
  *     state. Three exceptions: patch_linear_host calls on one handle share a
@@ -64,7 +64,7 @@ typedef enum {
                                   larger than a fixed limit of patch_linear_noalloc */
 } patch_status;
 
-/* Which kernel patch_linear_path runs. AUTO picks by M: GEMV for M <= 16,
+/* Which kernel patch_linear_path runs. AUTO picks by M: GEMV for M <= 64,
  * GEMM_SINGLE below M = 256, and above it GEMM_WIDE (GEMM_WIDE_24 for pure
  * 2:4 weights) when the call (or group) has at least two 512-row x 240-token
  * tiles per co-resident CTA pair, otherwise GEMM_PAIR. GEMM is AUTO
@@ -72,7 +72,8 @@ typedef enum {
 typedef enum {
     PATCH_PATH_AUTO = 0,
     PATCH_PATH_GEMM = 1,         /* tcgen05 tensor-core GEMM, variant chosen as for AUTO */
-    PATCH_PATH_GEMV = 2,         /* decode kernel (M <= 16): tcgen05 N=16, split-K */
+    PATCH_PATH_GEMV = 2,         /* decode kernel (M <= 64): tcgen05 with N = M rounded up
+                                    to 16, split-K over the weight stream */
     PATCH_PATH_GEMM_SINGLE = 3,  /* tcgen05, one CTA per 128-row x 128-token tile */
     PATCH_PATH_GEMM_PAIR = 4,    /* tcgen05 cta_group::2, one CTA pair per 256 x 256 tile */
     PATCH_PATH_GEMV_SIMT = 5,    /* decode on CUDA cores (M <= 16), no workspace */
@@ -212,8 +213,9 @@ patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flag
  * a new value of M builds that M's work schedule and uploads it
  * asynchronously on `stream` (it allocates device and pinned host memory);
  * a call on another stream waits for that upload on the device. The first
- * uncaptured decode call (M <= 16) on a stream allocates that stream's
- * workspace (a few MB, held until the handle or group is freed). Before
+ * uncaptured decode call (M <= 64) on a stream allocates that stream's
+ * workspace (a few MB, held until the handle or group is freed); the first
+ * with 16 < M <= 64 adds four times that for the wider partial sums. Before
  * capturing later calls in a CUDA graph, make one call with the same M and
  * let it complete.
  */
@@ -221,7 +223,8 @@ patch_status patch_linear(patch_handle h, const void* X_bf16, int64_t M, void* Y
                           void* stream);
 
 /* patch_linear with an explicit kernel choice (patch_path). GEMV requires
- * M <= 16. Any M works on the tensor-core variants. */
+ * M <= 64 and GEMV_SIMT M <= 16 (PATCH_ERR_SHAPE otherwise). Any M works on
+ * the tensor-core GEMM variants. */
 patch_status patch_linear_path(patch_handle h, const void* X_bf16, int64_t M, void* Y_bf16,
                                int path, void* stream);
 
@@ -255,8 +258,8 @@ patch_status patch_linear_host(patch_handle h, const void* X_host, int64_t M, vo
  *     M >= 256       the CTA-pair kernel patch_linear would run for this M:
  *                    GEMM_WIDE (512-row x 240-token tiles) or GEMM_PAIR
  *                    (256-row x 256-token tiles).
- *   For M >= 17 the result is bit-identical to patch_linear's (same kernel,
- *   same schedule); for M <= 16 patch_linear runs the tensor-core decode
+ *   For M >= 65 the result is bit-identical to patch_linear's (same kernel,
+ *   same schedule); for M <= 64 patch_linear runs the tensor-core decode
  *   kernel instead, which sums in another order (both within the tolerance
  *   of the fp32 product).
  * Limits: at most 65536 output tiles per call (tiles as above;

@@ -171,18 +171,35 @@ def test_gemv_small(hsg, oracle_lib, N, K, R, C, frac, M, kernel):
     lin.free()
 
 
+@pytest.mark.parametrize("N,K,R,C", SMALL_ODD)
+@pytest.mark.parametrize("frac", [0.0, 0.6, 1.0])
+@pytest.mark.parametrize("M", [17, 31, 33, 48, 63, 64])
+def test_decode_wide_small(hsg, oracle_lib, N, K, R, C, frac, M):
+    """The decode kernel's 64-token instance (16 < M <= 64): ragged M inside
+    its one token tile, every tile shape and fraction."""
+    p = synth.make_problem(N, K, M, R=R, C=C, frac=frac, seed=M + 300, device="cuda")
+    lin = pack(hsg, p)
+    Y = lin(p.X, path=hsg.PATH_GEMV)
+    torch.cuda.synchronize()
+    lin.check()
+    assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"decode wide M={M}")
+    lin.free()
+
+
 def test_decode_repeat_and_interleave(hsg, oracle_lib):
     """The split-K decode re-arms its per-strip counters: repeated and
     interleaved calls on one handle give identical bits."""
-    p = synth.make_problem(1152, 2048, 16, R=128, C=128, frac=0.7, seed=9, device="cuda")
+    p = synth.make_problem(1152, 2048, 64, R=128, C=128, frac=0.7, seed=9, device="cuda")
     lin = pack(hsg, p)
     outs = []
-    for M in (16, 1, 16, 5, 16):
+    # both instances (16- and 64-token MMAs) share the per-strip counters
+    for M in (16, 1, 64, 16, 5, 40, 16, 64):
         X = p.X[:M].contiguous()
         outs.append((M, lin(X, path=hsg.PATH_GEMV)))
     torch.cuda.synchronize()
     lin.check()
-    assert torch.equal(outs[0][1], outs[2][1]) and torch.equal(outs[0][1], outs[4][1])
+    assert torch.equal(outs[0][1], outs[3][1]) and torch.equal(outs[0][1], outs[6][1])
+    assert torch.equal(outs[2][1], outs[7][1])
     for M, Y in outs:
         assert_close(Y, oracle_lib, p.X[:M].contiguous(), p.W, p.bits, p.keep, what=f"decode repeat M={M}")
     lin.free()
@@ -306,8 +323,11 @@ def test_empty_and_misaligned(hsg):
     with pytest.raises(hsg.PatchError) as e:
         lin(Xmis)
     assert e.value.status == 3
-    with pytest.raises(hsg.PatchError) as e:  # the decode kernel takes M <= 16
-        lin(torch.zeros(17, 256, dtype=torch.bfloat16, device="cuda"), path=hsg.PATH_GEMV)
+    with pytest.raises(hsg.PatchError) as e:  # the decode kernel takes M <= 64
+        lin(torch.zeros(65, 256, dtype=torch.bfloat16, device="cuda"), path=hsg.PATH_GEMV)
+    assert e.value.status == 2
+    with pytest.raises(hsg.PatchError) as e:  # the CUDA-core one M <= 16
+        lin(torch.zeros(17, 256, dtype=torch.bfloat16, device="cuda"), path=hsg.PATH_GEMV_SIMT)
     assert e.value.status == 2
     lin.free()
 
@@ -317,25 +337,28 @@ def test_decode_concurrent_streams(hsg, oracle_lib):
     synchronisation between the streams: each stream has its own split-K
     workspace, so both streams' results equal the sequential ones bit for bit
     (and the oracle)."""
-    p = synth.make_problem(1152, 4096, 16, R=128, C=128, frac=0.7, seed=19, device="cuda")
+    p = synth.make_problem(1152, 4096, 64, R=128, C=128, frac=0.7, seed=19, device="cuda")
     q = synth.make_problem(640, 4096, 16, R=128, C=128, frac=0.5, seed=20, device="cuda")
     lp, lq = pack(hsg, p), pack(hsg, q)
     g = hsg.LinearGroup([lp, lq])
-    Xa, Xb = p.X[:16].contiguous(), p.X[:3].contiguous()
+    Xa, Xb, Xw = p.X[:16].contiguous(), p.X[:3].contiguous(), p.X[:50].contiguous()
     ref_a, ref_b = lp(Xa, path=hsg.PATH_GEMV), lp(Xb, path=hsg.PATH_GEMV)
+    ref_w = lp(Xw, path=hsg.PATH_GEMV)
     gref = g([Xa, q.X[:16].contiguous()], path=hsg.PATH_GEMV)
     torch.cuda.synchronize()
     sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
-    outs_a, outs_b, gouts = [], [], []
+    outs_a, outs_b, outs_w, gouts = [], [], [], []
     for _ in range(20):
         outs_a.append(lp(Xa, path=hsg.PATH_GEMV, stream=sa))
+        outs_w.append(lp(Xw, path=hsg.PATH_GEMV, stream=sa))
         outs_b.append(lp(Xb, path=hsg.PATH_GEMV, stream=sb))
         gouts.append(g([Xa, q.X[:16].contiguous()], path=hsg.PATH_GEMV, stream=sb))
     torch.cuda.synchronize()
     lp.check()
-    for Ya, Yb, Yg in zip(outs_a, outs_b, gouts):
-        assert torch.equal(Ya, ref_a) and torch.equal(Yb, ref_b)
+    for Ya, Yb, Yw, Yg in zip(outs_a, outs_b, outs_w, gouts):
+        assert torch.equal(Ya, ref_a) and torch.equal(Yb, ref_b) and torch.equal(Yw, ref_w)
         assert torch.equal(Yg[0], gref[0]) and torch.equal(Yg[1], gref[1])
+    assert_close(outs_w[-1], oracle_lib, Xw, p.W, p.bits, p.keep, what="decode stream a, 64-token instance")
     assert_close(outs_a[-1], oracle_lib, Xa, p.W, p.bits, p.keep, what="decode stream a")
     assert_close(outs_b[-1], oracle_lib, Xb, p.W, p.bits, p.keep, what="decode stream b")
     g.free()
@@ -399,27 +422,31 @@ def test_cuda_graph_capture_and_replay(hsg):
     lp, lq = pack(hsg, p), pack(hsg, q)
     g = hsg.LinearGroup([lp, lq])
     X16 = p.X[:16].contiguous()
+    X48 = [p.X[:48].contiguous(), q.X[:48].contiguous()]
     Y1 = torch.empty((600, 1024), dtype=torch.bfloat16, device="cuda")
     Y2 = torch.empty((16, 1024), dtype=torch.bfloat16, device="cuda")
     G = [torch.empty((600, 1024), dtype=torch.bfloat16, device="cuda"),
          torch.empty((600, 512), dtype=torch.bfloat16, device="cuda")]
+    G48 = [torch.empty((48, 1024), dtype=torch.bfloat16, device="cuda"),
+           torch.empty((48, 512), dtype=torch.bfloat16, device="cuda")]
     eager1, eager2 = lp(p.X), lp(X16)
     eg = g([p.X, q.X])
+    eg48 = g(X48, path=hsg.PATH_GEMV)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         lp(p.X, out=Y1)
         lp(X16, out=Y2)
         g([p.X, q.X], G)
+        g(X48, G48, path=hsg.PATH_GEMV)
     for _ in range(3):
-        Y1.zero_()
-        Y2.zero_()
-        G[0].zero_()
-        G[1].zero_()
+        for t in (Y1, Y2, *G, *G48):
+            t.zero_()
         graph.replay()
         torch.cuda.synchronize()
         assert torch.equal(Y1, eager1) and torch.equal(Y2, eager2)
         assert torch.equal(G[0], eg[0]) and torch.equal(G[1], eg[1])
+        assert torch.equal(G48[0], eg48[0]) and torch.equal(G48[1], eg48[1])
     lp.check()
     del graph
     g.free()
@@ -548,11 +575,11 @@ def test_pure_24_instance(hsg, oracle_lib, model, M, members):
         lin.free()
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("M", [1, 4, 16, 32, 64])
 def test_config3_llama2_7b_decode(hsg, oracle_lib, M):
     shapes = synth.llama2_7b()
-    _layer(hsg, oracle_lib, shapes, M, [0.7] * 7, tag="cfg3",
-           paths=[hsg.PATH_GEMV, hsg.PATH_GEMV_SIMT, hsg.PATH_GEMM], check_bytes=(M == 1))
+    paths = [hsg.PATH_GEMV, hsg.PATH_GEMM] + ([hsg.PATH_GEMV_SIMT] if M <= 16 else [])
+    _layer(hsg, oracle_lib, shapes, M, [0.7] * 7, tag="cfg3", paths=paths, check_bytes=(M == 1))
 
 
 @pytest.mark.parametrize("frac", [0.0, 0.5, 0.7, 0.9, 1.0])
@@ -572,7 +599,7 @@ def test_config5_llama2_13b_tiles(hsg, oracle_lib, R, C):
 
 @pytest.mark.parametrize("path_name,M", [("GEMM_PAIR", 300), ("GEMM_SINGLE", 130), ("GEMV", 16), ("GEMV", 3),
                                          ("GEMV_SIMT", 5), ("AUTO", 520), ("AUTO", 1), ("GEMM_WIDE", 300),
-                                         ("GEMM_WIDE", 17)])
+                                         ("GEMM_WIDE", 17), ("GEMV", 40), ("GEMV", 64)])
 def test_group_matches_members(hsg, oracle_lib, path_name, M):
     """One launch over several linears (shared and separate inputs, mixed tile
     shapes and 2:4 fractions) equals the members run one by one, bit for bit,
@@ -596,7 +623,7 @@ def test_group_matches_members(hsg, oracle_lib, path_name, M):
     lins[0].check()
     # the decode kernel may split K differently inside a group (different
     # summation order); every other kernel gives the same bits
-    decode = path == hsg.PATH_GEMV or (path == hsg.PATH_AUTO and M <= 16)
+    decode = path == hsg.PATH_GEMV or (path == hsg.PATH_AUTO and M <= 64)
     for i, (p, x) in enumerate(zip(probs, xs)):
         if not decode:
             assert torch.equal(Yg[i], Yi[i]), f"member {i} differs from its own launch"
@@ -617,7 +644,8 @@ def test_group_path_choice(hsg):
     big = pack(hsg, synth.make_problem(8192, 256, 0, seed=2, device="cuda", tag="gp2"))
     gs, gb = hsg.LinearGroup([small]), hsg.LinearGroup([big])
     assert gs.path(1) == hsg.PATH_GEMV and gs.path(16) == hsg.PATH_GEMV
-    assert gs.path(17) == hsg.PATH_GEMM_SINGLE and gs.path(255) == hsg.PATH_GEMM_SINGLE
+    assert gs.path(17) == hsg.PATH_GEMV and gs.path(64) == hsg.PATH_GEMV
+    assert gs.path(65) == hsg.PATH_GEMM_SINGLE and gs.path(255) == hsg.PATH_GEMM_SINGLE
     assert gs.path(256) == hsg.PATH_GEMM_PAIR          # one strip quad: too few tiles
     assert gb.path(4096) == hsg.PATH_GEMM_WIDE         # 16 quads x 18 token blocks
     assert gb.path(4096, hsg.PATH_GEMM_PAIR) == hsg.PATH_GEMM_PAIR

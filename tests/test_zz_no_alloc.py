@@ -6,8 +6,8 @@ call cudaMalloc) use this entry point; its tile schedule lives in a fixed array
 of the library's device image instead of memory the library allocates. These
 tests call it through the C ABI, two calls in a row on the shared array, and
 compare it with patch_linear: bit for bit where both run the same kernel on the
-same schedule (M >= 17), and against the CPU oracle within the parity bound of
-the other GPU tests where the kernels differ (M <= 16) and for one M >= 17 case.
+same schedule (M >= 65), and against the CPU oracle within the parity bound of
+the other GPU tests where the kernels differ (M <= 64) and for one M >= 65 case.
 This file is collected last, so a run that stops at its first failure has
 already run every other test.
 """
