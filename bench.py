@@ -24,12 +24,14 @@ Reported (one JSON line from rank 0):
                four tile shapes, with its own dense run
   cublas_bf16  torch.matmul (cuBLAS) on the dense weights of the same shapes,
                context only (not on the measured path)
-  e2e          the same metric through patch_linear_host (host buffers, copies
-               inside the timed region)
+  e2e          the same metric through patch_group_linear_host (host buffers,
+               copies inside the timed region)
   cpu_baseline the CPU oracle on a bounded sample of the same workload, on all
                host cores and on one
-  decode       the decode kernels on Llama-2-7B shapes at M = 1, 4, 16, and the
-               single-CTA kernel at M = 64, 128 (GB/s of the bytes they must read)
+  decode       on Llama-2-7B layer shapes (GB/s of the bytes that must be read):
+               the tensor-core decode kernel and the CUDA-core one at M = 1, 4,
+               16; the decode kernel and the single-CTA GEMM at M = 32, 64; the
+               automatic choice at M = 128
 
 Multi-GPU (torchrun): every rank runs the whole workload on its own GPU with
 its own tokens (data-parallel M split, weak scaling); no collective touches
@@ -583,6 +585,8 @@ def main():
     ap.add_argument("--no-13b", action="store_true", help="skip the Llama-2-13B tile-shape runs")
     ap.add_argument("--no-cublas", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-M", default="1,4,16,32,64,128",
+                    help="token counts of the decode section, comma-separated")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
@@ -750,7 +754,7 @@ def main():
     decode = None
     if not args.no_decode:
         with nvtx.range("decode"):
-            decode = decode_bench(hsg, stream, peaks)
+            decode = decode_bench(hsg, stream, peaks, Ms=tuple(int(m) for m in args.decode_M.split(",")))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
