@@ -766,6 +766,11 @@ patch_status run_group(patch_group g, const void* const* X, int64_t M, void* con
     a.work = sched_work;
     a.M = (int)M;
     a.MB = mb;
+    if (mb > 0) {
+        const int64_t gran = (M + 15) / 16;
+        a.tile_gran = (int)(gran / mb);
+        a.tile_extra = (int)(gran % mb);
+    }
     a.status = g->status_dev;
     cudaError_t e = kernel == 0   ? launch_gemm(maps, a, grid, st)
                     : kernel == 1 ? launch_gemm2(maps, a, grid, st)

@@ -76,10 +76,18 @@ constexpr int kECol1 = kBN + 8;                 // ... and of strip pair 1
 constexpr int kTmemCols = 512;
 static_assert(kECol1 + 4 <= kAcc1, "metadata columns fit between the accumulators");
 
-// Tokens of tile j (a multiple of 16: the MMA's N), at most kBN.
-__device__ __forceinline__ int tile_tokens(int j, int M) {
-    const int rem = M - j * kBN;
-    return rem >= kBN ? kBN : ((rem + 15) & ~15);
+// Token tiles: the MB = ceil(M / kBN) tiles share M's ceil(M / 16)
+// 16-token granules as evenly as possible (so no tile is a sliver that
+// streams a strip quad's weights for a few tokens): a.tile_gran each and one
+// more for the first a.tile_extra tiles (computed on the host). Tile j starts
+// at token tile_start(j) and its MMAs have N = tile_tokens(j), a multiple of
+// 16 and at most kBN; the last tile's N may reach past M (those columns are
+// never stored).
+__device__ __forceinline__ int tile_start(const GroupArgs& a, int j) {
+    return 16 * (j * a.tile_gran + min(j, a.tile_extra));
+}
+__device__ __forceinline__ int tile_tokens(const GroupArgs& a, int j) {
+    return 16 * (a.tile_gran + (j < a.tile_extra ? 1 : 0));
 }
 
 __device__ __forceinline__ uint32_t rec_bytes(uint32_t d) {
@@ -296,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                 }
                 const CUtensorMap* tm_x = &maps.x[l];
-                const int tok = j * kBN + (int)pr * (tile_tokens(j, a.M) >> 1);
+                const int tok = tile_start(a, j) + (int)pr * (tile_tokens(a, j) >> 1);
                 for (int kc = 0, part = 0; lane == 0 && kc < KC; ++g) {
                     const Chunk k0 = kPure24 ? pure_chunk(s0, kc, KB) : load_chunk(t0, kc, KB);
                     const Chunk k1 = kPure24 ? pure_chunk(s1, kc, KB) : load_chunk(t1, kc, KB);
@@ -404,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int t = 0;
             for (int it = w_begin; it < w_end && ok; ++it, ++t) {
                 const int j = (a.work[it] & kUnitMask) % a.MB;
-                const int nt = tile_tokens(j, a.M);
+                const int nt = tile_tokens(a, j);
                 const uint32_t idesc_d = idesc_bf16(256, nt, false);
                 const uint32_t idesc_s = idesc_bf16(256, nt, true);
                 if (!mbar_wait(&acc_empty[h], (t & 1) ^ 1u, abort_flag)) {
@@ -459,14 +467,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = lu / a.MB, j = lu % a.MB;
             const int s = 4 * c + 2 * h + (int)pr;
             const bool store = s < a.lins[l].S;
-            const int nt = tile_tokens(j, a.M);
+            const int nt = tile_tokens(a, j);
+            const int tok0 = tile_start(a, j);
+            const int mrem = a.M - tok0;  // tokens of the tile that exist
             if (!mbar_wait(&acc_full[h], t & 1, abort_flag)) {
                 if (lane == 0) raise();
                 break;
             }
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kAcc1);
-            __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + q * 32 + lane;
+            __nv_bfloat16* yc = a.Y[l] + (size_t)tok0 * N + (size_t)s * kStrip + q * 32 + lane;
             if (store) {
                 // 32-column chunks, alternating between the two warps of a lane
                 // quarter (the last chunk of a 240-token tile has 16 columns).
@@ -479,8 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         tmem_ld_32x32b_x16(taddr + c0, v);
                     tc_wait_ld();
-                    const int m0 = j * kBN + c0;
-                    if (m0 + cols <= a.M) {
+                    if (c0 + cols <= mrem) {
                         // Lanes 2i and 2i+1 hold rows 2i and 2i+1 of Y's columns;
                         // one swap per two tokens lets each lane store both rows'
                         // values of one token as a 4-byte pair (half the stores).
@@ -493,13 +502,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
                             const __nv_bfloat162 two =
                                 odd ? __floats2bfloat162_rn(recv, x1) : __floats2bfloat162_rn(x0, recv);
-                            *reinterpret_cast<__nv_bfloat162*>(yq + (size_t)(m0 + cc + (odd ? 1 : 0)) * N) = two;
+                            *reinterpret_cast<__nv_bfloat162*>(yq + (size_t)(c0 + cc + (odd ? 1 : 0)) * N) = two;
                         }
                     } else {
 #pragma unroll
                         for (int cc = 0; cc < 32; ++cc)
-                            if (cc < cols && m0 + cc < a.M)
-                                yc[(size_t)(m0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+                            if (cc < cols && c0 + cc < mrem)
+                                yc[(size_t)(c0 + cc) * N] = __float2bfloat16_rn(__uint_as_float(v[cc]));
                     }
                 }
             }

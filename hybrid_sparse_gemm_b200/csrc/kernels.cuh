@@ -50,7 +50,7 @@ struct GroupMaps {
 struct GroupArgs {
     const LinDesc* lins;
     __nv_bfloat16* Y[kMaxGroup];
-    // decode only: split-K workspace [S][P][128][16] fp32 and per-strip
+    // decode only: split-K workspace [S][P][BN][128] fp32 and per-strip
     // arrival counters (zero between calls) of each member, owned by the
     // calling stream so that calls on different streams never share them
     float* partial[kMaxGroup];
@@ -58,6 +58,9 @@ struct GroupArgs {
     const int* work_off;       // per CTA (or per CTA pair): [work_off[c], work_off[c+1])
     const int* work;
     int M, MB;
+    // two-strips-per-CTA kernel: its MB token tiles share M's ceil(M/16)
+    // 16-token granules, tile_gran each and one more for the first tile_extra
+    int tile_gran, tile_extra;
     int* status;               // device status word (timeouts)
 };
 constexpr int kUnitShift = 24;

@@ -271,6 +271,11 @@ def test_single_strip_single_slab(hsg, oracle_lib):
             Y = lin(p.X, path=path)
             torch.cuda.synchronize()
             assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, what=f"single slab {path}")
+        # the decode kernel's 64-token instance on the one slab
+        X = synth.normal_bf16((57, 64), 1.0, "cuda", "single-slab", frac)
+        Y = lin(X, path=hsg.PATH_GEMV)
+        torch.cuda.synchronize()
+        assert_close(Y, oracle_lib, X, p.W, p.bits, p.keep, what="single slab, 57 tokens")
         lin.free()
 
 
@@ -283,7 +288,7 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
     X = synth.normal_bf16((40, K), 1.0, "cuda", "zero", "X")
     lin = hsg.PackedLinear.pack(W, bits, fl, 64, 64)
     for path, M in ((hsg.PATH_GEMM_SINGLE, 40), (hsg.PATH_GEMM_PAIR, 40), (hsg.PATH_GEMV, 16),
-                    (hsg.PATH_GEMV_SIMT, 16)):
+                    (hsg.PATH_GEMV, 40), (hsg.PATH_GEMV_SIMT, 16)):
         Y = lin(X[:M].contiguous(), path=path)
         torch.cuda.synchronize()
         assert torch.count_nonzero(Y.float()) == 0
@@ -294,7 +299,7 @@ def test_zero_weights_and_checkerboard(hsg, oracle_lib):
     bits = synth.pack_bits(keep)
     lin = hsg.PackedLinear.pack(p.W, bits, fl, 64, 64)
     assert lin.info().slabs_sparse == 0
-    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR):
+    for path in (hsg.PATH_GEMM_SINGLE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMV):
         Y = lin(p.X, path=path)
         torch.cuda.synchronize()
         assert_close(Y, oracle_lib, p.X, p.W, bits, keep, what="checkerboard")
@@ -305,7 +310,7 @@ def test_one_sparse_tile(hsg, oracle_lib):
     p = synth.make_problem(512, 512, 50, R=128, C=128, n_sparse=1, seed=5, device="cuda")
     lin = pack(hsg, p)
     for path, M in ((hsg.PATH_GEMM_SINGLE, 50), (hsg.PATH_GEMM_PAIR, 50), (hsg.PATH_GEMV, 16),
-                    (hsg.PATH_GEMV_SIMT, 16)):
+                    (hsg.PATH_GEMV, 50), (hsg.PATH_GEMV_SIMT, 16)):
         X = p.X[:M].contiguous()
         Y = lin(X, path=path)
         torch.cuda.synchronize()
