@@ -35,7 +35,7 @@ EXPORTED = ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_hos
             "patch_info", "patch_copy_packed", "patch_check", "patch_free", "patch_last_error",
             "patch_version", "patch_plan", "patch_linear_noalloc", "patch_group_create",
             "patch_group_linear", "patch_group_path", "patch_group_free", "patch_selftest_wait",
-            "patch_partition_rows", "patch_classify_tiles", "patch_group_linear_host"]
+            "patch_partition_rows", "patch_classify_tiles", "patch_group_linear_host", "patch_plan_pairs"]
 
 
 class patch_info_t(ctypes.Structure):
@@ -68,6 +68,7 @@ _lib.patch_info.argtypes = [_P, ctypes.POINTER(patch_info_t)]
 _lib.patch_copy_packed.argtypes = [_P, _P, _I64, _P, _I64, _P, _I64, _P, _I64]
 _lib.patch_check.argtypes = [_P, _P]
 _lib.patch_plan.argtypes = [_I64, _I64, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I64)]
+_lib.patch_plan_pairs.argtypes = [_I64, _I64, _P, _I, _I, _P]
 _lib.patch_partition_rows.argtypes = [_I64, _I64, _P, _I, _I, _I, _I64, _P]
 _lib.patch_classify_tiles.argtypes = [_P, _I64, _I64, _I, _I, _P, ctypes.POINTER(_I64)]
 _lib.patch_free.argtypes = [_P]
@@ -77,7 +78,7 @@ _lib.patch_version.restype = ctypes.c_int
 for _n in ["patch_pack", "patch_linear", "patch_linear_path", "patch_linear_host", "patch_unpack",
            "patch_info", "patch_copy_packed", "patch_check", "patch_plan", "patch_linear_noalloc",
            "patch_group_create", "patch_group_linear", "patch_partition_rows", "patch_classify_tiles",
-           "patch_group_linear_host"]:
+           "patch_group_linear_host", "patch_plan_pairs"]:
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -124,6 +125,17 @@ def patch_plan(N: int, K: int, tile_flags, tile_rows: int = 128, tile_cols: int 
     _check(_lib.patch_plan(N, K, flags.ctypes.data, tile_rows, tile_cols, slab.ctypes.data,
                            meta.ctypes.data, gemm.ctypes.data, ctypes.byref(nbytes)))
     return (slab[:ns], meta[:nm], gemm[:ng]), int(nbytes.value)
+
+
+def patch_plan_pairs(N: int, K: int, tile_flags, tile_rows: int = 128, tile_cols: int = 128):
+    """Host-only: the strip order of the CTA-pair kernels as an int32 numpy
+    array of N/128 entries (pair i = strips order[2i], order[2i+1])."""
+    import numpy as np
+    flags = np.ascontiguousarray(np.asarray(tile_flags, dtype=np.uint8).reshape(-1))
+    S = N // 128 if N > 0 and N % 128 == 0 else 0
+    order = np.zeros(max(S, 1), np.int32)
+    _check(_lib.patch_plan_pairs(N, K, flags.ctypes.data, tile_rows, tile_cols, order.ctypes.data))
+    return order[:S]
 
 
 def patch_classify_tiles(mask_bits, N: int, K: int, tile_rows: int = 128, tile_cols: int = 128):

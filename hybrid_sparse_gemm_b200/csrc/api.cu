@@ -161,10 +161,80 @@ struct DecodeWs {
 struct Plan {
     int S = 0, KB = 0, KC = 0;
     std::vector<uint32_t> slab, meta, gemm;
-    std::vector<double> strip_cost, pair_cost;  // tensor-core time: dense slab 1, 2:4 slab 1/2
+    std::vector<int> order;                     // strips by pair position: pair i = (order[2i], order[2i+1])
+    std::vector<uint32_t> pgemm, pmeta;         // gemm and meta with rows in pair-position order
+    std::vector<double> strip_cost, pair_cost;  // tensor-core time: dense slab 1, 2:4 slab 1/2 (pair_cost by pair)
+    std::vector<double> adj_pair_cost;          // the same for strips (2q, 2q+1): the row-partition estimate
     std::vector<double> strip_bytes;            // bytes the decode kernel streams per strip
     int64_t bytes = 0, sparse = 0, pair_sparse = 0, meta_blocks = 0, images = 0;
 };
+
+// Partners of the CTA-pair kernels. One pair MMA covers two strips and must
+// be dense or 2:4 for both, so a 2:4 slab whose partner's slab is dense runs
+// from a dense image at dense cost. Strips are therefore paired by agreement:
+// score(i, j) = slabs that are 2:4 in both; repeatedly pair the two unpaired
+// strips of highest score (ties: smallest i, then smallest j); pairs go in
+// the order of their first strip, an odd strip out last (its own partner).
+// If the fixed pairs (2p, 2p+1) score at least as much in total, they are
+// kept (order 0, 1, 2, ...: so strips of equal patterns, all dense or all
+// 2:4, keep it), and so does a linear of more than kMaxPairedStrips strips
+// (the scores would take S^2 / 2 entries).
+constexpr int kMaxPairedStrips = 2048;
+
+std::vector<int> pair_order(const std::vector<uint8_t>& sp, int S, int KB) {
+    if (S > kMaxPairedStrips) {
+        std::vector<int> order(S);
+        for (int s = 0; s < S; ++s) order[s] = s;
+        return order;
+    }
+    const int words = (KB + 63) / 64;
+    std::vector<uint64_t> bits((size_t)S * words, 0);
+    for (int s = 0; s < S; ++s)
+        for (int b = 0; b < KB; ++b)
+            if (sp[(size_t)s * KB + b]) bits[(size_t)s * words + b / 64] |= 1ull << (b % 64);
+    struct Cand {
+        int score, i, j;
+    };
+    std::vector<Cand> cand;
+    cand.reserve((size_t)S * (S - 1) / 2);
+    for (int i = 0; i < S; ++i)
+        for (int j = i + 1; j < S; ++j) {
+            int sc = 0;
+            for (int w = 0; w < words; ++w)
+                sc += __builtin_popcountll(bits[(size_t)i * words + w] & bits[(size_t)j * words + w]);
+            cand.push_back({sc, i, j});
+        }
+    std::sort(cand.begin(), cand.end(), [](const Cand& x, const Cand& y) {
+        return x.score != y.score ? x.score > y.score : x.i != y.i ? x.i < y.i : x.j < y.j;
+    });
+    std::vector<uint8_t> used(S, 0);
+    std::vector<std::pair<int, int>> pairs;
+    int64_t greedy = 0, fixed = 0;
+    for (const Cand& c : cand) {
+        if (used[c.i] || used[c.j]) continue;
+        used[c.i] = used[c.j] = 1;
+        pairs.push_back({c.i, c.j});
+        greedy += c.score;
+    }
+    for (int i = 0; i + 1 < S; i += 2)
+        for (int w = 0; w < words; ++w)
+            fixed += __builtin_popcountll(bits[(size_t)i * words + w] & bits[(size_t)(i + 1) * words + w]);
+    if (fixed >= greedy) {
+        std::vector<int> order(S);
+        for (int s = 0; s < S; ++s) order[s] = s;
+        return order;
+    }
+    std::sort(pairs.begin(), pairs.end());
+    std::vector<int> order;
+    order.reserve(S);
+    for (const auto& pr : pairs) {
+        order.push_back(pr.first);
+        order.push_back(pr.second);
+    }
+    for (int s = 0; s < S; ++s)
+        if (!used[s]) order.push_back(s);
+    return order;
+}
 
 // Region V (every slab), region E (a metadata block per chunk holding a 2:4
 // slab), region D (dense images of 2:4 slabs whose partner strip is dense).
@@ -182,13 +252,16 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
             sp[(size_t)s * p.KB + b] = all;
         }
     auto is_sp = [&](int s, int b) { return sp[(size_t)s * p.KB + b] != 0; };
-    auto partner = [&](int s) { return ((s ^ 1) < p.S) ? (s ^ 1) : s; };
-    auto pair_sp = [&](int s, int b) { return is_sp(s, b) && is_sp(partner(s), b); };
+    p.order = pair_order(sp, p.S, p.KB);
+    std::vector<int> partner_of(p.S);
+    for (int q = 0; q < p.S; ++q) partner_of[p.order[q]] = (q ^ 1) < p.S ? p.order[q ^ 1] : p.order[q];
+    auto pair_sp = [&](int s, int b) { return is_sp(s, b) && is_sp(partner_of[s], b); };
     p.slab.assign((size_t)p.S * p.KB, 0u);
     p.meta.assign((size_t)p.S * p.KC, kNoMeta);
     p.gemm.assign((size_t)p.S * p.KB, 0u);
     p.strip_cost.assign(p.S, 0.0);
     p.pair_cost.assign((p.S + 1) / 2, 0.0);
+    p.adj_pair_cost.assign((p.S + 1) / 2, 0.0);
     p.strip_bytes.assign(p.S, 0.0);
     int64_t off = 0;
     for (int s = 0; s < p.S; ++s)
@@ -227,8 +300,19 @@ void build_plan(Plan& p, int64_t N, int64_t K, int R, int C, const uint8_t* flag
             p.gemm[(size_t)s * p.KB + b] =
                 (uint32_t)((a_off / 16) << 2) | (first ? kSlabFirst : 0u) | (px ? kSlabSparse : 0u);
             p.pair_sparse += px;
-            if ((s & 1) == 0) p.pair_cost[s / 2] += px ? 0.5 : 1.0;
+            if ((s & 1) == 0) {
+                const int t = (s + 1) < p.S ? s + 1 : s;
+                p.adj_pair_cost[s / 2] += (x && is_sp(t, b)) ? 0.5 : 1.0;
+            }
         }
+    for (int i = 0; i < (p.S + 1) / 2; ++i)
+        for (int b = 0; b < p.KB; ++b) p.pair_cost[i] += pair_sp(p.order[2 * i], b) ? 0.5 : 1.0;
+    p.pgemm.resize(p.gemm.size());
+    p.pmeta.resize(p.meta.size());
+    for (int q = 0; q < p.S; ++q) {
+        std::copy_n(p.gemm.begin() + (size_t)p.order[q] * p.KB, p.KB, p.pgemm.begin() + (size_t)q * p.KB);
+        std::copy_n(p.meta.begin() + (size_t)p.order[q] * p.KC, p.KC, p.pmeta.begin() + (size_t)q * p.KC);
+    }
     p.bytes = off;
 }
 
@@ -263,6 +347,9 @@ struct patch_handle_s {
     Plan plan;
     uint8_t* packed = nullptr;
     uint32_t* slab_dev = nullptr;
+    int* order_dev = nullptr;
+    uint32_t* pgemm_dev = nullptr;  // the pair kernels' tables, rows in pair-position order
+    uint32_t* pmeta_dev = nullptr;
     uint32_t* meta_dev = nullptr;
     uint32_t* gemm_dev = nullptr;
     int* status_dev = nullptr;
@@ -376,6 +463,9 @@ void free_handle(patch_handle h) {
     free_group(h->self);
     cudaFree(h->packed);
     cudaFree(h->slab_dev);
+    cudaFree(h->order_dev);
+    cudaFree(h->pgemm_dev);
+    cudaFree(h->pmeta_dev);
     cudaFree(h->meta_dev);
     cudaFree(h->gemm_dev);
     cudaFree(h->status_dev);
@@ -394,6 +484,11 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     g->pure24 = true;
     for (int i = 0; i < n; ++i)
         g->pure24 = g->pure24 && hs[i]->plan.pair_sparse == (int64_t)hs[i]->plan.S * hs[i]->plan.KB;
+    // the pure instance computes record offsets from the strip index, so it
+    // also needs the pair order to be the strip order (always the case when
+    // every slab is 2:4: all pairs then agree equally and the fixed ones stay)
+    for (int i = 0; i < n && g->pure24; ++i)
+        for (int q = 0; q < hs[i]->plan.S; ++q) g->pure24 = g->pure24 && hs[i]->plan.order[q] == q;
     LinDesc d[kMaxGroup];
     // Decode units: a lone linear keeps its own split (enough units for every
     // SM); in a group the members' units already fill the GPU, so parts are
@@ -810,6 +905,19 @@ patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int til
     return PATCH_OK;
 }
 
+patch_status patch_plan_pairs(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
+                              int32_t* order) {
+    if (!tile_flags || !order) return fail(PATCH_ERR_ARG, "tile_flags and order must be non-NULL");
+    patch_status st = check_shape(N, K, tile_rows, tile_cols);
+    if (st != PATCH_OK) return st;
+    st = check_flags(tile_flags, (N / tile_rows) * (K / tile_cols));
+    if (st != PATCH_OK) return st;
+    Plan p;
+    build_plan(p, N, K, tile_rows, tile_cols, tile_flags);
+    for (int q = 0; q < p.S; ++q) order[q] = p.order[q];
+    return PATCH_OK;
+}
+
 patch_status patch_classify_tiles(const uint8_t* mask_bits, int64_t N, int64_t K, int tile_rows, int tile_cols,
                                   uint8_t* tile_flags, int64_t* dense_with_pruned) {
     if (!mask_bits || !tile_flags) return fail(PATCH_ERR_ARG, "mask_bits and tile_flags must be non-NULL");
@@ -856,7 +964,7 @@ patch_status patch_partition_rows(int64_t N, int64_t K, const uint8_t* tile_flag
     const int64_t pairs = (int64_t)p.pair_cost.size();
     const int64_t units = (pairs + per_unit - 1) / per_unit;
     std::vector<int64_t> cost((size_t)units, 0);
-    for (int64_t q = 0; q < pairs; ++q) cost[(size_t)(q / per_unit)] += (int64_t)llround(2.0 * p.pair_cost[q]) + 2;
+    for (int64_t q = 0; q < pairs; ++q) cost[(size_t)(q / per_unit)] += (int64_t)llround(2.0 * p.adj_pair_cost[q]) + 2;
     // Smallest bottleneck T that a left-to-right greedy packing fits into
     // `parts` contiguous parts (the greedy is optimal for a given T).
     auto parts_needed = [&](int64_t T) {
@@ -948,6 +1056,9 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     };
     if (cudaMalloc(&h->packed, std::max<int64_t>(p.bytes, 2048)) != cudaSuccess ||
         cudaMalloc(&h->slab_dev, sizeof(uint32_t) * p.slab.size()) != cudaSuccess ||
+        cudaMalloc(&h->order_dev, sizeof(int) * p.order.size()) != cudaSuccess ||
+        cudaMalloc(&h->pgemm_dev, sizeof(uint32_t) * p.pgemm.size()) != cudaSuccess ||
+        cudaMalloc(&h->pmeta_dev, sizeof(uint32_t) * p.pmeta.size()) != cudaSuccess ||
         cudaMalloc(&h->meta_dev, sizeof(uint32_t) * p.meta.size()) != cudaSuccess ||
         cudaMalloc(&h->gemm_dev, sizeof(uint32_t) * p.gemm.size()) != cudaSuccess ||
         cudaMalloc(&h->status_dev, sizeof(int)) != cudaSuccess ||
@@ -972,6 +1083,12 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
                              s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(h->gemm_dev, p.gemm.data(), sizeof(uint32_t) * p.gemm.size(), cudaMemcpyHostToDevice,
                              s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(h->order_dev, p.order.data(), sizeof(int) * p.order.size(), cudaMemcpyHostToDevice,
+                             s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(h->pgemm_dev, p.pgemm.data(), sizeof(uint32_t) * p.pgemm.size(),
+                             cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(h->pmeta_dev, p.pmeta.data(), sizeof(uint32_t) * p.pmeta.size(),
+                             cudaMemcpyHostToDevice, s)) != cudaSuccess ||
         (e = cudaMemcpyAsync(flags_dev, tile_flags, ntiles, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
         (e = cudaMemsetAsync(counters, 0, 3 * sizeof(unsigned long long), s)) != cudaSuccess ||
         (e = cudaMemsetAsync(h->status_dev, 0, sizeof(int), s)) != cudaSuccess)
@@ -1002,7 +1119,9 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     h->desc.packed = h->packed;
     h->desc.slab = h->slab_dev;
     h->desc.meta = h->meta_dev;
-    h->desc.gemm = h->gemm_dev;
+    h->desc.gemm = h->pgemm_dev;
+    h->desc.pmeta = h->pmeta_dev;
+    h->desc.order = h->order_dev;
     h->desc.N = (int)N;
     h->desc.S = p.S;
     h->desc.KB = p.KB;

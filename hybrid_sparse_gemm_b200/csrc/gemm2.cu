@@ -90,12 +90,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         atomicCAS(a.status, 0, kStatusTimeout);
     };
-    // strip this CTA loads for pair-unit c of a member with S strips (an odd
-    // last strip is duplicated into the second CTA and not stored)
-    auto own_strip = [&](int c, int S) {
-        int s = 2 * c + (int)pr;
-        if (s >= S) s = 2 * c;
-        return s;
+    // pair position of the strip this CTA loads for pair-unit c of member L
+    // (an odd last strip is duplicated into the second CTA and not stored);
+    // the tables L.gemm and L.pmeta have their rows in this order
+    auto own_pos = [&](const LinDesc& L, int c) {
+        const int pos = 2 * c + (int)pr;
+        return pos < L.S ? pos : 2 * c;
     };
 
     const int w_begin = a.work_off[cl];
@@ -116,9 +116,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
                 const int c = lu / a.MB, j = lu % a.MB;
-                const int s = own_strip(c, L.S);
-                const uint32_t* trow = L.gemm + (size_t)s * L.KB;
-                const uint32_t* mrow = L.meta + (size_t)s * L.KC;
+                const int pos = own_pos(L, c);
+                const uint32_t* trow = L.gemm + (size_t)pos * L.KB;
+                const uint32_t* mrow = L.pmeta + (size_t)pos * L.KC;
                 const int KB = L.KB;
                 const CUtensorMap* tm_x = &maps.x[l];
                 const CUtensorMap* tm_a16 = &maps.a16[l];
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int u = a.work[it];
                 const LinDesc& L = a.lins[u >> kUnitShift];
                 const int KB = L.KB;
-                const uint32_t* trow = L.gemm + (size_t)own_strip((u & kUnitMask) / a.MB, L.S) * KB;
+                const uint32_t* trow = L.gemm + (size_t)own_pos(L, (u & kUnitMask) / a.MB) * KB;
                 uint32_t d = trow[0];
                 const int acc = t & 1;
                 if (!mbar_wait(&acc_empty[acc], ((t >> 1) & 1) ^ 1u, abort_flag)) {
@@ -265,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const int N = a.lins[l].N;
             const int c = lu / a.MB, j = lu % a.MB;
-            const int s = 2 * c + (int)pr;
-            const bool store = s < a.lins[l].S;
+            const int pos = 2 * c + (int)pr;  // pair position of this CTA's strip
+            const bool store = pos < a.lins[l].S;
+            const int s = store ? a.lins[l].order[pos] : 0;
             const int acc = t & 1;
             if (!mbar_wait(&acc_full[acc], (t >> 1) & 1, abort_flag)) {
                 if (lane == 0) raise();

@@ -248,15 +248,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         atomicCAS(a.status, 0, kStatusTimeout);
     };
-    // Strip this CTA loads for strip pair h of quad c (S strips in the
-    // member); missing strips fall back to a strip whose partner relation is
-    // kept, so both halves of every MMA stay one kind.
-    auto strip_of = [&](int c, int h, int S) {
-        int s = 4 * c + 2 * h + (int)pr;
-        if (s >= S) s = 4 * c + 2 * h;
-        if (s >= S) s = 4 * c + (int)pr;
-        if (s >= S) s = 4 * c;
-        return s;
+    // Pair position of the strip this CTA loads for strip pair h of quad c
+    // of member L (the tables L.gemm and L.pmeta have their rows in this
+    // order; with pure 2:4 weights it is the strip order). Missing positions
+    // fall back to one whose partner relation is kept, so both halves of
+    // every MMA stay one kind.
+    auto pos_of = [&](const LinDesc& L, int c, int h) {
+        const int S = L.S;
+        int pos = 4 * c + 2 * h + (int)pr;
+        if (pos >= S) pos = 4 * c + 2 * h;
+        if (pos >= S) pos = 4 * c + (int)pr;
+        if (pos >= S) pos = 4 * c;
+        return pos;
     };
 
     const int w_begin = a.work_off[cl];
@@ -292,14 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const LinDesc& L = a.lins[l];
                 const int c = lu / a.MB, j = lu % a.MB;
                 const int KB = L.KB, KC = L.KC;
-                const int s0 = strip_of(c, 0, L.S), s1 = strip_of(c, 1, L.S);
+                const int s0 = pos_of(L, c, 0), s1 = pos_of(L, c, 1);
                 uint32_t* tab = tabs + warp * kTabWords;
                 const uint32_t *t0 = nullptr, *t1 = nullptr, *m0 = nullptr, *m1 = nullptr;
                 if (!kPure24) {
                     t0 = stage_table(tab, L.gemm + (size_t)s0 * KB, KB);
                     t1 = stage_table(tab + kTabKB, L.gemm + (size_t)s1 * KB, KB);
-                    m0 = stage_table(tab + 2 * kTabKB, L.meta + (size_t)s0 * KC, KB > kTabKB ? kTabKB + 1 : KC);
-                    m1 = stage_table(tab + 2 * kTabKB + kTabKB / 2, L.meta + (size_t)s1 * KC,
+                    m0 = stage_table(tab + 2 * kTabKB, L.pmeta + (size_t)s0 * KC, KB > kTabKB ? kTabKB + 1 : KC);
+                    m1 = stage_table(tab + 2 * kTabKB + kTabKB / 2, L.pmeta + (size_t)s1 * KC,
                                      KB > kTabKB ? kTabKB + 1 : KC);
                     __syncwarp();
                 }
@@ -465,8 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const int N = a.lins[l].N;
             const int c = lu / a.MB, j = lu % a.MB;
-            const int s = 4 * c + 2 * h + (int)pr;
-            const bool store = s < a.lins[l].S;
+            const int pos = 4 * c + 2 * h + (int)pr;  // pair position of this CTA's strip
+            const bool store = pos < a.lins[l].S;
+            const int s = store ? a.lins[l].order[pos] : 0;
             const int nt = tile_tokens(a, j);
             const int tok0 = tile_start(a, j);
             const int mrem = a.M - tok0;  // tokens of the tile that exist

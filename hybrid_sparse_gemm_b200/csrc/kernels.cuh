@@ -33,7 +33,9 @@ struct LinDesc {
     const uint8_t* packed;
     const uint32_t* slab;      // per-strip slab table
     const uint32_t* meta;      // metadata block table
-    const uint32_t* gemm;      // CTA-pair slab table
+    const uint32_t* gemm;      // CTA-pair slab table, rows in pair-position order
+    const uint32_t* pmeta;     // metadata block table, rows in pair-position order
+    const int* order;          // strips by pair position: pair i = strips order[2i], order[2i+1]
     int N, S, KB, KC, P;       // P: decode K-parts per strip
 };
 

@@ -97,7 +97,8 @@ typedef struct {
     int64_t slabs_sparse;       /* slabs stored compressed */
     int64_t slabs_pair_sparse;  /* slabs the CTA-pair kernel runs on the sparse MMA */
     int64_t meta_blocks;        /* 2048-byte metadata blocks */
-    int64_t dense_images;       /* dense images of 2:4 slabs whose partner strip is dense */
+    int64_t dense_images;       /* dense images of 2:4 slabs whose partner strip is dense
+                                   (partners: patch_plan_pairs) */
     int64_t packed_bytes;       /* device bytes of the packed weights */
     int64_t pruned;             /* mask zeros over all N*K elements */
     int64_t stray_zeros;        /* mask zeros inside tiles flagged dense */
@@ -148,6 +149,28 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
 patch_status patch_plan(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows, int tile_cols,
                         uint32_t* slab_table, uint32_t* meta_table, uint32_t* gemm_table,
                         int64_t* packed_bytes);
+
+/*
+ * patch_plan_pairs - which strips patch_pack makes partners for the CTA-pair
+ * kernels, computed on the host without touching any device.
+ *
+ * The pages fix no kernel; this is the packed format's own rule. A CTA-pair
+ * MMA covers two 128-row strips and is either dense or 2:4 for both, so a
+ * 2:4 slab whose partner's slab is dense runs from a dense image at dense
+ * cost (the tiles' dense / 2:4 choices are learned independently: abstract of
+ * "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs"). Strips are paired
+ * by agreement: score(i, j) = number of 64-column slabs 2:4 in both strips;
+ * the two unpaired strips of highest score are paired first (ties: smallest
+ * i, then smallest j); pairs are listed in the order of their first strip and
+ * an odd strip out comes last as its own partner. Linears of more than 2048
+ * strips keep the order 0, 1, 2, ...
+ *
+ *   N, K, tile_flags, tile_rows, tile_cols  as for patch_pack.
+ *   order       host, N/128 int32: pair i is strips order[2i], order[2i+1].
+ * Same shape rules and errors as patch_plan.
+ */
+patch_status patch_plan_pairs(int64_t N, int64_t K, const uint8_t* tile_flags, int tile_rows,
+                              int tile_cols, int32_t* order);
 
 /*
  * patch_classify_tiles - the tile flags a keep/prune mask implies, computed
@@ -357,8 +380,9 @@ patch_status patch_info(patch_handle h, patch_info_t* info);
  *   meta[s*KC+c] = offset/16 of the chunk's 2048-byte metadata block, or
  *     0xFFFFFFFF when the chunk has no 2:4 slab.
  *   gemm[s*KB+b] = (offset/16)<<2 | first<<1 | pair_sparse: the record the
- *     CTA-pair kernel loads (strips 2p and 2p+1 agree on every slab; a 2:4
- *     slab whose partner is dense points at its dense image).
+ *     CTA-pair kernels load (a strip and its partner, patch_plan_pairs, agree
+ *     on every slab; a 2:4 slab whose partner's slab is dense points at its
+ *     dense image).
  * Synchronous.
  */
 patch_status patch_copy_packed(patch_handle h, void* packed_host, int64_t packed_cap,

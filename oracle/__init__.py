@@ -58,6 +58,8 @@ def _load():
         lib.oracle_abs_scale.argtypes = [P, I64, P, I64, P, I64, P]
         lib.oracle_pack_table.argtypes = [I64, I64, P, I, I, P, P, P]
         lib.oracle_pack_table.restype = I64
+        lib.oracle_pair_order.argtypes = [I64, I64, P, I, I, P]
+        lib.oracle_pair_order.restype = I
         lib.oracle_pack.argtypes = [P, P, I64, I64, P, P, P, P]
         lib.oracle_pack.restype = I
         lib.oracle_unpack.argtypes = [P, P, P, I64, I64, P]
@@ -191,7 +193,18 @@ def pack_table(N: int, K: int, flags, R: int, C: int) -> Tables:
     meta = np.empty((N // 128) * KC, np.uint32)
     gemm = np.empty((N // 128) * KB, np.uint32)
     total = _load().oracle_pack_table(N, K, _p(flags), R, C, _p(slab), _p(meta), _p(gemm))
+    if total < 0:
+        raise MemoryError("oracle_pack_table: out of memory")
     return Tables(slab, meta, gemm, int(total))
+
+
+def pair_order(N: int, K: int, flags, R: int, C: int) -> np.ndarray:
+    """Strip order of the CTA-pair view: pair i is strips order[2i], order[2i+1]."""
+    flags = np.ascontiguousarray(flags, dtype=np.uint8).reshape(-1)
+    order = np.empty(max(N // 128, 1), np.int32)
+    if _load().oracle_pair_order(N, K, _p(flags), R, C, _p(order)) != 0:
+        raise MemoryError("oracle_pair_order: out of memory")
+    return order[:N // 128]
 
 
 def pack(W, keep: np.ndarray, flags: np.ndarray, R: int, C: int):

@@ -32,11 +32,19 @@
  * The packed format is this library's own (the pages give none). Its
  * independent restatement here lets tests check the GPU pack byte by byte:
  *   - A "strip" is 128 consecutive rows of W, a "slab" a strip times 64
- *     consecutive columns, a "chunk" two slabs (128 columns). Strips s and
- *     s^1 are partners (the last strip of an odd count is its own partner).
+ *     consecutive columns, a "chunk" two slabs (128 columns).
  *   - A slab is sparse when every mask tile it overlaps is flagged 2:4,
- *     otherwise dense; a slab is pair-sparse when it and its partner's slab
- *     are both sparse.
+ *     otherwise dense.
+ *   - Partners: the agreement of strips i and j is the number of slabs sparse
+ *     in both. Among strips not yet paired, the two of greatest agreement
+ *     become partners (ties: smallest i, then smallest j), until fewer than
+ *     two remain; a strip left over is its own partner. Strips 2p and 2p+1
+ *     are partners instead (the last of an odd count its own) when these
+ *     pairs' agreements add up to at least those of the pairs chosen, or
+ *     when there are more than 2048 strips. The pair order lists
+ *     each pair's two strips (smaller first) in increasing order of its
+ *     smaller strip, then the strip left over.
+ *   - A slab is pair-sparse when it and its partner's slab are both sparse.
  *   - Region V, strip-major then slab: a dense slab is 16384 bytes, element
  *     (r, c) of W' (r < 128, c < 64) at byte r*128 + ((c/8) ^ (r%8))*16 +
  *     (c%8)*2; a sparse slab is 8192 bytes of the two kept bf16 of each
@@ -189,17 +197,83 @@ static int or_slab_sparse(const uint8_t* flags, int64_t K, int R, int C, int64_t
     return 1;
 }
 
-static int or_pair_sparse(const uint8_t* flags, int64_t N, int64_t K, int R, int C, int64_t s,
-                          int64_t b) {
-    int64_t S = N / OR_STRIP;
-    int64_t partner = ((s ^ 1) < S) ? (s ^ 1) : s;
-    return or_slab_sparse(flags, K, R, C, s, b) && or_slab_sparse(flags, K, R, C, partner, b);
+static int64_t or_agreement(const uint8_t* flags, int64_t K, int R, int C, int64_t i, int64_t j) {
+    int64_t agree = 0;
+    for (int64_t b = 0; b < K / OR_SLAB; ++b)
+        agree += or_slab_sparse(flags, K, R, C, i, b) && or_slab_sparse(flags, K, R, C, j, b);
+    return agree;
 }
 
-/* Fills the three tables and returns the total packed byte count. */
+/* partner[s] of every strip, by the rule above; returns 0. */
+static int or_partners(const uint8_t* flags, int64_t N, int64_t K, int R, int C, int64_t* partner) {
+    int64_t S = N / OR_STRIP, chosen = 0, fixed = 0;
+    for (int64_t s = 0; s + 1 < S; s += 2) fixed += or_agreement(flags, K, R, C, s, s + 1);
+    for (int64_t s = 0; s < S; ++s) partner[s] = -1;
+    for (;;) {
+        int64_t bi = -1, bj = -1, best = -1;
+        for (int64_t i = 0; i < S; ++i) {
+            if (partner[i] >= 0) continue;
+            for (int64_t j = i + 1; j < S && S <= 2048; ++j) {
+                if (partner[j] >= 0) continue;
+                int64_t agree = or_agreement(flags, K, R, C, i, j);
+                if (agree > best) { /* strictly greater: the first (i, j) wins a tie */
+                    best = agree;
+                    bi = i;
+                    bj = j;
+                }
+            }
+        }
+        if (bi < 0) break;
+        partner[bi] = bj;
+        partner[bj] = bi;
+        chosen += best;
+    }
+    if (S > 2048 || fixed >= chosen)
+        for (int64_t s = 0; s < S; ++s) partner[s] = -1;
+    for (int64_t s = 0; s + 1 < S; s += 2)
+        if (partner[s] < 0 && partner[s + 1] < 0) {
+            partner[s] = s + 1;
+            partner[s + 1] = s;
+        }
+    for (int64_t s = 0; s < S; ++s)
+        if (partner[s] < 0) partner[s] = s;
+    return 0;
+}
+
+/* The pair order: pair i is order[2i], order[2i+1]. Returns 0 or -1. */
+int oracle_pair_order(int64_t N, int64_t K, const uint8_t* flags, int R, int C, int32_t* order) {
+    int64_t S = N / OR_STRIP, n = 0;
+    int64_t* partner = (int64_t*)malloc(sizeof(int64_t) * (size_t)(S > 0 ? S : 1));
+    if (!partner || or_partners(flags, N, K, R, C, partner) != 0) {
+        free(partner);
+        return -1;
+    }
+    for (int64_t s = 0; s < S; ++s)
+        if (partner[s] > s) {
+            order[n++] = (int32_t)s;
+            order[n++] = (int32_t)partner[s];
+        }
+    for (int64_t s = 0; s < S; ++s)
+        if (partner[s] == s) order[n++] = (int32_t)s;
+    free(partner);
+    return 0;
+}
+
+static int or_pair_sparse(const uint8_t* flags, int64_t K, int R, int C, const int64_t* partner,
+                          int64_t s, int64_t b) {
+    return or_slab_sparse(flags, K, R, C, s, b) && or_slab_sparse(flags, K, R, C, partner[s], b);
+}
+
+/* Fills the three tables and returns the total packed byte count (-1 when
+ * out of memory). */
 int64_t oracle_pack_table(int64_t N, int64_t K, const uint8_t* flags, int R, int C,
                           uint32_t* slab, uint32_t* meta, uint32_t* gemm) {
     int64_t S = N / OR_STRIP, KB = K / OR_SLAB, KC = (KB + 1) / 2, off = 0;
+    int64_t* partner = (int64_t*)malloc(sizeof(int64_t) * (size_t)(S > 0 ? S : 1));
+    if (!partner || or_partners(flags, N, K, R, C, partner) != 0) {
+        free(partner);
+        return -1;
+    }
     /* region V */
     for (int64_t s = 0; s < S; ++s)
         for (int64_t b = 0; b < KB; ++b) {
@@ -225,7 +299,7 @@ int64_t oracle_pack_table(int64_t N, int64_t K, const uint8_t* flags, int R, int
     for (int64_t s = 0; s < S; ++s)
         for (int64_t b = 0; b < KB; ++b) {
             int sp = or_slab_sparse(flags, K, R, C, s, b);
-            int psp = or_pair_sparse(flags, N, K, R, C, s, b);
+            int psp = or_pair_sparse(flags, K, R, C, partner, s, b);
             int64_t a_off;
             if (sp && !psp) {
                 a_off = off;
@@ -233,10 +307,11 @@ int64_t oracle_pack_table(int64_t N, int64_t K, const uint8_t* flags, int R, int
             } else {
                 a_off = (int64_t)(slab[s * KB + b] >> 2) * 16;
             }
-            int load_meta = psp && (b % 2 == 0 || !or_pair_sparse(flags, N, K, R, C, s, b - 1));
+            int load_meta = psp && (b % 2 == 0 || !or_pair_sparse(flags, K, R, C, partner, s, b - 1));
             gemm[s * KB + b] = (uint32_t)((a_off / 16) << 2) | (uint32_t)(load_meta << 1) |
                                (uint32_t)psp;
         }
+    free(partner);
     return off;
 }
 

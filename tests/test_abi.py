@@ -105,6 +105,21 @@ def test_plan_matches_oracle_tables(hsg, oracle_lib, R, C, N, K, frac):
     assert np.array_equal(gemm, t.gemm)
 
 
+@pytest.mark.parametrize("R,C", [(128, 128), (64, 64)])
+@pytest.mark.parametrize("N,K,frac,seed", [(1152, 1024, 0.9, 1), (1280, 512, 0.7, 2), (896, 768, 0.5, 3),
+                                           (11008, 4096, 0.9, 4), (4096, 4096, 0.6, 5), (640, 256, 1.0, 6),
+                                           (384, 2048, 0.0, 7)])
+def test_plan_pairs_match_oracle(hsg, oracle_lib, R, C, N, K, frac, seed):
+    """The strip pairing of the CTA-pair kernels equals the oracle's
+    restatement, and the tables built on it too."""
+    flags = synth.tile_flags(N, K, R, C, frac, "pairs", seed).numpy().reshape(-1)
+    order = hsg.patch_plan_pairs(N, K, flags, R, C)
+    assert np.array_equal(order, oracle_lib.pair_order(N, K, flags, R, C))
+    (slab, meta, gemm), nbytes = hsg.patch_plan(N, K, flags, R, C)
+    t = oracle_lib.pack_table(N, K, flags, R, C)
+    assert nbytes == t.nbytes and np.array_equal(gemm, t.gemm)
+
+
 def test_plan_checkerboard_and_llama_sizes(hsg, oracle_lib):
     # checkerboard of 64x64 tiles: no 128x64 slab is all-2:4, so nothing compresses
     N, K = 256, 256
@@ -124,6 +139,9 @@ def test_plan_errors(hsg):
     with pytest.raises(hsg.PatchError) as e:
         hsg.patch_plan(256, 256, np.full(4, 3, np.uint8), 128, 128)
     assert e.value.status == 1
+    with pytest.raises(hsg.PatchError) as e:
+        hsg.patch_plan_pairs(256, 256, np.zeros(4, np.uint8), 128, 96)
+    assert e.value.status == 2
 
 
 def test_group_and_noalloc_reject_bad_arguments(hsg):

@@ -263,6 +263,32 @@ def test_wide_tables_beyond_shared_copy(hsg, oracle_lib, frac):
     lin.free()
 
 
+def test_large_m_and_wide_n(hsg, oracle_lib):
+    """Maximum-size cases on small weights: 100003 tokens (hundreds of token
+    tiles, ragged last tile, Y beyond 2^26 elements) through every large-M
+    kernel, and a 28672-row linear (224 strips) on the decode and automatic
+    paths; sampled rows (first and last included) against the oracle."""
+    p = synth.make_problem(512, 256, 100003, R=128, C=128, frac=0.7, seed=41, device="cuda", tag="bigM")
+    lin = pack(hsg, p)
+    rows = sample_rows(p.X.shape[0], 96, 41)
+    for path in (hsg.PATH_GEMM_WIDE, hsg.PATH_GEMM_PAIR, hsg.PATH_GEMM_SINGLE, hsg.PATH_AUTO):
+        Y = lin(p.X, path=path)
+        torch.cuda.synchronize()
+        lin.check()
+        assert_close(Y, oracle_lib, p.X, p.W, p.bits, p.keep, rows=rows, what=f"M=100003 path {path}")
+        del Y
+    lin.free()
+    q = synth.make_problem(28672, 256, 300, R=128, C=64, frac=0.5, seed=42, device="cuda", tag="bigN")
+    lin = pack(hsg, q)
+    for path, M in ((hsg.PATH_GEMV, 37), (hsg.PATH_GEMV, 3), (hsg.PATH_AUTO, 300)):
+        X = q.X[:M].contiguous()
+        Y = lin(X, path=path)
+        torch.cuda.synchronize()
+        lin.check()
+        assert_close(Y, oracle_lib, X, q.W, q.bits, q.keep, what=f"N=28672 path {path} M={M}")
+    lin.free()
+
+
 def test_single_strip_single_slab(hsg, oracle_lib):
     for frac in (0.0, 1.0):
         p = synth.make_problem(128, 64, 9, R=128, C=64, frac=frac, seed=3, device="cuda")

@@ -249,9 +249,14 @@ def test_pack_roundtrip(oracle_lib, R, C, N):
         rows = range(s * 128 // R, (s + 1) * 128 // R)
         return all(fl[r, (b * 64) // C] for r in rows)
 
+    order = oracle_lib.pair_order(N, K, flags, R, C)
+    partner_of = {}
+    for i in range(0, S, 2):
+        a, b2 = order[i], order[i + 1] if i + 1 < S else order[i]
+        partner_of[a], partner_of[b2] = b2, a
     n_shadow = 0
     for s in range(S):
-        partner = s ^ 1 if (s ^ 1) < S else s
+        partner = partner_of[s]
         for b in range(KB):
             sp = sparse(s, b)
             psp = sp and sparse(partner, b)
@@ -297,6 +302,81 @@ def test_pack_metadata_codes_and_sizes(oracle_lib):
     # every kept value appears in the compressed values
     vals = np.concatenate([packed[int(x >> 2) * 16:][:8192].view(np.uint16) for x in t.slab])
     assert sorted(vals.tolist()) == sorted(bits_of(W)[keep.astype(bool)].tolist())
+
+
+def _flags_from_slabs(rows):
+    """Tile flags for 128 x 64 tiles from per-strip strings of slab kinds."""
+    return np.array([[int(c) for c in r] for r in rows], np.uint8)
+
+
+def _agreement(fl, i, j):
+    return int((fl[i] & fl[j]).sum())
+
+
+def test_pair_order_hand_cases(oracle_lib):
+    """The pairing rule of the CTA-pair view on cases whose answer is fixed by
+    the rule's statement: strips of matching patterns pair up; ties go to the
+    smallest indices; fixed pairs (2p, 2p+1) are kept when they agree at
+    least as much in total; an odd strip out comes last."""
+    def order(rows):
+        fl = _flags_from_slabs(rows)
+        S, KB = fl.shape
+        return oracle_lib.pair_order(128 * S, 64 * KB, fl.reshape(-1), 128, 64).tolist()
+    assert order(["1100", "0011", "1100", "0011"]) == [0, 2, 1, 3]
+    assert order(["1111", "0000", "1111"]) == [0, 2, 1]
+    assert order(["1111"] * 5) == [0, 1, 2, 3, 4]
+    assert order(["0000"] * 4) == [0, 1, 2, 3]
+    # three strips agree equally: the first two pair (ties), then 2 with 3;
+    # the fixed pairs agree as much in total, so they stay
+    assert order(["1010", "1010", "1010", "0101"]) == [0, 1, 2, 3]
+    # greedy would pair (1, 2) (11 slabs) and leave (0, 3) with none; the fixed
+    # pairs agree on 10 + 10 and are kept
+    s0 = "0" * 11 + "1" * 10 + "0" * 11
+    s1 = "1" * 21 + "0" * 11
+    s2 = "1" * 11 + "0" * 10 + "1" * 10 + "0"
+    s3 = "0" * 21 + "1" * 10 + "0"
+    fl = _flags_from_slabs([s0, s1, s2, s3])
+    assert (_agreement(fl, 0, 1), _agreement(fl, 2, 3), _agreement(fl, 1, 2)) == (10, 10, 11)
+    assert order([s0, s1, s2, s3]) == [0, 1, 2, 3]
+    # the same strips with one more slab shared by 0 and 3: greedy's 11 + 1
+    # still loses to 10 + 10; with 0 and 3 sharing 10, greedy wins 11 + 10
+    s0b = "0" * 11 + "1" * 10 + "1" * 10 + "0"
+    assert order([s0b, s1, s2, s3]) == [0, 3, 1, 2]
+
+
+def _best_matching(fl):
+    """Maximum total agreement over all pairings (brute force, small S)."""
+    S = fl.shape[0]
+
+    def go(rest):
+        if len(rest) < 2:
+            return 0
+        a, best = rest[0], 0
+        for k in range(1, len(rest)):
+            best = max(best, _agreement(fl, a, rest[k]) + go(rest[1:k] + rest[k + 1:]))
+        if len(rest) % 2:
+            best = max(best, go(rest[1:]))
+        return best
+    return go(list(range(S)))
+
+
+@pytest.mark.parametrize("S,KB,p,seed", [(4, 8, 0.8, 0), (5, 16, 0.9, 1), (6, 12, 0.5, 2), (7, 20, 0.7, 3),
+                                         (8, 24, 0.9, 4), (8, 6, 0.3, 5)])
+def test_pair_order_bounds(oracle_lib, S, KB, p, seed):
+    """On random slab patterns the pair order is a valid pairing whose total
+    agreement is at least that of the fixed pairs and at least half the best
+    pairing's (the greedy bound), checked against a brute-force optimum."""
+    g = np.random.default_rng(seed)
+    fl = (g.random((S, KB)) < p).astype(np.uint8)
+    order = oracle_lib.pair_order(128 * S, 64 * KB, fl.reshape(-1), 128, 64).tolist()
+    assert sorted(order) == list(range(S))
+    pairs = [(order[i], order[i + 1]) for i in range(0, S - 1, 2)]
+    total = sum(_agreement(fl, a, b) for a, b in pairs)
+    fixed = sum(_agreement(fl, i, i + 1) for i in range(0, S - 1, 2))
+    assert total >= fixed
+    assert 2 * total >= _best_matching(fl)
+    assert all(a < b for a, b in pairs)
+    assert [a for a, _ in pairs] == sorted(a for a, _ in pairs) or total == fixed
 
 
 def test_pair_rule_dense_images(oracle_lib):
