@@ -11,7 +11,9 @@ namespace patch {
 
 // ---- packed weight format --------------------------------------------------
 // A strip is 128 rows of W, a slab is a strip times 64 columns, a chunk two
-// slabs. Strips 2p and 2p+1 are partners (an odd last strip is its own).
+// slabs. The CTA-pair kernels run two partner strips per MMA; partners are
+// chosen when the plan is built (pairs of strips that share the most 2:4
+// slabs; an odd strip out is its own partner).
 // Region V holds every slab, strip-major with K ascending: a dense slab is the
 // 128x64 bf16 block in the 128-byte-swizzled K-major layout the tensor core
 // reads; a sparse slab is 128x32 kept values in the 64-byte-swizzled layout.

@@ -18,11 +18,11 @@
 // 248. The accumulators are single-buffered: a tile's MMAs start once the
 // previous tile has been drained, while the producers keep filling the ring.
 //
-// Partner strips (2p, 2p+1) load the same kind of record at every slab (the
-// packed format's dense images stand in for 2:4 slabs whose partner is
-// dense), so one MMA instruction always covers both halves of a pair. Strips
-// past the end of the weight are replaced by duplicates whose results are not
-// stored.
+// Partner strips (the strips at pair positions 2p and 2p+1 of the member's
+// pair order) load the same kind of record at every slab (the packed
+// format's dense images stand in for 2:4 slabs whose partner is dense), so
+// one MMA instruction always covers both halves of a pair. Positions past the
+// end of the weight are replaced by duplicates whose results are not stored.
 #include "kernels.cuh"
 #include "pair.cuh"
 
