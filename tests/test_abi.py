@@ -144,6 +144,17 @@ def test_plan_errors(hsg):
     assert e.value.status == 2
 
 
+@pytest.mark.parametrize("S", [2048, 2049])
+def test_plan_pairs_size_limit(hsg, oracle_lib, S):
+    """Up to 2048 strips the pairing follows agreement; above, the fixed
+    pairs stay (both sides of the limit, against the oracle)."""
+    g = np.random.default_rng(S)
+    flags = (g.random((S, 2)) < 0.5).astype(np.uint8).reshape(-1)
+    order = hsg.patch_plan_pairs(128 * S, 128, flags, 128, 64)
+    assert np.array_equal(order, oracle_lib.pair_order(128 * S, 128, flags, 128, 64))
+    assert np.array_equal(order, np.arange(S)) == (S > 2048)
+
+
 def test_group_and_noalloc_reject_bad_arguments(hsg):
     lib = hsg.library()
     g = ctypes.c_void_p()
