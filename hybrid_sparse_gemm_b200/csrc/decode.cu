@@ -269,8 +269,9 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             }
             tc_fence_after();
             __nv_bfloat16* yc = a.Y[l] + (size_t)s * kStrip + row;
-            // this unit's partial, workspace[s][p][token][row]: a warp's
-            // stores and loads of one token cover 128 contiguous bytes
+            // this unit's partial, workspace[s][p][token][row], for the M
+            // tokens only: a warp's stores and loads of one token cover 128
+            // contiguous bytes
             float* dst = P > 1 ? a.partial[l] + ((size_t)s * P + p) * kBN * 128 + row : nullptr;
             const int cols = n_tok;
             // 16 columns at a time: Y directly when the strip is one unit,
@@ -287,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                         if (c0 + c < a.M) yc[(size_t)(c0 + c) * L.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) __stcg(dst + (c0 + c) * 128, __uint_as_float(v[c]));
+                    for (int c = 0; c < 16; ++c)
+                        if (c0 + c < a.M) __stcg(dst + (c0 + c) * 128, __uint_as_float(v[c]));
                 }
             }
             tc_fence_before();
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                     for (int pp = 0; pp < P; ++pp, src += kBN * 128) {
                         float v[kRed];
 #pragma unroll
-                        for (int c = 0; c < kRed; ++c) v[c] = c0 + c < cols ? __ldcg(src + c * 128) : 0.f;
+                        for (int c = 0; c < kRed; ++c) v[c] = c0 + c < a.M ? __ldcg(src + c * 128) : 0.f;
 #pragma unroll
                         for (int c = 0; c < kRed; ++c) sum[c] += v[c];
                     }
