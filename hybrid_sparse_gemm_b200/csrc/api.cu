@@ -23,6 +23,12 @@
 
 using namespace patch;
 
+// Smallest K-part (packed bytes) of the decode kernel's 64-token instance in
+// a group (a macro so that other sizes can be measured).
+#ifndef PATCH_DECODE_WIDE_PART_KB
+#define PATCH_DECODE_WIDE_PART_KB 512.0
+#endif
+
 namespace {
 
 thread_local std::string g_err;
@@ -373,6 +379,7 @@ struct patch_group_s {
     int n = 0;
     patch_handle h[kMaxGroup] = {};
     int parts[kMaxGroup] = {};    // decode K-parts per strip of each member in this group
+    int parts_w[kMaxGroup] = {};  // the same for the decode kernel's 64-token instance
     LinDesc* lins_dev = nullptr;  // n descriptors
     int* status_dev = nullptr;    // the first member's status word
     bool pure24 = false;          // every slab of every member runs on the sparse MMA
@@ -497,20 +504,38 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
     for (int i = 0; i < n; ++i)
         for (double b : hs[i]->plan.strip_bytes) total += b;
     const double target = std::max(256.0 * 1024.0, total / (4.0 * kDecodeCtasPerSm * g->dev.sms));
+    // the 64-token instance writes and sums four times the partial bytes per
+    // part, so its parts are larger (a 4096-column strip is then one part;
+    // on Llama-2-7B layers at M = 64, 78 % of HBM instead of 68 %)
+    const double target_w =
+        std::max(PATCH_DECODE_WIDE_PART_KB * 1024.0, total / (4.0 * kDecodeWideCtasPerSm * g->dev.sms));
     for (int i = 0; i < n; ++i) {
         g->h[i] = hs[i];
         d[i] = hs[i]->desc;
-        int P = hs[i]->decode_parts;
+        int P = hs[i]->decode_parts, PW = P;
         if (n > 1) {
             const Plan& pl = hs[i]->plan;
             double avg = 0.0;
             for (double b : pl.strip_bytes) avg += b;
             avg /= std::max(1, pl.S);
             P = std::max(1, std::min(hs[i]->decode_parts, (int)(avg / target + 0.5)));
+            PW = std::max(1, std::min(hs[i]->decode_parts, (int)(avg / target_w + 0.5)));
         }
         g->parts[i] = P;
+        g->parts_w[i] = PW;
         d[i].P = P;
+        d[i].PW = PW;
     }
+    // Larger parts leave fewer units: keep them only while the group still
+    // has about 2.5 units per SM (below that, SMs run one or two issue loops
+    // and the stream slows more than the partial sums cost).
+    int64_t units_w = 0;
+    for (int i = 0; i < n; ++i) units_w += (int64_t)hs[i]->plan.S * g->parts_w[i];
+    if (units_w * 2 < 5 * (int64_t)g->dev.sms)
+        for (int i = 0; i < n; ++i) {
+            g->parts_w[i] = g->parts[i];
+            d[i].PW = d[i].P;
+        }
     if (cudaMalloc(&g->lins_dev, sizeof(LinDesc) * n) != cudaSuccess) {
         cudaGetLastError();
         delete g;
@@ -540,8 +565,8 @@ patch_status make_group(const patch_handle* hs, int n, patch_group* out) {
 // until the group is destroyed, so captured graphs may keep their address).
 patch_status ensure_wide_ws(patch_group g, DecodeWs* w) {
     for (int i = 0; i < g->n; ++i) {
-        if (g->parts[i] <= 1 || w->partial_wide[i]) continue;
-        if (cudaMalloc(&w->partial_wide[i], sizeof(float) * (size_t)w->S[i] * g->parts[i] * 128 * kDecodeWideBN) !=
+        if (g->parts_w[i] <= 1 || w->partial_wide[i]) continue;
+        if (cudaMalloc(&w->partial_wide[i], sizeof(float) * (size_t)w->S[i] * g->parts_w[i] * 128 * kDecodeWideBN) !=
             cudaSuccess) {
             cudaGetLastError();
             w->partial_wide[i] = nullptr;
@@ -639,7 +664,7 @@ void lpt_schedule(patch_group g, int kernel, int mb, std::vector<int>& off, std:
                 for (int j = 0; j < mb; ++j) units.push_back({cost + 2.0, (l << kUnitShift) | (r * mb + j)});
             }
         } else {
-            const int P = g->parts[l];
+            const int P = kernel == 5 ? g->parts_w[l] : g->parts[l];
             for (int s = 0; s < p.S; ++s)
                 for (int q = 0; q < P; ++q)
                     units.push_back({p.strip_bytes[s] / P + 16384.0, (l << kUnitShift) | (s * P + q)});
@@ -1127,6 +1152,7 @@ patch_status patch_pack(const void* W_bf16, int64_t N, int64_t K, const uint8_t*
     h->desc.KB = p.KB;
     h->desc.KC = p.KC;
     h->desc.P = h->decode_parts;
+    h->desc.PW = h->decode_parts;
     patch_handle self[1] = {h};
     if ((st = make_group(self, 1, &h->self)) != PATCH_OK) return cleanup(st);
     patch_info_t& info = h->info;

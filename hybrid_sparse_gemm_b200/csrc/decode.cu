@@ -108,8 +108,9 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     const int w_end = a.work_off[blockIdx.x + 1];
     // part p of a strip covers chunks [p*KC/P, (p+1)*KC/P), i.e. slabs from 2x that
     auto part_range = [](const LinDesc& L, int p, int& b0, int& b1) {
-        b0 = 2 * (int)(((int64_t)p * L.KC) / L.P);
-        b1 = min(L.KB, 2 * (int)(((int64_t)(p + 1) * L.KC) / L.P));
+        const int P = BN == kDecodeBN ? L.P : L.PW;
+        b0 = 2 * (int)(((int64_t)p * L.KC) / P);
+        b1 = min(L.KB, 2 * (int)(((int64_t)(p + 1) * L.KC) / P));
     };
 
     if (warp == 0) {
@@ -123,7 +124,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
-                const int s = lu / L.P, p = lu % L.P;
+                const int P = BN == kDecodeBN ? L.P : L.PW;
+                const int s = lu / P, p = lu % P;
                 int b0, b1;
                 part_range(L, p, b0, b1);
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
@@ -183,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
                 const int u = a.work[it];
                 const int l = u >> kUnitShift, lu = u & kUnitMask;
                 const LinDesc& L = a.lins[l];
-                const int s = lu / L.P, p = lu % L.P;
+                const int P = BN == kDecodeBN ? L.P : L.PW;
+                const int s = lu / P, p = lu % P;
                 int b0, b1;
                 part_range(L, p, b0, b1);
                 const uint32_t* trow = L.slab + (size_t)s * L.KB;
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
             const int u = a.work[it];
             const int l = u >> kUnitShift, lu = u & kUnitMask;
             const LinDesc& L = a.lins[l];
-            const int P = L.P;
+            const int P = BN == kDecodeBN ? L.P : L.PW;
             const int s = lu / P, p = lu % P;
             if (!mbar_wait(&acc_full[acc], (t / ACCS) & 1, abort_flag)) {
                 if (lane == 0) raise();

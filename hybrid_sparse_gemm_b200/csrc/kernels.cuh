@@ -36,7 +36,8 @@ struct LinDesc {
     const uint32_t* gemm;      // CTA-pair slab table, rows in pair-position order
     const uint32_t* pmeta;     // metadata block table, rows in pair-position order
     const int* order;          // strips by pair position: pair i = strips order[2i], order[2i+1]
-    int N, S, KB, KC, P;       // P: decode K-parts per strip
+    int N, S, KB, KC, P;       // P: decode K-parts per strip (16-token instance)
+    int PW;                    // decode K-parts per strip of the 64-token instance
 };
 
 // Tensor maps: X of every member (per call) and the packed bytes of every
