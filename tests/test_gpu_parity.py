@@ -413,7 +413,7 @@ def test_first_call_schedule_used_from_another_stream(hsg, oracle_lib):
     lin.free()
 
 
-@pytest.mark.parametrize("M", [5, 300, 1000, 2048])
+@pytest.mark.parametrize("M", [5, 40, 100, 300, 1000, 2048])
 def test_group_host_matches_device(hsg, M):
     """patch_group_linear_host (token chunks whose copies overlap the product)
     gives the device call's bits; members sharing a host input (q, k, v) and
